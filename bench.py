@@ -1,0 +1,687 @@
+#!/usr/bin/env python
+"""Benchmark: Q8_0 decode tokens/s and effective weight GB/s on B200.
+
+Default workload: one single-token decode step of the Llama-2-110M-shaped Q8_0
+matvec set (12 layers x {wq, wk, wv, wo 768x768, w1, w3 2048x768, w2 768x2048}
++ classifier 32000x768, 85 matvecs, batch 1), the Q8_0 int8 decode that the
+"narray-llm" README measures.  Every matvec gets its own seeded N(0,1) x and
+the set runs as one step: one q8_gemv_batched launch (each problem quantizes
+its x to Q8_0 inside the kernel, then streams its weights).
+
+Other workloads (--workload): gemv_768, dense_ffn (--tokens 1|8),
+moe_layer (--tokens 1|16), moe_30layer (--tokens 1|4|16|64|256).
+
+Contract: ``python bench.py --gpus N --steps K --warmup W [--impl reference]``;
+for N > 1 it is launched under torch.distributed.run, one rank per GPU, each
+rank an independent replica of the step (weak scaling; the path has no
+cross-GPU exchange).  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+Q8_BLOCK_BYTES = 34  # per 32 weights
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama2_110m_q8_decode",
+                    choices=["llama2_110m_q8_decode", "gemv_768", "dense_ffn", "moe_layer",
+                             "moe_30layer"])
+    ap.add_argument("--tokens", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="bound on the CPU baseline sample")
+    return ap.parse_args()
+
+
+def q8_bytes(rows, k):
+    return rows * k // 32 * Q8_BLOCK_BYTES
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend):
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        import torch
+        t = torch.tensor([v], dtype=torch.float64,
+                         device="cuda" if torch.cuda.is_available() else "cpu")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+REASON_FIELDS = ["clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+                 "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        q = "clocks.sm,clocks.max.sm,power.draw," + ",".join(REASON_FIELDS)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thr = threading.Thread(target=self._read, daemon=True)
+        self.thr.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thr.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 3 + len(names):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# in-graph event marks around the dominant kernel's launches
+# ---------------------------------------------------------------------------
+class Marks:
+    """Records timing events as nodes of the graph being captured (external
+    event records), so each replay times the marked launches on the device.
+    The events are created (recorded once) before the capture starts."""
+
+    def __init__(self, n_pairs: int):
+        import torch
+        self.events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(n_pairs)]
+        for a, b in self.events:
+            a.record()
+            b.record()
+        self.used = 0
+
+    @staticmethod
+    def _rec(ev):
+        import torch
+        from cuda.bindings import runtime as rt
+        err = rt.cudaEventRecordWithFlags(rt.cudaEvent_t(ev.cuda_event),
+                                          rt.cudaStream_t(torch.cuda.current_stream().cuda_stream),
+                                          rt.cudaEventRecordExternal)
+        if int(err[0]) != 0:
+            raise RuntimeError(f"cudaEventRecordWithFlags: {err}")
+
+    def begin(self):
+        self._rec(self.events[self.used][0])
+
+    def end(self):
+        self._rec(self.events[self.used][1])
+        self.used += 1
+
+    def ms(self):
+        return [a.elapsed_time(b) for a, b in self.events[:self.used]]
+
+
+class NoMarks:
+    def begin(self):
+        pass
+
+    def end(self):
+        pass
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+class LlamaDecode:
+    """85 Q8_0 matvecs of one Llama-2-110M-shaped decode step, one batched launch."""
+    name = "llama2_110m_q8_decode"
+    kernel = "gemv_batched_kernel"
+
+    def __init__(self, dev, tokens=None, gemv768=False):
+        import torch
+
+        from moe_up_gate_b200 import q8, synth
+        self.q8 = q8
+        self.dev = dev
+        if gemv768:
+            self.name = "gemv_768"
+            mats = [("w", 768, 768)]
+            seeds = [(synth.seed_of(1, 0, 0), synth.seed_of(1, 0, 1))]
+        else:
+            mats = synth.llama_matvec_set()
+            seeds = []
+            for i, (nm, rows, k) in enumerate(mats):
+                layer, j = (i // 7, i % 7) if nm != "classifier" else (12, 0)
+                seeds.append((synth.seed_of(2, layer, j), synth.seed_of(2, layer, j) + 500))
+        self.mats = mats
+        self.weight_bytes = sum(q8_bytes(r, k) for _, r, k in mats)
+        # x: one fp32 buffer, each problem's x 16-byte aligned
+        offs, o = [], 0
+        for _, rows, k in mats:
+            offs.append(o)
+            o += k
+        self.x_host = torch.empty(o, dtype=torch.float32).pin_memory()
+        for (_, rows, k), off, (ws, xs) in zip(mats, offs, seeds):
+            self.x_host[off:off + k] = synth.normal((1, k), xs)[0]
+        self.x = self.x_host.to(dev)
+        self.y = [torch.empty((1, rows), dtype=torch.float32, device=dev) for _, rows, _ in mats]
+        self.out_host = torch.empty(mats[-1][1], dtype=torch.float32).pin_memory()
+        self.w_fp32_seeds = seeds
+        # L2 defeat: rotate through enough byte-identical weight copies
+        self.copies = max(1, -(-3 * L2_BYTES // self.weight_bytes)) if self.weight_bytes > 4e6 else 1
+        self.flush = self.weight_bytes < 4e6
+        packed = []
+        for (_, rows, k), (ws, _) in zip(mats, seeds):
+            w = synth.normal((rows, k), ws, std=synth.W_STD, device=dev)
+            packed.append(q8.pack(w))
+            del w
+        self.W = [packed]
+        for c in range(1, self.copies):
+            self.W.append([q8.Q8Tensor(P.qs.clone(), P.d.clone(), P.k, P.rows, P.n_mat, P.ld_d,
+                                       P.mat_stride) for P in packed])
+        self.offs = offs
+        self.sets = 1
+        self.dominant_launches = 1
+        self.tokens_per_step = 1
+        self.launches_per_step = 1
+        self.dominant_bytes = self.weight_bytes
+        self.h2d_bytes = self.x_host.numel() * 4
+        self.d2h_bytes = self.out_host.numel() * 4
+        self.config = {"workload": self.name, "matvecs": len(mats), "batch": 1,
+                       "weight_bytes_per_step": self.weight_bytes,
+                       "l2": ("flush 256 MiB between steps" if self.flush else
+                              f"{self.copies} rotating weight copies "
+                              f"({self.copies * self.weight_bytes / 2**20:.0f} MiB)")}
+
+    def issue(self, i, marks, input_set=None):
+        W = self.W[i % self.copies]
+        probs = [(Wm, self.x[off:off + Wm.k], y) for Wm, off, y in zip(W, self.offs, self.y)]
+        marks.begin()
+        self.q8.gemv_batched(probs, n_tok=1)
+        marks.end()
+
+    def unique_bytes(self, i):
+        return self.weight_bytes
+
+    def e2e_pre(self):
+        self.x.copy_(self.x_host, non_blocking=True)
+
+    def e2e_post(self):
+        self.out_host.copy_(self.y[-1][0], non_blocking=True)
+
+    # CPU oracle: one token of the same matvec set
+    def oracle_setup(self):
+        import oracle
+        from moe_up_gate_b200 import synth
+        self.ow = []
+        for (_, rows, k), (ws, _) in zip(self.mats, self.w_fp32_seeds):
+            w = synth.normal((rows, k), ws, std=synth.W_STD, device=self.dev).cpu().numpy()
+            self.ow.append(oracle.quantize_rows(w))
+        self.ox = [self.x_host[o:o + k].numpy().reshape(1, k) for o, (_, _, k) in
+                   zip(self.offs, self.mats)]
+
+    def oracle_step(self):
+        import oracle
+        for (wq, wd), x in zip(self.ow, self.ox):
+            xq, xd = oracle.quantize_rows(x)
+            oracle.gemv(wq, wd, xq, xd)
+        return 1  # tokens
+
+
+class MoeWorkload:
+    """MoE (or dense) feed-forward layers through the public calls:
+    quantize x -> group -> fused up/gate + SwiGLU (+ h quantization) -> down
+    mul_mat_id -> combine (dense: quantize -> up/gate -> down GEMV)."""
+    kernel = "up_gate_kernel"
+
+    def __init__(self, dev, kind, tokens):
+        import torch
+
+        from moe_up_gate_b200 import q8, synth
+        self.q8 = q8
+        self.dev = dev
+        if kind == "dense_ffn":
+            shape, layers, c, x_std = synth.DENSE_FFN, 1, 3, 1.0
+            tokens = tokens or 1
+        elif kind == "moe_layer":
+            shape, layers, c, x_std = synth.MOE_LAYER, 1, 4, 1.0
+            tokens = tokens or 1
+        else:
+            shape, layers, c, x_std = synth.MOE_LAYER, synth.MOE_LAYERS, 5, synth.W_STD
+            tokens = tokens or 1
+        self.name = kind
+        self.shape, self.layers, self.T = shape, layers, tokens
+        self.routed = shape.n_exp > 1
+        U = shape.n_used
+        D, F, E = shape.n_embd, shape.n_ff, shape.n_exp
+        self.expert_bytes = q8_bytes(2 * F, D) + q8_bytes(D, F)
+        layer_bytes = E * self.expert_bytes
+        # L2 defeat: enough layer copies that a step never re-reads from L2
+        per_step_max = layers * layer_bytes
+        self.copies = 1 if per_step_max >= 3 * L2_BYTES else -(-3 * L2_BYTES // per_step_max)
+        self.sets = max(self.copies, 4 if self.routed else 1)  # rotating input sets
+        self.L = []
+        for l in range(layers):
+            t = synth.moe_layer_tensors(c, l, shape, tokens, x_std, device=dev)
+            UG = q8.pack(t["up_gate"])
+            DN = q8.pack(t["down"])
+            del t["up_gate"], t["down"]
+            self.L.append((UG, DN))
+        torch.cuda.synchronize()
+        self.Lc = [self.L]
+        for cc in range(1, self.copies):
+            self.Lc.append([tuple(q8.Q8Tensor(P.qs.clone(), P.d.clone(), P.k, P.rows, P.n_mat,
+                                              P.ld_d, P.mat_stride) for P in pair)
+                            for pair in self.L])
+        # inputs per (set, layer)
+        self.x_host, self.ids_host, self.p_host = [], [], []
+        for s in range(self.sets):
+            xs, ids, ps = [], [], []
+            for l in range(layers):
+                xs.append(synth.normal((tokens, D), synth.seed_of(c, l, 2) + 7919 * s, x_std))
+                if self.routed:
+                    ids.append(synth.routing_ids(tokens, E, U, synth.seed_of(c, l, 3) + 7919 * s))
+                    ps.append(synth.routing_weights(tokens, U, synth.seed_of(c, l, 4) + 7919 * s))
+            self.x_host.append(torch.stack(xs).pin_memory())
+            if self.routed:
+                self.ids_host.append(torch.stack(ids).pin_memory())
+                self.p_host.append(torch.stack(ps).pin_memory())
+        self.x = [xh.to(dev) for xh in self.x_host]
+        self.ids = [ih.to(dev) for ih in self.ids_host]
+        self.p = [ph.to(dev) for ph in self.p_host]
+        Uu = U if self.routed else 1
+        P = tokens * Uu
+        self.ws = q8.moe_workspace(tokens, Uu, E, dev) if self.routed else None
+        self.xq = torch.empty((tokens, D), dtype=torch.int8, device=dev)
+        self.xd = torch.empty((tokens, D // 32), dtype=torch.float16, device=dev)
+        self.h = torch.empty((P, F), dtype=torch.float32, device=dev)
+        self.hq = torch.empty((P, F), dtype=torch.int8, device=dev)
+        self.hd = torch.empty((P, F // 32), dtype=torch.float16, device=dev)
+        self.y = torch.empty((tokens, Uu, D), dtype=torch.float32, device=dev)
+        self.out = torch.empty((layers, tokens, D), dtype=torch.float32, device=dev)
+        self.out_host = torch.empty((layers, tokens, D), dtype=torch.float32).pin_memory()
+        # algorithmic bytes: the experts each layer's ids actually name
+        self.step_bytes, self.up_gate_bytes = [], []
+        for s in range(self.sets):
+            tot, ug = 0, 0
+            for l in range(layers):
+                ne = len(set(self.ids_host[s][l].flatten().tolist())) if self.routed else 1
+                tot += ne * self.expert_bytes
+                ug += ne * q8_bytes(2 * F, D)
+            self.step_bytes.append(tot)
+            self.up_gate_bytes.append(ug / layers)
+        self.tokens_per_step = tokens
+        self.launches_per_step = layers * (5 if self.routed else 3)
+        self.dominant_launches = layers
+        self.h2d_bytes = self.x_host[0].numel() * 4 + (
+            (self.ids_host[0].numel() * 4 + self.p_host[0].numel() * 4) if self.routed else 0)
+        self.d2h_bytes = self.out_host.numel() * 4
+        self.config = {"workload": kind, "tokens": tokens, "layers": layers, "n_embd": D,
+                       "n_ff": F, "n_experts": E, "n_used": Uu,
+                       "mean_weight_bytes_per_step": statistics.mean(self.step_bytes),
+                       "l2": (f"{self.copies} rotating weight copies, {self.sets} input sets"
+                              if self.copies > 1 else
+                              f"weights per step > 3x L2; {self.sets} input sets")}
+
+    def issue(self, i, marks, input_set=None):
+        q8 = self.q8
+        s = i % self.sets if input_set is None else input_set
+        layers = self.Lc[i % self.copies]
+        T = self.T
+        for l, (UG, DN) in enumerate(layers):
+            x = self.x[s][l]
+            q8._call("q8_quantize_row", q8._ptr(x), T, UG.k, q8._ptr(self.xq), q8._ptr(self.xd),
+                     q8._stream())
+            if self.routed:
+                U = self.shape.n_used
+                q8.moe_group(self.ids[s][l], UG.n_mat, ws=self.ws)
+                marks.begin()
+                q8.moe_up_gate_swiglu_pregrouped(UG, self.xq, self.xd, U, self.ws, self.h, self.hq,
+                                                 self.hd)
+                marks.end()
+                q8.mul_mat_id_pregrouped(DN, self.hq, self.hd, T, U, True, self.ws, self.y)
+                q8.moe_combine(self.y, self.p[s][l], out=self.out[l])
+            else:
+                marks.begin()
+                q8._call("q8_moe_up_gate_swiglu", q8.ctypes.byref(UG.c()), q8._ptr(self.xq),
+                         q8._ptr(self.xd), T, None, 1, q8._ptr(self.h), q8._ptr(self.hq),
+                         q8._ptr(self.hd), None, None, None, 0, q8._stream())
+                marks.end()
+                q8.gemv(DN, self.hq, self.hd, y=self.out[l])
+
+    def unique_bytes(self, i):
+        return self.step_bytes[i % self.sets]
+
+    def dominant_bytes_at(self, i):
+        return self.up_gate_bytes[i % self.sets]
+
+    def e2e_pre(self):
+        self.x[0].copy_(self.x_host[0], non_blocking=True)
+        if self.routed:
+            self.ids[0].copy_(self.ids_host[0], non_blocking=True)
+            self.p[0].copy_(self.p_host[0], non_blocking=True)
+
+    def e2e_post(self):
+        self.out_host.copy_(self.out, non_blocking=True)
+
+    def oracle_setup(self):
+        import oracle
+        from moe_up_gate_b200 import synth
+        # one layer through the oracle (its own quantization of the fp32 weights)
+        c = {"dense_ffn": 3, "moe_layer": 4, "moe_30layer": 5}[self.name]
+        x_std = synth.W_STD if self.name == "moe_30layer" else 1.0
+        t = synth.moe_layer_tensors(c, 0, self.shape, self.T, x_std, device=self.dev)
+        self.o_ug = oracle.quantize_rows(t["up_gate"].cpu().numpy())
+        self.o_dn = oracle.quantize_rows(t["down"].cpu().numpy())
+        self.o_x = self.x_host[0][0].numpy()
+        self.o_ids = self.ids_host[0][0].numpy() if self.routed else None
+        self.o_p = self.p_host[0][0].numpy() if self.routed else None
+
+    def oracle_step(self):
+        import oracle
+        oracle.moe_ffn(self.o_ug[0], self.o_ug[1], self.o_dn[0], self.o_dn[1], self.o_x,
+                       self.o_ids, self.o_p)
+        return self.T / self.layers  # one layer of a layers-deep step
+
+
+def make_workload(args, dev):
+    if args.workload == "llama2_110m_q8_decode":
+        return LlamaDecode(dev)
+    if args.workload == "gemv_768":
+        return LlamaDecode(dev, gemv768=True)
+    return MoeWorkload(dev, args.workload, args.tokens)
+
+
+# ---------------------------------------------------------------------------
+# traffic counters recorded by ncu (profiles/traffic.json), valid only for
+# the kernel sources they were taken on
+# ---------------------------------------------------------------------------
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "moe_up_gate_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, kernel):
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(f"{workload}:{kernel}")
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing
+# ---------------------------------------------------------------------------
+def time_oracle(wl, seconds, steps=None):
+    import oracle
+    wl.oracle_setup()
+    cores = oracle.max_threads()
+    done, t0, n = 0.0, time.perf_counter(), 0
+    times = []
+    while True:
+        a = time.perf_counter()
+        done += wl.oracle_step()
+        times.append(time.perf_counter() - a)
+        n += 1
+        if steps is not None:
+            if n >= steps:
+                break
+        elif time.perf_counter() - t0 >= seconds:
+            break
+    return done, sum(times), n, cores, times
+
+
+# ---------------------------------------------------------------------------
+def run_reference(args, dist):
+    """The reference arm: the CPU oracle, as it stands, on the host cores."""
+    if dist.rank != 0:
+        return
+    import torch
+    dev = "cuda:0" if torch.cuda.is_available() else "cpu"
+    wl = make_workload(args, dev) if dev != "cpu" else None
+    if wl is None:
+        print(json.dumps({"impl": "reference", "unavailable": "needs a CUDA device to draw the "
+                          "same synthetic inputs"}))
+        return
+    import oracle
+    wl.oracle_setup()
+    for _ in range(args.warmup):
+        wl.oracle_step()
+    t0 = time.perf_counter()
+    toks = 0.0
+    for _ in range(args.steps):
+        toks += wl.oracle_step()
+    el = time.perf_counter() - t0
+    v = toks / el
+    sample = (f"{args.steps} steps of one {wl.name} token through the scalar C oracle"
+              if isinstance(wl, LlamaDecode) else
+              f"{args.steps} x one layer of {wl.name} (T={wl.T}) through the scalar C oracle, "
+              f"counted as 1/{wl.layers} of a step")
+    out = {"metric": "Q8_0 decode tokens/s", "value": v, "unit": "tokens/s", "impl": "reference",
+           "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "int8 x int8 -> int32, fp64 sums", "data": "synthetic",
+           "config": wl.config,
+           "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.max_threads(),
+                            "kind": "oracle", "sample": sample},
+           "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+
+
+def main():
+    args = parse()
+    dist = Dist()
+    if args.impl == "reference":
+        run_reference(args, dist)
+        return
+    import torch
+    torch.cuda.set_device(dist.local)
+    dev = f"cuda:{dist.local}"
+    dist.init("nccl")
+    from moe_up_gate_b200 import q8
+    q8.load()
+    wl = make_workload(args, dev)
+    stream = torch.cuda.Stream(device=dev)
+    K, W = args.steps, max(args.warmup, 3)
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev) if getattr(wl, "flush", False) \
+        else None
+
+    # one CUDA graph per step index (each with its own timing marks)
+    graphs, marks = [], []
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        wl.issue(0, NoMarks())  # eager warm-up (sets kernel attributes)
+    torch.cuda.synchronize()
+    for i in range(W + K):
+        m = Marks(wl.dominant_launches) if i >= W else NoMarks()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            wl.issue(i, m)
+        graphs.append(g)
+        marks.append(m)
+    torch.cuda.synchronize()
+
+    # device-timed region
+    st_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    en_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            if flush is not None:
+                flush.zero_()
+            graphs[i].replay()
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = ClockSampler(dist.local)
+    clocks.start()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(K):
+            if flush is not None:
+                flush.zero_()
+            st_ev[i].record(stream)
+            graphs[W + i].replay()
+            en_ev[i].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in zip(st_ev, en_ev)]
+    total_ms = dist.max(sum(step_ms))
+    dom_ms = []
+    for m in marks[W:]:
+        dom_ms.extend(m.ms())
+
+    # end to end through the public API with host buffers: every step copies
+    # its inputs from pinned host memory, runs the step (graphs of the same
+    # public calls, reading input set 0) and copies its result back
+    e2e_graphs = []
+    for c in range(wl.copies):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            wl.issue(c, NoMarks(), input_set=0)
+        e2e_graphs.append(g)
+    e2e_ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    torch.cuda.synchronize()
+    dist.barrier()
+    with torch.cuda.stream(stream):
+        e2e_ev[0].record(stream)
+        for i in range(K):
+            wl.e2e_pre()
+            e2e_graphs[i % wl.copies].replay()
+            wl.e2e_post()
+        e2e_ev[1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = dist.max(e2e_ev[0].elapsed_time(e2e_ev[1]))
+    dist.barrier()
+
+    n = dist.world
+    tokens = wl.tokens_per_step * K * n
+    value = tokens / (total_ms / 1e3)
+    step_bytes = statistics.mean(wl.unique_bytes(W + i) for i in range(K))
+    peak, peak_kind = measured_peak()
+    if isinstance(wl, LlamaDecode):
+        dom_bytes = wl.dominant_bytes
+    else:
+        dom_bytes = statistics.mean(wl.dominant_bytes_at(W + i) for i in range(K))
+    dom_avg_ms = statistics.mean(dom_ms) if dom_ms else None
+    achieved = dom_bytes / (dom_avg_ms / 1e3) / 1e9 if dom_avg_ms else None
+    traffic = recorded_traffic(wl.name + (f"_t{wl.T}" if hasattr(wl, "T") else ""), wl.kernel)
+    out = {
+        "metric": "Q8_0 decode tokens/s", "value": value, "unit": "tokens/s", "n_gpus": n,
+        "steps": K, "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8 x int8 -> int32, fp32 sums",
+        "data": "synthetic (seeded N(0, 0.02) weights quantized to Q8_0, N(0,1) inputs)",
+        "config": dict(wl.config, parallelism=f"replicas x{n}"),
+        "effective_weight_GBps": step_bytes * K * n / (total_ms / 1e3) / 1e9 / n,
+        "effective_weight_frac_of_hbm": step_bytes / (total_ms / K / 1e3) / 1e9 / peak,
+        "roofline": {"bound": "hbm", "kernel": wl.kernel, "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": (achieved / peak) if achieved else None,
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "bytes_per_launch": dom_bytes, "avg_launch_ms": dom_avg_ms,
+                     "traffic": traffic},
+        "clocks": clk,
+        "e2e": {"value": wl.tokens_per_step * K * n / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": wl.h2d_bytes, "d2h_bytes_per_step": wl.d2h_bytes},
+        "gpu_launches": wl.launches_per_step * K,
+    }
+    if dist.rank == 0 and n == 1 and not args.no_cpu_baseline:
+        done, el, nsteps, cores, _ = time_oracle(wl, args.cpu_seconds)
+        out["cpu_baseline"] = {
+            "value": done / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": (f"{nsteps} tokens of {wl.name} through the scalar C oracle "
+                       f"(OpenMP over output rows), {el:.1f} s"
+                       if isinstance(wl, LlamaDecode) else
+                       f"{nsteps} x one layer of {wl.name} (T={wl.T}) through the scalar C "
+                       f"oracle, counted as 1/{wl.layers} of a step, {el:.1f} s")}
+    if dist.rank == 0:
+        print(json.dumps(out))
+    del graphs, e2e_graphs
+    dist.close()
+
+
+if __name__ == "__main__":
+    main()

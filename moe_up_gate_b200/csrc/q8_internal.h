@@ -1,0 +1,80 @@
+// q8_internal.h -- host-side helpers shared by the libq8 translation units:
+// argument validation, the per-thread error detail, launch checks and the
+// workspace layout of the routed (MoE) calls.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include "../../include/q8.h"
+
+namespace q8 {
+
+// Per-thread detail text of the last failure (q8_last_error).
+void set_error_detail(const char *fmt, ...);
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+#define Q8_FAIL(code, ...)                 \
+    do {                                   \
+        ::q8::set_error_detail(__VA_ARGS__); \
+        return (code);                     \
+    } while (0)
+
+#define Q8_REQUIRE(cond, code, ...)        \
+    do {                                   \
+        if (!(cond)) Q8_FAIL(code, __VA_ARGS__); \
+    } while (0)
+
+// After a kernel launch: turn a launch error into Q8_E_CUDA.
+inline q8_status launch_status(const char *what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        set_error_detail("%s: %s", what, cudaGetErrorString(e));
+        return Q8_E_CUDA;
+    }
+    return Q8_OK;
+}
+
+// Validate a weight view.  need_single: n_mat must be 1.
+q8_status check_tensor(const q8_tensor *W, const char *name, bool need_single);
+
+// ---------------------------------------------------------------------------
+// Routed-call workspace: int32 words.
+//   [0] error flags  [1] number of experts in the dp4a list  [2] number in the
+//   tensor-core list  [3] pairs  then count[E], offset[E+1], list_small[E],
+//   list_big[E], pairs[P] (pair index p = t * n_used + s, sorted by expert,
+//   then p).
+// ---------------------------------------------------------------------------
+enum : int { WS_ERR = 0, WS_N_SMALL = 1, WS_N_BIG = 2, WS_N_PAIRS = 3, WS_HEADER = 4 };
+enum : int { ERR_ID_RANGE = 1, ERR_ID_REPEAT = 2 };
+
+struct GroupLayout {
+    int64_t count, offset, list_small, list_big, pairs, words;
+};
+
+inline GroupLayout group_layout(int64_t n_pairs, int64_t n_mat) {
+    GroupLayout L;
+    L.count = WS_HEADER;
+    L.offset = L.count + n_mat;
+    L.list_small = L.offset + n_mat + 1;
+    L.list_big = L.list_small + n_mat;
+    L.pairs = L.list_big + n_mat;
+    L.words = L.pairs + n_pairs;
+    return L;
+}
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline size_t group_bytes(int64_t n_pairs, int64_t n_mat) {
+    return round_up((size_t)group_layout(n_pairs, n_mat).words * 4, 256);
+}
+
+// Launch the expert-grouping kernel (q8_moe.cu).  big_threshold: experts with
+// at least this many pairs go to the tensor-core list.
+q8_status launch_group(const int32_t *ids, int64_t n_tok, int32_t n_used, int64_t n_mat,
+                       int32_t big_threshold, int32_t *ws, cudaStream_t s);
+
+}  // namespace q8
