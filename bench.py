@@ -25,6 +25,7 @@ import os
 import statistics
 import subprocess
 import sys
+import math
 import threading
 import time
 
@@ -48,6 +49,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="bound on the CPU baseline sample")
+    ap.add_argument("--min-seconds", type=float, default=1.0,
+                    help="timed work, in rounds of exactly --steps steps")
     return ap.parse_args()
 
 
@@ -109,7 +112,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
             return
@@ -461,6 +464,18 @@ def make_workload(args, dev):
 # traffic counters recorded by ncu (profiles/traffic.json), valid only for
 # the kernel sources they were taken on
 # ---------------------------------------------------------------------------
+def gpu_id(local_rank: int) -> str:
+    """nvidia-smi --id for this rank's device (PCI bus id when torch knows it)."""
+    import torch
+    try:
+        bus = torch.cuda.get_device_properties(local_rank).pci_bus_id
+        if bus:
+            return str(bus)
+    except (AttributeError, RuntimeError):
+        pass
+    return str(local_rank)
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "moe_up_gate_b200", "csrc")
@@ -586,7 +601,10 @@ def main():
         marks.append(m)
     torch.cuda.synchronize()
 
-    # device-timed region
+    # device-timed region: rounds of exactly K steps, each bracketed by a
+    # barrier and a synchronize; enough rounds for about --min-seconds of
+    # timed work (the clock sampler needs that long); the median round is
+    # reported (after the 11-round, median protocol of the narray-llm README)
     st_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     en_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     with torch.cuda.stream(stream):
@@ -595,25 +613,37 @@ def main():
                 flush.zero_()
             graphs[i].replay()
     torch.cuda.synchronize()
-    dist.barrier()
-    clocks = ClockSampler(dist.local)
+    clocks = ClockSampler(gpu_id(dist.local))
     clocks.start()
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        for i in range(K):
-            if flush is not None:
-                flush.zero_()
-            st_ev[i].record(stream)
-            graphs[W + i].replay()
-            en_ev[i].record(stream)
-    torch.cuda.synchronize()
+    time.sleep(0.5)  # let the sampler start before the timed work
+
+    def one_round():
+        torch.cuda.synchronize()
+        dist.barrier()
+        with torch.cuda.stream(stream):
+            for i in range(K):
+                if flush is not None:
+                    flush.zero_()
+                st_ev[i].record(stream)
+                graphs[W + i].replay()
+                en_ev[i].record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        ms = dist.max(sum(a.elapsed_time(b) for a, b in zip(st_ev, en_ev)))
+        dom = []
+        for m in marks[W:]:
+            dom.extend(m.ms())
+        return ms, dom
+
+    first_ms, dom_ms = one_round()
+    rounds = int(min(1000, max(3, math.ceil(args.min_seconds * 1e3 / max(first_ms, 1e-3)))))
+    round_ms = [first_ms]
+    for _ in range(rounds - 1):
+        ms, dom = one_round()
+        round_ms.append(ms)
+        dom_ms.extend(dom)
     clk = clocks.stop()
-    dist.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in zip(st_ev, en_ev)]
-    total_ms = dist.max(sum(step_ms))
-    dom_ms = []
-    for m in marks[W:]:
-        dom_ms.extend(m.ms())
+    total_ms = statistics.median(round_ms)
 
     # end to end through the public API with host buffers: every step copies
     # its inputs from pinned host memory, runs the step (graphs of the same
@@ -655,7 +685,8 @@ def main():
         "steps": K, "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8 x int8 -> int32, fp32 sums",
         "data": "synthetic (seeded N(0, 0.02) weights quantized to Q8_0, N(0,1) inputs)",
-        "config": dict(wl.config, parallelism=f"replicas x{n}"),
+        "config": dict(wl.config, parallelism=f"replicas x{n}", rounds=len(round_ms),
+                       round_ms_min_median_max=[min(round_ms), total_ms, max(round_ms)]),
         "effective_weight_GBps": step_bytes * K * n / (total_ms / 1e3) / 1e9 / n,
         "effective_weight_frac_of_hbm": step_bytes / (total_ms / K / 1e3) / 1e9 / peak,
         "roofline": {"bound": "hbm", "kernel": wl.kernel, "achieved": achieved, "peak": peak,
