@@ -222,6 +222,38 @@ q8_status q8_mul_mat_id_pregrouped(const q8_tensor *W, const int8_t *aq, const u
                                    const void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * q8_moe_up_gate_swiglu_noalloc -- q8_moe_up_gate_swiglu for callers that
+ * cannot allocate device memory (no counterpart on the pages: this is a
+ * library convenience, not part of the method).  Some callers cannot call
+ * cudaMalloc or an allocating library routine at the point where they run
+ * the step: code inside a custom allocator or memory-pool hook, plugins whose
+ * host forbids device allocation, or hot loops that must not touch the
+ * allocator.  This variant takes no workspace: the expert-grouping tables live
+ * in a file-scope device array of Q8_NOALLOC_SCRATCH_BYTES bytes inside
+ * libq8, which every GPU that loads the library holds until the process exits.
+ *  Arguments, outputs and results are those of q8_moe_up_gate_swiglu (ids
+ *  required), except that there is no ws / ws_bytes.
+ *  Limit: the grouping tables must fit the scratch, i.e.
+ *  q8_moe_workspace_size(n_tok, n_used, up_gate->n_mat) <= Q8_NOALLOC_SCRATCH_BYTES
+ *  (for 128 experts and 8 per token: up to 1983 tokens); larger calls return
+ *  Q8_E_WORKSPACE and launch nothing.
+ *  The first call on each device looks up the scratch address on that device
+ *  (cudaGetSymbolAddress, with that device current); make that first call
+ *  before any stream capture.  Every call shares the one scratch array: calls
+ *  that overlap on the GPU (other streams, other host threads) race and give
+ *  wrong results; serialize them.  The scratch keeps the last call's contents;
+ *  nothing in it needs clearing, because the grouping kernel rewrites every
+ *  word that the up/gate kernel later reads.  Routing-id errors are not
+ *  reported by this variant (no q8_check): pairs whose id is out of range are
+ *  skipped and their outputs left unwritten.
+ */
+#define Q8_NOALLOC_SCRATCH_BYTES 65536
+q8_status q8_moe_up_gate_swiglu_noalloc(const q8_tensor *up_gate, const int8_t *xq,
+                                        const uint16_t *xd, int64_t n_tok, const int32_t *ids,
+                                        int32_t n_used, float *h, int8_t *hq, uint16_t *hd,
+                                        float *g_out, float *u_out, void *stream);
+
+/*
  * q8_moe_combine -- out[t] = sum_{s < n_used} route_w[t][s] * y[t][s], summed in
  * ascending s (the routing-weight combine after the down projection).
  *  y: fp32 [n_tok][n_used][n_out]; route_w: fp32 [n_tok][n_used];

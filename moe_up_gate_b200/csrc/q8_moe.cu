@@ -10,6 +10,7 @@
 // view_3d slices and a separate fused_mul_unary, this kernel reads gate row r
 // and up row n_ff + r in the same pass and applies SwiGLU in registers.
 #include <algorithm>
+#include <mutex>
 
 #include "q8_internal.h"
 #include "q8_tile.cuh"
@@ -398,6 +399,39 @@ q8_status q8_moe_up_gate_swiglu_pregrouped(const q8_tensor *up_gate, const int8_
                          (cudaStream_t)stream);
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free variant: the grouping tables live in this file-scope device
+// array instead of a caller workspace.  Host code must not pass the array's
+// name to a kernel (on the host it is only a stand-in symbol); its device
+// address is looked up once per device with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) int32_t g_noalloc_scratch[Q8_NOALLOC_SCRATCH_BYTES / 4];
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_noalloc_mu;
+static void *g_noalloc_addr[kMaxDevices] = {};
+
+static q8_status noalloc_scratch_address(void **out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        Q8_FAIL(Q8_E_CUDA, "q8_moe_up_gate_swiglu_noalloc: cudaGetDevice: %s",
+                cudaGetErrorString(e));
+    Q8_REQUIRE(dev >= 0 && dev < kMaxDevices, Q8_E_UNSUPPORTED,
+               "q8_moe_up_gate_swiglu_noalloc: device %d beyond %d", dev, kMaxDevices);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr)
+            Q8_FAIL(Q8_E_CUDA, "q8_moe_up_gate_swiglu_noalloc: cudaGetSymbolAddress: %s",
+                    cudaGetErrorString(e));
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return Q8_OK;
+}
+
 q8_status q8_moe_group(const int32_t *ids, int64_t n_tok, int32_t n_used, int64_t n_mat,
                        void *ws, size_t ws_bytes, void *stream) {
     Q8_REQUIRE(ids != nullptr, Q8_E_NULL, "q8_moe_group: ids is NULL");
@@ -412,6 +446,29 @@ q8_status q8_moe_group(const int32_t *ids, int64_t n_tok, int32_t n_used, int64_
     Q8_REQUIRE(ws_bytes >= q8_moe_workspace_size(n_tok, n_used, n_mat), Q8_E_WORKSPACE,
                "q8_moe_group: workspace too small");
     return launch_group(ids, n_tok, n_used, n_mat, 1 << 30, (int32_t *)ws, (cudaStream_t)stream);
+}
+
+q8_status q8_moe_up_gate_swiglu_noalloc(const q8_tensor *up_gate, const int8_t *xq,
+                                        const uint16_t *xd, int64_t n_tok, const int32_t *ids,
+                                        int32_t n_used, float *h, int8_t *hq, uint16_t *hd,
+                                        float *g_out, float *u_out, void *stream) {
+    const char *fn = "q8_moe_up_gate_swiglu_noalloc";
+    Q8_REQUIRE(up_gate != nullptr && ids != nullptr, Q8_E_NULL, "%s: up_gate and ids required",
+               fn);
+    Q8_REQUIRE(n_tok >= 1 && n_used >= 1 && n_used <= Q8_MAX_USED &&
+                   n_tok * n_used <= (1LL << 24) && up_gate->n_mat >= 1,
+               Q8_E_SHAPE, "%s: n_tok=%lld n_used=%d", fn, (long long)n_tok, n_used);
+    const size_t need = q8_moe_workspace_size(n_tok, n_used, up_gate->n_mat);
+    Q8_REQUIRE(need <= (size_t)Q8_NOALLOC_SCRATCH_BYTES, Q8_E_WORKSPACE,
+               "%s: n_tok*n_used=%lld with n_mat=%lld needs %zu bytes of grouping scratch; the "
+               "built-in scratch holds %d (use q8_moe_up_gate_swiglu with a workspace)",
+               fn, (long long)(n_tok * n_used), (long long)up_gate->n_mat, need,
+               Q8_NOALLOC_SCRATCH_BYTES);
+    void *scratch = nullptr;
+    q8_status st = noalloc_scratch_address(&scratch);
+    if (st != Q8_OK) return st;
+    return up_gate_entry(fn, up_gate, xq, xd, n_tok, ids, true, true, n_used, h, hq, hd, g_out,
+                         u_out, scratch, Q8_NOALLOC_SCRATCH_BYTES, (cudaStream_t)stream);
 }
 
 q8_status q8_moe_combine(const float *y, const float *route_w, int64_t n_tok, int32_t n_used,

@@ -46,7 +46,8 @@ EXPORTS = ["q8_scale_stride", "q8_pack", "q8_quantize_row", "q8_gemv", "q8_gemv_
            "q8_moe_workspace_size", "q8_moe_up_gate_swiglu", "q8_mul_mat_id", "q8_moe_combine",
            "q8_moe_ffn_workspace_size", "q8_moe_ffn", "q8_check", "q8_debug_block_dots",
            "q8_status_string", "q8_last_error", "q8_moe_group",
-           "q8_moe_up_gate_swiglu_pregrouped", "q8_mul_mat_id_pregrouped"]
+           "q8_moe_up_gate_swiglu_pregrouped", "q8_mul_mat_id_pregrouped",
+           "q8_moe_up_gate_swiglu_noalloc"]
 
 
 def lib_path() -> str:
@@ -88,6 +89,8 @@ def load(auto_build: bool = True):
                                                       vp, vp, vp, sz, vp]),
             "q8_mul_mat_id_pregrouped": (st, [P(_Tensor), vp, vp, i32, i64, i32, vp, vp, sz,
                                               vp]),
+            "q8_moe_up_gate_swiglu_noalloc": (st, [P(_Tensor), vp, vp, i64, vp, i32, vp, vp, vp,
+                                                   vp, vp, vp]),
             "q8_status_string": (ctypes.c_char_p, [st]),
             "q8_last_error": (ctypes.c_char_p, []),
         }
@@ -242,6 +245,16 @@ def moe_up_gate_swiglu(W: Q8Tensor, xq, xd, ids=None, want_hq=True, want_gu=Fals
           n_used, _ptr(h), _ptr(hq), _ptr(hd), _ptr(g), _ptr(u), _ptr(ws),
           0 if ws is None else ws.numel(), _stream(stream))
     return dict(h=h, hq=hq, hd=hd, g=g, u=u, ws=ws)
+
+
+def moe_up_gate_swiglu_noalloc(W: Q8Tensor, xq, xd, ids, h, hq=None, hd=None, g=None, u=None,
+                               stream=None):
+    """Routed up/gate + SwiGLU into caller-provided outputs, with no workspace
+    (the grouping tables live in libq8's built-in device scratch)."""
+    _call("q8_moe_up_gate_swiglu_noalloc", ctypes.byref(W.c()), _ptr(xq), _ptr(xd),
+          xq.shape[0], _ptr(ids), ids.shape[1], _ptr(h), _ptr(hq), _ptr(hd), _ptr(g), _ptr(u),
+          _stream(stream))
+    return h
 
 
 def mul_mat_id(W: Q8Tensor, aq, ad, ids, a_per_slot: bool, ws=None, y=None, stream=None):
