@@ -112,7 +112,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
         except (OSError, ValueError):
             self.proc = None
             return
@@ -132,6 +132,10 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.thr.join(timeout=2)
+        try:
+            err = self.proc.stderr.read()[-300:]
+        except (OSError, ValueError):
+            err = ""
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
@@ -146,9 +150,12 @@ class ClockSampler:
             for n, v in zip(names, parts[3:]):
                 if v.lower() == "active":
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        out = {"sm_mhz": statistics.median(sm) if sm else None,
+               "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+               "samples": len(sm)}
+        if not sm:
+            out["sampler_output"] = (self.lines[:2], err.strip())
+        return out
 
 
 # ---------------------------------------------------------------------------
@@ -468,12 +475,10 @@ def gpu_id(local_rank: int) -> str:
     """nvidia-smi --id for this rank's device (PCI bus id when torch knows it)."""
     import torch
     try:
-        bus = torch.cuda.get_device_properties(local_rank).pci_bus_id
-        if bus:
-            return str(bus)
-    except (AttributeError, RuntimeError):
-        pass
-    return str(local_rank)
+        pr = torch.cuda.get_device_properties(local_rank)
+        return f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+    except (AttributeError, RuntimeError, TypeError, ValueError):
+        return str(local_rank)
 
 
 def kernel_source_hash():
@@ -635,6 +640,7 @@ def main():
             dom.extend(m.ms())
         return ms, dom
 
+    torch.cuda.nvtx.range_push("timed")
     first_ms, dom_ms = one_round()
     rounds = int(min(1000, max(3, math.ceil(args.min_seconds * 1e3 / max(first_ms, 1e-3)))))
     round_ms = [first_ms]
@@ -642,6 +648,7 @@ def main():
         ms, dom = one_round()
         round_ms.append(ms)
         dom_ms.extend(dom)
+    torch.cuda.nvtx.range_pop()
     clk = clocks.stop()
     total_ms = statistics.median(round_ms)
 

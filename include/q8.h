@@ -281,11 +281,16 @@ q8_status q8_moe_ffn(const q8_tensor *up_gate, const q8_tensor *down, const floa
                      float *out, void *ws, size_t ws_bytes, void *stream);
 
 /*
- * q8_check -- synchronize `stream`, read the device error word in ws (written
- * by the last routed call that used ws) and return Q8_E_BAD_ID if an id was
- * out of range or repeated within a token, else Q8_OK (or Q8_E_CUDA if the
- * stream reported an error).  When it returns Q8_E_BAD_ID, the outputs of
- * pairs with out-of-range ids are unspecified.
+ * q8_check -- synchronize `stream` and report errors found on the device:
+ *  - Q8_E_BAD_ID if ws (optional; NULL skips this check) holds a routing-id
+ *    error from the last routed call that used it: an id out of range or
+ *    repeated within a token.  The outputs of pairs with out-of-range ids are
+ *    then unspecified.
+ *  - Q8_E_CUDA if the stream reported an error, or if a streaming kernel on
+ *    this device ever gave up waiting (after about 2 s) for a shared-memory
+ *    stage; that flag stays set for the life of the process, and results
+ *    computed after it are not to be trusted.
+ * Else Q8_OK.
  */
 q8_status q8_check(const void *ws, void *stream);
 

@@ -74,17 +74,18 @@ __device__ __forceinline__ uint16_t ld_stream_u16(const uint16_t *p) {
 // ---------------------------------------------------------------------------
 // exact block dot: 32 int8 x 32 int8 -> int32, as 8 dp4a
 // ---------------------------------------------------------------------------
+// (two independent 4-deep dp4a chains, then one add: exact in int32)
 __device__ __forceinline__ int block_dot(const uint4 &w0, const uint4 &w1, const uint4 &x0,
                                          const uint4 &x1) {
-    int s = __dp4a((int)w0.x, (int)x0.x, 0);
-    s = __dp4a((int)w0.y, (int)x0.y, s);
-    s = __dp4a((int)w0.z, (int)x0.z, s);
-    s = __dp4a((int)w0.w, (int)x0.w, s);
-    s = __dp4a((int)w1.x, (int)x1.x, s);
-    s = __dp4a((int)w1.y, (int)x1.y, s);
-    s = __dp4a((int)w1.z, (int)x1.z, s);
-    s = __dp4a((int)w1.w, (int)x1.w, s);
-    return s;
+    int a = __dp4a((int)w0.x, (int)x0.x, 0);
+    int b = __dp4a((int)w1.x, (int)x1.x, 0);
+    a = __dp4a((int)w0.y, (int)x0.y, a);
+    b = __dp4a((int)w1.y, (int)x1.y, b);
+    a = __dp4a((int)w0.z, (int)x0.z, a);
+    b = __dp4a((int)w1.z, (int)x1.z, b);
+    a = __dp4a((int)w0.w, (int)x0.w, a);
+    b = __dp4a((int)w1.w, (int)x1.w, b);
+    return a + b;
 }
 
 }  // namespace q8

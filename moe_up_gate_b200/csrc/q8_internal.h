@@ -38,6 +38,30 @@ inline q8_status launch_status(const char *what) {
     return Q8_OK;
 }
 
+// Launch with programmatic stream serialization.  The kernel must execute
+// griddepcontrol.wait before it reads anything an earlier kernel writes
+// (and before it writes anything an earlier kernel reads).
+template <typename... KArgs, typename... Args>
+inline q8_status launch_pdl(const char *what, void (*kern)(KArgs...), dim3 grid, dim3 block,
+                            size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e != cudaSuccess) {
+        set_error_detail("%s: launch: %s", what, cudaGetErrorString(e));
+        return Q8_E_CUDA;
+    }
+    return Q8_OK;
+}
+
 // Validate a weight view.  need_single: n_mat must be 1.
 q8_status check_tensor(const q8_tensor *W, const char *name, bool need_single);
 
@@ -71,6 +95,31 @@ inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline size_t group_bytes(int64_t n_pairs, int64_t n_mat) {
     return round_up((size_t)group_layout(n_pairs, n_mat).words * 4, 256);
 }
+
+// Whether a kernel has been given the full shared-memory opt-in on a device
+// (q8_quant.cu keeps the registry, guarded by a mutex).
+bool smem_opted_in(const void *kernel, int device);
+void set_smem_opted_in(const void *kernel, int device);
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+// Quantize rows (q8_quant.cu): scales to d[row * ld_d + b].  weights: the
+// output is packed weights (the next kernel may not start before it ends).
+q8_status launch_quantize(const float *x, int64_t n_rows, int64_t k, int8_t *qs, uint16_t *d,
+                          int64_t ld_d, cudaStream_t s, bool weights = false);
+
+// Streaming matmuls (q8_matmul.cu).  Activations are Q8_0 (aq, ad) or fp32
+// (af, quantized by the Q8_0 rule as they are staged).
+q8_status launch_matmul_routed(const q8_tensor *W, const int8_t *aq, const uint16_t *ad,
+                               const float *af, int a_per_slot, int64_t n_tok, int32_t n_used,
+                               float *y, const int32_t *ws, cudaStream_t s);
+q8_status launch_matmul_dense(const q8_tensor *W, const int8_t *aq, const uint16_t *ad,
+                              const float *af, int64_t n_tok, float *y, cudaStream_t s);
+
+// Wait-timeout flags latched by the streaming kernels of each file.
+q8_status read_wait_errors_matmul(int *flags);
+q8_status read_wait_errors_moe(int *flags);
 
 // Launch the expert-grouping kernel (q8_moe.cu).  big_threshold: experts with
 // at least this many pairs go to the tensor-core list.

@@ -4,24 +4,33 @@
 //
 // The Q8_0 decode matvec is the hot loop of the Llama 2 110M int8 decode in
 // the "narray-llm" README (section "Llama 2 110M を int8 (Q8_0) で");
-// mul_mat_id is ggml_mul_mat_id of the news.hada.io article (section
-// 「3段階で構成された修正」), applied per routed expert.
+// mul_mat_id is ggml_mul_mat_id of the news.hada.io article on Gemma 4
+// 26B-A4B Q8_0 (section 「3段階で構成された修正」), applied per routed expert.
+// All of them run on the streaming engine of q8_stream.cuh.
 #include <algorithm>
 
 #include "q8_internal.h"
-#include "q8_tile.cuh"
+#include "q8_stream.cuh"
 
 namespace q8 {
 
-constexpr int kThreads = 256;
+// Wait timeouts of the kernels in this file (read by q8_check).
+static __device__ int g_err_matmul;
+
+q8_status read_wait_errors_matmul(int *flags) {
+    cudaError_t e = cudaMemcpyFromSymbol(flags, g_err_matmul, sizeof(int));
+    return e == cudaSuccess ? Q8_OK : Q8_E_CUDA;
+}
 
 // ---------------------------------------------------------------------------
-// matmul over a group of activation rows per matrix.
-//   dense  (ws == nullptr): matrix 0, pairs 0..n_dense-1, activation row = pair.
-//   routed (ws != nullptr): CTA row blockIdx.y is the blockIdx.y-th expert of
-//     the grouping list; its pairs come from the grouping tables; activation
-//     row = pair (a_per_slot) or pair / n_used.
-// Output y[pair][row].
+// matmul over the activation rows of each matrix.
+//   dense  (ws == nullptr): matrix 0; activation rows 0..n_dense-1; output
+//          row = activation row.
+//   routed (ws != nullptr): the experts of the grouping list; for expert e the
+//          pairs p of its list; activation row = p (a_per_slot) or p / n_used;
+//          output row = p.
+// Activations are Q8_0 (aq, ad) or fp32 (af, quantized while staged).
+// Output y[out_row * rows + r].
 // ---------------------------------------------------------------------------
 struct MatmulParams {
     const int8_t *wq;
@@ -32,103 +41,205 @@ struct MatmulParams {
     int rows;
     const int8_t *aq;
     const uint16_t *ad;
+    const float *af;
     float *y;
     const int32_t *ws;
     int64_t lay_count, lay_offset, lay_list, lay_pairs;
-    int list_word;  // WS_N_SMALL or WS_N_BIG
+    int list_word;
     int n_dense;
     int a_per_slot;
     int n_used;
-    int rows_per_cta;
+    Plan plan;
 };
 
-template <int NT, int R>
-__global__ void __launch_bounds__(kThreads) matmul_kernel(const MatmulParams p) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ int s_pair[NT];
-    __shared__ int s_arow[NT];
-    const int nb = p.k / QK;
-    int e = 0, cnt = p.n_dense;
-    const int32_t *plist = nullptr;
-    if (p.ws) {
-        if ((int)blockIdx.y >= p.ws[p.list_word]) return;
-        e = p.ws[p.lay_list + blockIdx.y];
-        cnt = p.ws[p.lay_count + e];
-        plist = p.ws + p.lay_pairs + p.ws[p.lay_offset + e];
-    }
-    const int row0 = blockIdx.x * p.rows_per_cta;
-    const int row_end = min(p.rows, row0 + p.rows_per_cta);
-    const int8_t *wq = p.wq + (int64_t)e * p.mat_stride * p.k;
-    const uint16_t *wd = p.wd + (int64_t)e * p.mat_stride * p.ld_d;
-    const XStage xs = make_xstage(smem, NT, nb);
-    for (int pg = 0; pg < cnt; pg += NT) {
-        const int n = min(NT, cnt - pg);
-        if ((int)threadIdx.x < n) {
-            const int pr = plist ? plist[pg + threadIdx.x] : pg + (int)threadIdx.x;
-            s_pair[threadIdx.x] = pr;
-            s_arow[threadIdx.x] = (!p.ws || p.a_per_slot) ? pr : pr / p.n_used;
+template <int NT>
+__global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
+    stream_matmul_kernel(const __grid_constant__ MatmulParams p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const Ring R = ring_init(smem, p.plan);
+    const Geo g = geo_for_k(p.k);
+    const int tpm = (p.rows + g.nr - 1) / g.nr;
+    const bool routed = p.ws != nullptr;
+    griddep_launch_dependents();
+    if (routed) griddep_wait();
+    const int n_mat = routed ? p.ws[p.list_word] : 1;
+    int64_t tb, te;
+    my_tiles((int64_t)n_mat * tpm, &tb, &te);
+    if ((threadIdx.x >> 5) == kCW) {  // producer warp
+        if ((threadIdx.x & 31) == 0 && tb < te) {
+            auto src = [&](int64_t t) {
+                TileSrc ts{};
+                const int mi = (int)(t / tpm), ti = (int)(t % tpm);
+                const int e = routed ? p.ws[p.lay_list + mi] : 0;
+                const int r0 = ti * g.nr;
+                const int64_t row = (int64_t)e * p.mat_stride + r0;
+                ts.q0 = p.wq + row * p.k;
+                ts.d0 = p.wd + row * p.ld_d;
+                ts.rows0 = min(g.nr, p.rows - r0);
+                ts.k = p.k;
+                ts.ld_d = (int)p.ld_d;
+                return ts;
+            };
+            produce(R, tb, te, src, &g_err_matmul);
         }
-        __syncthreads();
-        stage_q8_rows(xs, p.aq, p.ad, p.k, s_arow, n);
-        __syncthreads();
-        run_rows<NT, R>(wq, wd, p.k, p.ld_d, p.rows, row0, row_end, xs, n, s_pair, p.y);
-        __syncthreads();
+        return;
+    }
+    if (!routed) griddep_wait();
+    const XStage xs{reinterpret_cast<int8_t *>(smem + p.plan.off_xq),
+                    reinterpret_cast<float *>(smem + p.plan.off_xd)};
+    float *part0 = reinterpret_cast<float *>(smem + p.plan.off_part);
+    const int xmax = p.plan.xmax;
+    int buf = 0, staged_mi = -1, staged_grp = -1, it = 0;
+    for (int64_t t = tb; t < te; ++t, ++it) {
+        const int s = it % R.stages;
+        mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_matmul);
+        const int mi = (int)(t / tpm), ti = (int)(t % tpm);
+        const int e = routed ? p.ws[p.lay_list + mi] : 0;
+        const int cnt = routed ? p.ws[p.lay_count + e] : p.n_dense;
+        const int32_t *plist = routed ? p.ws + p.lay_pairs + p.ws[p.lay_offset + e] : nullptr;
+        const int r0 = ti * g.nr;
+        const int rows_valid = min(g.nr, p.rows - r0);
+        const int n_grp = (cnt + xmax - 1) / xmax;
+        if (n_grp == 0) {
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
+        }
+        for (int grp = 0; grp < n_grp; ++grp) {
+            const int x0 = grp * xmax;
+            const int nx = min(xmax, cnt - x0);
+            if (mi != staged_mi || grp != staged_grp) {
+                auto arow = [&](int j) {
+                    const int pr = plist ? plist[x0 + j] : x0 + j;
+                    return (!routed || p.a_per_slot) ? pr : pr / p.n_used;
+                };
+                if (p.af)
+                    stage_f32(xs, p.af, p.k, nx, arow);
+                else
+                    stage_q8(xs, p.aq, p.ad, p.k, nx, arow);
+                named_bar_sync(kBarConsumers, kCT);
+                staged_mi = mi;
+                staged_grp = grp;
+            }
+            for (int tg = 0; tg < nx; tg += NT) {
+                const int n = min(NT, nx - tg);
+                float *part = part0 + buf * 32 * NT;
+                warp_rows_to_part<NT>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, xs, tg, n, part);
+                if (grp == n_grp - 1 && tg + NT >= nx) {  // last read of this stage
+                    __syncwarp();
+                    if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
+                }
+                named_bar_sync(kBarConsumers, kCT);
+                for (int i = threadIdx.x; i < rows_valid * n; i += kCT) {
+                    const int row = i / n;
+                    const int tt = i - row * n;
+                    const int pr = plist ? plist[x0 + tg + tt] : x0 + tg + tt;
+                    p.y[(int64_t)pr * p.rows + r0 + row] = part_sum<NT>(part, g, row, tt);
+                }
+                buf ^= 1;
+            }
+        }
     }
 }
 
-static int pick_nt(int64_t max_rows_per_group) {
-    if (max_rows_per_group <= 1) return 1;
-    if (max_rows_per_group <= 2) return 2;
-    if (max_rows_per_group <= 4) return 4;
-    return 8;
+static int g_num_sms[64];
+
+int num_sms() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (g_num_sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        g_num_sms[dev] = n;
+    }
+    return g_num_sms[dev];
 }
 
-// Rows per CTA: enough CTAs to cover the SMs several times over, in whole
-// warp row groups.
-static int pick_rows_per_cta(int64_t rows, int64_t slots, int R) {
-    const int64_t unit = (int64_t)(kThreads / 32) * R;
-    int64_t rpc = unit * 4;
-    while (rpc > unit && ((rows + rpc - 1) / rpc) * slots < 4 * 148) rpc -= unit;
-    return (int)rpc;
-}
-
-q8_status launch_matmul(const MatmulParams &base, int64_t max_group, int64_t slots,
+// max_group: the most activation rows any one matrix has (bounds NT);
+// max_tiles: an upper bound of the tile count (sizes the grid).
+q8_status launch_matmul(const MatmulParams &base, int64_t max_group, int64_t max_tiles,
                         cudaStream_t s) {
     MatmulParams p = base;
     const int nt = pick_nt(max_group);
-    const int R = (nt <= 2) ? 4 : 2;
-    p.rows_per_cta = pick_rows_per_cta(p.rows, slots, R);
-    const dim3 grid((unsigned)((p.rows + p.rows_per_cta - 1) / p.rows_per_cta), (unsigned)slots);
-    const size_t smem = (size_t)nt * xstage_bytes_per_row(p.k / QK);
-#define Q8_LAUNCH_MM(NT_, R_)                                                                \
-    do {                                                                                     \
-        if (smem > 48 * 1024)                                                                \
-            cudaFuncSetAttribute(matmul_kernel<NT_, R_>,                                     \
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);     \
-        matmul_kernel<NT_, R_><<<grid, kThreads, smem, s>>>(p);                              \
-    } while (0)
+    if (!make_plan(p.k, (int)std::min<int64_t>(max_group, kMaxXRows), nt, &p.plan))
+        Q8_FAIL(Q8_E_UNSUPPORTED, "matmul: k=%d does not fit the shared-memory plan", p.k);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * ctas_per_sm(nt), max_tiles));
     switch (nt) {
-        case 1: Q8_LAUNCH_MM(1, 4); break;
-        case 2: Q8_LAUNCH_MM(2, 4); break;
-        case 4: Q8_LAUNCH_MM(4, 2); break;
-        default: Q8_LAUNCH_MM(8, 2); break;
+        case 1: return launch_stream(stream_matmul_kernel<1>, grid, p.plan.bytes, s, p, "matmul");
+        case 2: return launch_stream(stream_matmul_kernel<2>, grid, p.plan.bytes, s, p, "matmul");
+        case 4: return launch_stream(stream_matmul_kernel<4>, grid, p.plan.bytes, s, p, "matmul");
+        default: return launch_stream(stream_matmul_kernel<8>, grid, p.plan.bytes, s, p, "matmul");
     }
-#undef Q8_LAUNCH_MM
-    return launch_status("matmul_kernel");
+}
+
+// mul_mat_id over grouping tables already written to ws.  af: fp32
+// activations instead of aq/ad (quantized while staged).
+q8_status launch_matmul_routed(const q8_tensor *W, const int8_t *aq, const uint16_t *ad,
+                               const float *af, int a_per_slot, int64_t n_tok, int32_t n_used,
+                               float *y, const int32_t *ws, cudaStream_t s) {
+    const int64_t P = n_tok * n_used;
+    const GroupLayout L = group_layout(P, W->n_mat);
+    MatmulParams p{};
+    p.wq = W->qs;
+    p.wd = W->d;
+    p.ld_d = W->ld_d;
+    p.mat_stride = W->mat_stride;
+    p.k = (int)W->k;
+    p.rows = (int)W->rows;
+    p.aq = aq;
+    p.ad = ad;
+    p.af = af;
+    p.y = y;
+    p.ws = ws;
+    p.lay_count = L.count;
+    p.lay_offset = L.offset;
+    p.lay_list = L.list_small;
+    p.lay_pairs = L.pairs;
+    p.list_word = WS_N_SMALL;
+    p.a_per_slot = a_per_slot ? 1 : 0;
+    p.n_used = n_used;
+    const Geo g = geo_for_k(p.k);
+    const int64_t tiles = std::min<int64_t>(W->n_mat, P) * ((p.rows + g.nr - 1) / g.nr);
+    return launch_matmul(p, n_tok, tiles, s);
+}
+
+// Dense matmul of fp32 (af) or Q8_0 (aq/ad) activation rows: y = W a.
+q8_status launch_matmul_dense(const q8_tensor *W, const int8_t *aq, const uint16_t *ad,
+                              const float *af, int64_t n_tok, float *y, cudaStream_t s) {
+    const Geo g = geo_for_k((int)W->k);
+    const int64_t tiles = (W->rows + g.nr - 1) / g.nr;
+    for (int64_t t0 = 0; t0 < n_tok; t0 += kMaxXRows) {
+        const int64_t nt = std::min<int64_t>(kMaxXRows, n_tok - t0);
+        MatmulParams p{};
+        p.wq = W->qs;
+        p.wd = W->d;
+        p.ld_d = W->ld_d;
+        p.mat_stride = W->mat_stride;
+        p.k = (int)W->k;
+        p.rows = (int)W->rows;
+        p.aq = aq ? aq + t0 * W->k : nullptr;
+        p.ad = ad ? ad + t0 * (W->k / QK) : nullptr;
+        p.af = af ? af + t0 * W->k : nullptr;
+        p.y = y + t0 * W->rows;
+        p.ws = nullptr;
+        p.n_dense = (int)nt;
+        q8_status st = launch_matmul(p, nt, tiles, s);
+        if (st != Q8_OK) return st;
+    }
+    return Q8_OK;
 }
 
 // ---------------------------------------------------------------------------
-// Batched GEMV: independent problems, fp32 inputs quantized in the CTA.
+// Batched GEMV: independent problems, fp32 inputs quantized while staged.
 // ---------------------------------------------------------------------------
 struct GemvProblem {
     const int8_t *wq;
     const uint16_t *wd;
     const float *x;
     float *y;
-    int64_t ld_d;
+    int ld_d;
     int k;
     int rows;
-    int rows_per_cta;
     int tile_begin;
 };
 
@@ -136,40 +247,97 @@ struct GemvBatchParams {
     int n_desc;
     int n_tok;
     int total_tiles;
-    int max_nb;
+    Plan plan;
     GemvProblem pr[Q8_MAX_GEMV_DESC];
 };
 
-template <int NT, int R>
-__global__ void __launch_bounds__(kThreads) gemv_batched_kernel(const __grid_constant__ GemvBatchParams p) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ int s_pair[NT];
-    // which problem does this tile belong to (tile_begin is increasing)
+__device__ __forceinline__ int find_problem(const GemvBatchParams &p, int64_t t) {
     int lo = 0, hi = p.n_desc - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (p.pr[mid].tile_begin <= (int)blockIdx.x) lo = mid; else hi = mid - 1;
+        if (p.pr[mid].tile_begin <= t) lo = mid; else hi = mid - 1;
     }
-    const GemvProblem &q = p.pr[lo];
-    const int tile = blockIdx.x - q.tile_begin;
-    const int row0 = tile * q.rows_per_cta;
-    const int row_end = min(q.rows, row0 + q.rows_per_cta);
-    const XStage xs = make_xstage(smem, NT, q.k / QK);
-    for (int pg = 0; pg < p.n_tok; pg += NT) {
-        const int n = min(NT, p.n_tok - pg);
-        if ((int)threadIdx.x < n) s_pair[threadIdx.x] = pg + threadIdx.x;
-        stage_f32_rows(xs, q.x + (int64_t)pg * q.k, q.k, n);
-        __syncthreads();
-        run_rows<NT, R>(q.wq, q.wd, q.k, q.ld_d, q.rows, row0, row_end, xs, n, s_pair, q.y);
-        __syncthreads();
+    return lo;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
+    gemv_batched_kernel(const __grid_constant__ GemvBatchParams p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const Ring R = ring_init(smem, p.plan);
+    griddep_launch_dependents();
+    int64_t tb, te;
+    my_tiles(p.total_tiles, &tb, &te);
+    if ((threadIdx.x >> 5) == kCW) {
+        if ((threadIdx.x & 31) == 0 && tb < te) {
+            int cur = find_problem(p, tb);
+            auto src = [&](int64_t t) {
+                while (cur + 1 < p.n_desc && p.pr[cur + 1].tile_begin <= t) ++cur;
+                const GemvProblem &q = p.pr[cur];
+                const Geo g = geo_for_k(q.k);
+                const int r0 = (int)(t - q.tile_begin) * g.nr;
+                TileSrc ts{};
+                ts.q0 = q.wq + (int64_t)r0 * q.k;
+                ts.d0 = q.wd + (int64_t)r0 * q.ld_d;
+                ts.rows0 = min(g.nr, q.rows - r0);
+                ts.k = q.k;
+                ts.ld_d = q.ld_d;
+                return ts;
+            };
+            produce(R, tb, te, src, &g_err_matmul);
+        }
+        return;
+    }
+    griddep_wait();
+    const XStage xs{reinterpret_cast<int8_t *>(smem + p.plan.off_xq),
+                    reinterpret_cast<float *>(smem + p.plan.off_xd)};
+    float *part0 = reinterpret_cast<float *>(smem + p.plan.off_part);
+    const int xmax = p.plan.xmax;
+    int buf = 0, staged = -1, staged_grp = -1, it = 0;
+    int cur = tb < te ? find_problem(p, tb) : 0;
+    for (int64_t t = tb; t < te; ++t, ++it) {
+        while (cur + 1 < p.n_desc && p.pr[cur + 1].tile_begin <= t) ++cur;
+        const GemvProblem &q = p.pr[cur];
+        const Geo g = geo_for_k(q.k);
+        const int s = it % R.stages;
+        mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_matmul);
+        const int r0 = (int)(t - q.tile_begin) * g.nr;
+        const int rows_valid = min(g.nr, q.rows - r0);
+        const int n_grp = (p.n_tok + xmax - 1) / xmax;
+        for (int grp = 0; grp < n_grp; ++grp) {
+            const int x0 = grp * xmax;
+            const int nx = min(xmax, p.n_tok - x0);
+            if (cur != staged || grp != staged_grp) {
+                stage_f32(xs, q.x, q.k, nx, [&](int j) { return x0 + j; });
+                named_bar_sync(kBarConsumers, kCT);
+                staged = cur;
+                staged_grp = grp;
+            }
+            for (int tg = 0; tg < nx; tg += NT) {
+                const int n = min(NT, nx - tg);
+                float *part = part0 + buf * 32 * NT;
+                warp_rows_to_part<NT>(R.qs(s), R.d(s), q.k, q.ld_d, g, xs, tg, n, part);
+                if (grp == n_grp - 1 && tg + NT >= nx) {
+                    __syncwarp();
+                    if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
+                }
+                named_bar_sync(kBarConsumers, kCT);
+                for (int i = threadIdx.x; i < rows_valid * n; i += kCT) {
+                    const int row = i / n;
+                    const int tt = i - row * n;
+                    q.y[(int64_t)(x0 + tg + tt) * q.rows + r0 + row] = part_sum<NT>(part, g, row, tt);
+                }
+                buf ^= 1;
+            }
+        }
     }
 }
 
 // ---------------------------------------------------------------------------
 // Test hook: per-block int32 dots through block_dot.
-// ---------------------------------------------------------------------------
 // A row index outside [0, n_w_rows) writes INT32_MIN for each of its blocks
 // and reads nothing.
+// ---------------------------------------------------------------------------
 __global__ void block_dots_kernel(const int8_t *__restrict__ wq, int k, int64_t n_w_rows,
                                   const int64_t *rows, int64_t n_rows,
                                   const int8_t *__restrict__ xq, int32_t *__restrict__ isum) {
@@ -194,34 +362,6 @@ __global__ void block_dots_kernel(const int8_t *__restrict__ wq, int k, int64_t 
     }
 }
 
-// mul_mat_id over grouping tables already written to ws by launch_group.
-q8_status launch_matmul_routed(const q8_tensor *W, const int8_t *aq, const uint16_t *ad,
-                               int a_per_slot, int64_t n_tok, int32_t n_used, float *y,
-                               const int32_t *ws, cudaStream_t s) {
-    const int64_t P = n_tok * n_used;
-    const GroupLayout L = group_layout(P, W->n_mat);
-    MatmulParams p{};
-    p.wq = W->qs;
-    p.wd = W->d;
-    p.ld_d = W->ld_d;
-    p.mat_stride = W->mat_stride;
-    p.k = (int)W->k;
-    p.rows = (int)W->rows;
-    p.aq = aq;
-    p.ad = ad;
-    p.y = y;
-    p.ws = ws;
-    p.lay_count = L.count;
-    p.lay_offset = L.offset;
-    p.lay_list = L.list_small;
-    p.lay_pairs = L.pairs;
-    p.list_word = WS_N_SMALL;
-    p.a_per_slot = a_per_slot ? 1 : 0;
-    p.n_used = n_used;
-    const int64_t slots = std::min<int64_t>(W->n_mat, P);
-    return launch_matmul(p, n_tok, slots, s);
-}
-
 }  // namespace q8
 
 using namespace q8;
@@ -233,25 +373,13 @@ q8_status q8_gemv(const q8_tensor *W, const int8_t *xq, const uint16_t *xd, int6
     q8_status st = check_tensor(W, "q8_gemv: W", true);
     if (st != Q8_OK) return st;
     Q8_REQUIRE(xq && xd && y, Q8_E_NULL, "q8_gemv: NULL pointer");
-    Q8_REQUIRE(n_tok >= 1 && n_tok <= (1 << 20), Q8_E_SHAPE, "q8_gemv: n_tok=%lld",
+    Q8_REQUIRE(n_tok >= 1 && n_tok <= 4096, Q8_E_SHAPE, "q8_gemv: n_tok=%lld (1..4096)",
                (long long)n_tok);
     Q8_REQUIRE(W->rows < (1LL << 31), Q8_E_SHAPE, "q8_gemv: rows too large");
     Q8_REQUIRE(aligned16(xq), Q8_E_ALIGN, "q8_gemv: xq must be 16-byte aligned");
     Q8_REQUIRE(((uintptr_t)xd & 1u) == 0 && ((uintptr_t)y & 3u) == 0, Q8_E_ALIGN,
                "q8_gemv: xd/y misaligned");
-    MatmulParams p{};
-    p.wq = W->qs;
-    p.wd = W->d;
-    p.ld_d = W->ld_d;
-    p.mat_stride = W->mat_stride;
-    p.k = (int)W->k;
-    p.rows = (int)W->rows;
-    p.aq = xq;
-    p.ad = xd;
-    p.y = y;
-    p.ws = nullptr;
-    p.n_dense = (int)n_tok;
-    return launch_matmul(p, n_tok, 1, (cudaStream_t)stream);
+    return launch_matmul_dense(W, xq, xd, nullptr, n_tok, y, (cudaStream_t)stream);
 }
 
 static q8_status mul_mat_id_entry(const char *fn, const q8_tensor *W, const int8_t *aq,
@@ -278,7 +406,8 @@ static q8_status mul_mat_id_entry(const char *fn, const q8_tensor *W, const int8
         st = launch_group(ids, n_tok, n_used, W->n_mat, 1 << 30, (int32_t *)ws, s);
         if (st != Q8_OK) return st;
     }
-    return launch_matmul_routed(W, aq, ad, a_per_slot, n_tok, n_used, y, (const int32_t *)ws, s);
+    return launch_matmul_routed(W, aq, ad, nullptr, a_per_slot, n_tok, n_used, y,
+                                (const int32_t *)ws, s);
 }
 
 q8_status q8_mul_mat_id(const q8_tensor *W, const int8_t *aq, const uint16_t *ad,
@@ -306,11 +435,8 @@ q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_t
     GemvBatchParams p{};
     p.n_desc = n_desc;
     p.n_tok = (int)n_tok;
-    const int nt = pick_nt(n_tok);
-    const int R = (nt <= 2) ? 4 : 2;
-    int tiles = 0, max_nb = 0;
-    int64_t total_rows = 0;
-    for (int i = 0; i < n_desc; ++i) total_rows += descs[i].W.rows;
+    int64_t tiles = 0;
+    int max_k = 32;
     for (int i = 0; i < n_desc; ++i) {
         const q8_gemv_desc &d = descs[i];
         q8_status st = check_tensor(&d.W, "q8_gemv_batched: W", true);
@@ -324,36 +450,27 @@ q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_t
         q.wd = d.W.d;
         q.x = d.x;
         q.y = d.y;
-        q.ld_d = d.W.ld_d;
+        q.ld_d = (int)d.W.ld_d;
         q.k = (int)d.W.k;
         q.rows = (int)d.W.rows;
-        // equal weight bytes per CTA across problems: ~16 KB, whole warp row groups
-        const int unit = (kThreads / 32) * R;
-        int rpc = (int)std::max<int64_t>(unit, (16384 / d.W.k) / unit * unit);
-        q.rows_per_cta = rpc;
-        q.tile_begin = tiles;
-        tiles += (int)((d.W.rows + rpc - 1) / rpc);
-        max_nb = std::max(max_nb, (int)(d.W.k / QK));
+        q.tile_begin = (int)tiles;
+        const Geo g = geo_for_k(q.k);
+        tiles += (d.W.rows + g.nr - 1) / g.nr;
+        max_k = std::max(max_k, q.k);
     }
-    p.total_tiles = tiles;
-    p.max_nb = max_nb;
-    const size_t smem = (size_t)nt * xstage_bytes_per_row(max_nb);
+    Q8_REQUIRE(tiles < (1LL << 31), Q8_E_SHAPE, "q8_gemv_batched: too many tiles");
+    p.total_tiles = (int)tiles;
+    const int nt = pick_nt(n_tok);
+    if (!make_plan(max_k, (int)std::min<int64_t>(n_tok, kMaxXRows), nt, &p.plan))
+        Q8_FAIL(Q8_E_UNSUPPORTED, "q8_gemv_batched: k=%d does not fit the plan", max_k);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * ctas_per_sm(nt), tiles));
     cudaStream_t s = (cudaStream_t)stream;
-#define Q8_LAUNCH_GB(NT_, R_)                                                                \
-    do {                                                                                     \
-        if (smem > 48 * 1024)                                                                \
-            cudaFuncSetAttribute(gemv_batched_kernel<NT_, R_>,                               \
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);     \
-        gemv_batched_kernel<NT_, R_><<<tiles, kThreads, smem, s>>>(p);                       \
-    } while (0)
     switch (nt) {
-        case 1: Q8_LAUNCH_GB(1, 4); break;
-        case 2: Q8_LAUNCH_GB(2, 4); break;
-        case 4: Q8_LAUNCH_GB(4, 2); break;
-        default: Q8_LAUNCH_GB(8, 2); break;
+        case 1: return launch_stream(gemv_batched_kernel<1>, grid, p.plan.bytes, s, p, "gemv_batched");
+        case 2: return launch_stream(gemv_batched_kernel<2>, grid, p.plan.bytes, s, p, "gemv_batched");
+        case 4: return launch_stream(gemv_batched_kernel<4>, grid, p.plan.bytes, s, p, "gemv_batched");
+        default: return launch_stream(gemv_batched_kernel<8>, grid, p.plan.bytes, s, p, "gemv_batched");
     }
-#undef Q8_LAUNCH_GB
-    return launch_status("gemv_batched_kernel");
 }
 
 q8_status q8_debug_block_dots(const q8_tensor *W, int64_t mat, const int64_t *rows,

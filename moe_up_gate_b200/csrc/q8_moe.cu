@@ -13,11 +13,9 @@
 #include <mutex>
 
 #include "q8_internal.h"
-#include "q8_tile.cuh"
+#include "q8_stream.cuh"
 
 namespace q8 {
-
-constexpr int kThreadsMoe = 256;
 
 // ---------------------------------------------------------------------------
 // Expert grouping: one CTA.  Validates ids (range, repeats within a token),
@@ -34,6 +32,8 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t *__restrict__
     int *cursor = sm_group + n_mat;
     __shared__ int s_err;
     const int P = n_tok * n_used;
+    griddep_wait();  // ids may come from, and ws may still be read by, earlier kernels
+    griddep_launch_dependents();
     for (int e = threadIdx.x; e < n_mat; e += blockDim.x) cnt[e] = 0;
     if (threadIdx.x == 0) s_err = 0;
     __syncthreads();
@@ -109,17 +109,27 @@ q8_status launch_group(const int32_t *ids, int64_t n_tok, int32_t n_used, int64_
                        int32_t big_threshold, int32_t *ws, cudaStream_t s) {
     const GroupLayout L = group_layout(n_tok * n_used, n_mat);
     const size_t smem = (size_t)2 * n_mat * sizeof(int);
-    group_kernel<<<1, 1024, smem, s>>>(ids, (int)n_tok, n_used, (int)n_mat, big_threshold, ws, L);
-    return launch_status("group_kernel");
+    return launch_pdl("group_kernel", group_kernel, dim3(1), dim3(1024), smem, s, ids, (int)n_tok,
+                      n_used, (int)n_mat, big_threshold, ws, L);
+}
+
+// Wait timeouts of the kernels in this file (read by q8_check).
+static __device__ int g_err_moe;
+
+q8_status read_wait_errors_moe(int *flags) {
+    cudaError_t e = cudaMemcpyFromSymbol(flags, g_err_moe, sizeof(int));
+    return e == cudaSuccess ? Q8_OK : Q8_E_CUDA;
 }
 
 // ---------------------------------------------------------------------------
-// Fused up/gate + SwiGLU.  CTA (tile, slot): gate rows [32*tile, 32*tile+32)
-// of expert e (the slot-th expert of the grouping list, or matrix 0 when
-// dense) and the matching up rows n_ff + r, for every pair routed to e, NT
-// pairs at a time.  Each warp takes G gate rows and their G up rows in one
-// streaming pass (2G rows through dot_rows).  The 32 h values of a pair form
-// exactly one Q8_0 block of h, quantized in the epilogue.
+// Fused up/gate + SwiGLU on the streaming engine.  A tile is nr/2 gate rows
+// [r0, r0 + nr/2) of one expert and the matching up rows n_ff + r0 ..., both
+// streamed into one stage (gate rows first, up rows from stage row nr/2), so
+// one pass over the combined weight yields g and u of every routed pair of
+// that expert; the epilogue applies h = silu(g) * u in registers.
+// Dense (ws == nullptr): matrix 0, activation rows = pairs 0..n_dense-1.
+// Routed: the experts of the grouping list; activation row of pair p is
+// p / n_used (every slot of a token reads the token's x).
 // ---------------------------------------------------------------------------
 struct UpGateParams {
     const int8_t *wq;
@@ -131,8 +141,6 @@ struct UpGateParams {
     const int8_t *xq;
     const uint16_t *xd;
     float *h;
-    int8_t *hq;
-    uint16_t *hd;
     float *g_out;
     float *u_out;
     const int32_t *ws;
@@ -140,120 +148,120 @@ struct UpGateParams {
     int list_word;
     int n_dense;
     int n_used;
+    Plan plan;
 };
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 
-template <int NT, int G>
-__global__ void __launch_bounds__(kThreadsMoe) up_gate_kernel(const UpGateParams p) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ int s_pair[NT];
-    __shared__ int s_arow[NT];
-    __shared__ float s_h[NT][32];
-    const int nb = p.k / QK;
-    int e = 0, cnt = p.n_dense;
-    const int32_t *plist = nullptr;
-    if (p.ws) {
-        if ((int)blockIdx.y >= p.ws[p.list_word]) return;
-        e = p.ws[p.lay_list + blockIdx.y];
-        cnt = p.ws[p.lay_count + e];
-        plist = p.ws + p.lay_pairs + p.ws[p.lay_offset + e];
+template <int NT>
+__global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
+    up_gate_kernel(const __grid_constant__ UpGateParams p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const Ring R = ring_init(smem, p.plan);
+    const Geo g = geo_for_k(p.k);
+    const int half_rows = g.nr / 2;
+    const int tpm = p.n_ff / half_rows;
+    const bool routed = p.ws != nullptr;
+    griddep_launch_dependents();
+    if (routed) griddep_wait();
+    const int n_mat = routed ? p.ws[p.list_word] : 1;
+    int64_t tb, te;
+    my_tiles((int64_t)n_mat * tpm, &tb, &te);
+    if ((threadIdx.x >> 5) == kCW) {  // producer warp
+        if ((threadIdx.x & 31) == 0 && tb < te) {
+            auto src = [&](int64_t t) {
+                TileSrc ts{};
+                const int mi = (int)(t / tpm), ti = (int)(t % tpm);
+                const int e = routed ? p.ws[p.lay_list + mi] : 0;
+                const int64_t gate_row = (int64_t)e * p.mat_stride + (int64_t)ti * half_rows;
+                const int64_t up_row = gate_row + p.n_ff;
+                ts.q0 = p.wq + gate_row * p.k;
+                ts.d0 = p.wd + gate_row * p.ld_d;
+                ts.rows0 = half_rows;
+                ts.q1 = p.wq + up_row * p.k;
+                ts.d1 = p.wd + up_row * p.ld_d;
+                ts.rows1 = half_rows;
+                ts.row_off1 = half_rows;
+                ts.k = p.k;
+                ts.ld_d = (int)p.ld_d;
+                return ts;
+            };
+            produce(R, tb, te, src, &g_err_moe);
+        }
+        return;
     }
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int nwarps = blockDim.x >> 5;
-    const int tile = blockIdx.x;
-    const int r_base = tile * 32;
-    const int8_t *wq = p.wq + (int64_t)e * p.mat_stride * p.k;
-    const uint16_t *wd = p.wd + (int64_t)e * p.mat_stride * p.ld_d;
-    const XStage xs = make_xstage(smem, NT, nb);
-    for (int pg = 0; pg < cnt; pg += NT) {
-        const int n = min(NT, cnt - pg);
-        if ((int)threadIdx.x < n) {
-            const int pr = plist ? plist[pg + threadIdx.x] : pg + (int)threadIdx.x;
-            s_pair[threadIdx.x] = pr;
-            s_arow[threadIdx.x] = p.ws ? pr / p.n_used : pr;
+    if (!routed) griddep_wait();
+    const XStage xs{reinterpret_cast<int8_t *>(smem + p.plan.off_xq),
+                    reinterpret_cast<float *>(smem + p.plan.off_xd)};
+    float *part0 = reinterpret_cast<float *>(smem + p.plan.off_part);
+    const int xmax = p.plan.xmax;
+    int buf = 0, staged_mi = -1, staged_grp = -1, it = 0;
+    for (int64_t t = tb; t < te; ++t, ++it) {
+        const int s = it % R.stages;
+        mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_moe);
+        const int mi = (int)(t / tpm), ti = (int)(t % tpm);
+        const int e = routed ? p.ws[p.lay_list + mi] : 0;
+        const int cnt = routed ? p.ws[p.lay_count + e] : p.n_dense;
+        const int32_t *plist = routed ? p.ws + p.lay_pairs + p.ws[p.lay_offset + e] : nullptr;
+        const int r0 = ti * half_rows;
+        const int n_grp = (cnt + xmax - 1) / xmax;
+        if (n_grp == 0) {
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
         }
-        __syncthreads();
-        stage_q8_rows(xs, p.xq, p.xd, p.k, s_arow, n);
-        __syncthreads();
-        for (int gg = warp * G; gg < 32; gg += nwarps * G) {
-            const int8_t *wrow[2 * G];
-            const uint16_t *drow[2 * G];
-#pragma unroll
-            for (int j = 0; j < G; ++j) {
-                const int64_t rg = r_base + gg + j;
-                const int64_t ru = p.n_ff + rg;
-                wrow[j] = wq + rg * p.k;
-                drow[j] = wd + rg * p.ld_d;
-                wrow[G + j] = wq + ru * p.k;
-                drow[G + j] = wd + ru * p.ld_d;
+        for (int grp = 0; grp < n_grp; ++grp) {
+            const int x0 = grp * xmax;
+            const int nx = min(xmax, cnt - x0);
+            if (mi != staged_mi || grp != staged_grp) {
+                stage_q8(xs, p.xq, p.xd, p.k, nx, [&](int j) {
+                    const int pr = plist ? plist[x0 + j] : x0 + j;
+                    return routed ? pr / p.n_used : pr;
+                });
+                named_bar_sync(kBarConsumers, kCT);
+                staged_mi = mi;
+                staged_grp = grp;
             }
-            float acc[2 * G][NT];
-#pragma unroll
-            for (int r = 0; r < 2 * G; ++r)
-#pragma unroll
-                for (int t = 0; t < NT; ++t) acc[r][t] = 0.0f;
-            dot_rows<NT, 2 * G>(wrow, drow, xs, n, lane, acc);
-            reduce_rows<NT, 2 * G>(acc);
-#pragma unroll
-            for (int j = 0; j < G; ++j)
-#pragma unroll
-                for (int t = 0; t < NT; ++t)
-                    if (lane == ((j * NT + t) & 31) && t < n) {
-                        const float g = acc[j][t];
-                        const float u = acc[G + j][t];
-                        const float hv = silu_f(g) * u;
-                        const int64_t o = (int64_t)s_pair[t] * p.n_ff + r_base + gg + j;
-                        p.h[o] = hv;
-                        s_h[t][gg + j] = hv;
-                        if (p.g_out) p.g_out[o] = g;
-                        if (p.u_out) p.u_out[o] = u;
-                    }
-        }
-        __syncthreads();
-        if (p.hq) {
-            for (int t = warp; t < n; t += nwarps) {
-                const float v = s_h[t][lane];
-                const float amax = warp_max_all(fabsf(v));
-                const float d32 = block_scale(amax);
-                const float id = block_inv_scale(d32);
-                const int64_t pr = s_pair[t];
-                p.hq[pr * p.n_ff + r_base + lane] = (int8_t)quantize_one(v, id);
-                if (lane == 0) p.hd[pr * (p.n_ff / QK) + tile] = scale_bits(d32);
+            for (int tg = 0; tg < nx; tg += NT) {
+                const int n = min(NT, nx - tg);
+                float *part = part0 + buf * 32 * NT;
+                warp_rows_to_part<NT>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, xs, tg, n, part);
+                if (grp == n_grp - 1 && tg + NT >= nx) {
+                    __syncwarp();
+                    if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
+                }
+                named_bar_sync(kBarConsumers, kCT);
+                for (int i = threadIdx.x; i < half_rows * n; i += kCT) {
+                    const int row = i / n;
+                    const int tt = i - row * n;
+                    const int pr = plist ? plist[x0 + tg + tt] : x0 + tg + tt;
+                    const float gv = part_sum<NT>(part, g, row, tt);
+                    const float uv = part_sum<NT>(part, g, row + half_rows, tt);
+                    const int64_t o = (int64_t)pr * p.n_ff + r0 + row;
+                    p.h[o] = silu_f(gv) * uv;
+                    if (p.g_out) p.g_out[o] = gv;
+                    if (p.u_out) p.u_out[o] = uv;
+                }
+                buf ^= 1;
             }
         }
-        __syncthreads();
     }
 }
 
-static int pick_nt_moe(int64_t max_group) {
-    if (max_group <= 1) return 1;
-    if (max_group <= 2) return 2;
-    if (max_group <= 4) return 4;
-    return 8;
-}
-
-static q8_status launch_up_gate(const UpGateParams &p, int64_t max_group, int64_t slots,
+static q8_status launch_up_gate(const UpGateParams &base, int64_t max_group, int64_t slots,
                                 cudaStream_t s) {
-    const int nt = pick_nt_moe(max_group);
-    const dim3 grid((unsigned)(p.n_ff / 32), (unsigned)slots);
-    const size_t smem = (size_t)nt * xstage_bytes_per_row(p.k / QK);
-#define Q8_LAUNCH_UG(NT_, G_)                                                                \
-    do {                                                                                     \
-        if (smem > 48 * 1024)                                                                \
-            cudaFuncSetAttribute(up_gate_kernel<NT_, G_>,                                    \
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);     \
-        up_gate_kernel<NT_, G_><<<grid, kThreadsMoe, smem, s>>>(p);                          \
-    } while (0)
+    UpGateParams p = base;
+    const int nt = pick_nt(max_group);
+    if (!make_plan(p.k, (int)std::min<int64_t>(max_group, kMaxXRows), nt, &p.plan))
+        Q8_FAIL(Q8_E_UNSUPPORTED, "up_gate: k=%d does not fit the shared-memory plan", p.k);
+    const Geo g = geo_for_k(p.k);
+    const int64_t tiles = slots * (p.n_ff / (g.nr / 2));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * ctas_per_sm(nt), tiles));
     switch (nt) {
-        case 1: Q8_LAUNCH_UG(1, 4); break;
-        case 2: Q8_LAUNCH_UG(2, 2); break;
-        case 4: Q8_LAUNCH_UG(4, 2); break;
-        default: Q8_LAUNCH_UG(8, 1); break;
+        case 1: return launch_stream(up_gate_kernel<1>, grid, p.plan.bytes, s, p, "up_gate");
+        case 2: return launch_stream(up_gate_kernel<2>, grid, p.plan.bytes, s, p, "up_gate");
+        case 4: return launch_stream(up_gate_kernel<4>, grid, p.plan.bytes, s, p, "up_gate");
+        default: return launch_stream(up_gate_kernel<8>, grid, p.plan.bytes, s, p, "up_gate");
     }
-#undef Q8_LAUNCH_UG
-    return launch_status("up_gate_kernel");
 }
 
 // ---------------------------------------------------------------------------
@@ -261,6 +269,8 @@ static q8_status launch_up_gate(const UpGateParams &p, int64_t max_group, int64_
 // ---------------------------------------------------------------------------
 __global__ void combine_kernel(const float *__restrict__ y, const float *__restrict__ w,
                                int n_tok, int n_used, int n_out, float *__restrict__ out) {
+    griddep_wait();
+    griddep_launch_dependents();
     const int64_t total = (int64_t)n_tok * n_out;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
          i += (int64_t)gridDim.x * blockDim.x) {
@@ -277,13 +287,13 @@ static q8_status launch_combine(const float *y, const float *w, int64_t n_tok, i
                                 int64_t n_out, float *out, cudaStream_t s) {
     const int64_t total = n_tok * n_out;
     const int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 8);
-    combine_kernel<<<blocks, 256, 0, s>>>(y, w, (int)n_tok, n_used, (int)n_out, out);
-    return launch_status("combine_kernel");
+    return launch_pdl("combine_kernel", combine_kernel, dim3((unsigned)blocks), dim3(256), 0, s, y,
+                      w, (int)n_tok, n_used, (int)n_out, out);
 }
 
 // moe_ffn workspace regions
 struct FfnLayout {
-    size_t group, xq, xd, h, hq, hd, y, total;
+    size_t group, xq, xd, h, y, total;
 };
 
 static FfnLayout ffn_layout(int64_t n_tok, int32_t n_used, int64_t n_mat, int64_t n_embd,
@@ -299,10 +309,6 @@ static FfnLayout ffn_layout(int64_t n_tok, int32_t n_used, int64_t n_mat, int64_
     o += round_up((size_t)n_tok * (n_embd / QK) * 2, 256);
     L.h = o;
     o += round_up((size_t)P * n_ff * 4, 256);
-    L.hq = o;
-    o += round_up((size_t)P * n_ff, 256);
-    L.hd = o;
-    o += round_up((size_t)P * (n_ff / QK) * 2, 256);
     L.y = o;
     o += routed ? round_up((size_t)P * n_embd * 4, 256) : 0;
     L.total = o;
@@ -348,8 +354,6 @@ static q8_status up_gate_entry(const char *fn, const q8_tensor *up_gate, const i
     p.xq = xq;
     p.xd = xd;
     p.h = h;
-    p.hq = hq;
-    p.hd = hd;
     p.g_out = g_out;
     p.u_out = u_out;
     p.n_used = n_used;
@@ -358,7 +362,11 @@ static q8_status up_gate_entry(const char *fn, const q8_tensor *up_gate, const i
                    "%s: dense call (ids NULL) needs n_mat == 1, n_used == 1", fn);
         p.ws = nullptr;
         p.n_dense = (int)n_tok;
-        return launch_up_gate(p, n_tok, 1, s);
+        st = launch_up_gate(p, n_tok, 1, s);
+        if (st != Q8_OK || hq == nullptr) return st;
+        // h -> Q8_0 with the activation quantizer (a 32-block of h spans
+        // several weight tiles, so it is not formed inside one tile)
+        return launch_quantize(h, n_tok * n_used, n_ff, hq, hd, n_ff / QK, s);
     }
     Q8_REQUIRE(up_gate->n_mat <= 4096, Q8_E_UNSUPPORTED, "%s: n_mat > 4096", fn);
     Q8_REQUIRE(ws != nullptr && aligned256(ws), Q8_E_WORKSPACE,
@@ -377,7 +385,9 @@ static q8_status up_gate_entry(const char *fn, const q8_tensor *up_gate, const i
     p.lay_list = L.list_small;
     p.lay_pairs = L.pairs;
     p.list_word = WS_N_SMALL;
-    return launch_up_gate(p, n_tok, std::min<int64_t>(up_gate->n_mat, P), s);
+    st = launch_up_gate(p, n_tok, std::min<int64_t>(up_gate->n_mat, P), s);
+    if (st != Q8_OK || hq == nullptr) return st;
+    return launch_quantize(h, P, n_ff, hq, hd, n_ff / QK, s);
 }
 
 q8_status q8_moe_up_gate_swiglu(const q8_tensor *up_gate, const int8_t *xq, const uint16_t *xd,
@@ -521,37 +531,42 @@ q8_status q8_moe_ffn(const q8_tensor *up_gate, const q8_tensor *down, const floa
     int8_t *xq = (int8_t *)(w8 + F.xq);
     uint16_t *xd = (uint16_t *)(w8 + F.xd);
     float *h = (float *)(w8 + F.h);
-    int8_t *hq = (int8_t *)(w8 + F.hq);
-    uint16_t *hd = (uint16_t *)(w8 + F.hd);
     st = q8_quantize_row(x, n_tok, n_embd, xq, xd, s);
     if (st != Q8_OK) return st;
     if (!routed) {
-        st = q8_moe_up_gate_swiglu(up_gate, xq, xd, n_tok, nullptr, 1, h, hq, hd, nullptr, nullptr,
-                                   nullptr, 0, s);
+        st = q8_moe_up_gate_swiglu(up_gate, xq, xd, n_tok, nullptr, 1, h, nullptr, nullptr,
+                                   nullptr, nullptr, nullptr, 0, s);
         if (st != Q8_OK) return st;
-        return q8_gemv(down, hq, hd, n_tok, out, s);
+        // the down projection quantizes h to Q8_0 as it stages it
+        return launch_matmul_dense(down, nullptr, nullptr, h, n_tok, out, s);
     }
     int32_t *wsg = (int32_t *)(w8 + F.group);
     const size_t gbytes = group_bytes(n_tok * n_used, up_gate->n_mat);
     // one grouping serves the gate/up and the down projection
     st = q8_moe_group(ids, n_tok, n_used, up_gate->n_mat, wsg, gbytes, s);
     if (st != Q8_OK) return st;
-    st = q8_moe_up_gate_swiglu_pregrouped(up_gate, xq, xd, n_tok, n_used, h, hq, hd, nullptr,
-                                          nullptr, wsg, gbytes, s);
+    st = q8_moe_up_gate_swiglu_pregrouped(up_gate, xq, xd, n_tok, n_used, h, nullptr, nullptr,
+                                          nullptr, nullptr, wsg, gbytes, s);
     if (st != Q8_OK) return st;
     float *y = (float *)(w8 + F.y);
-    st = q8_mul_mat_id_pregrouped(down, hq, hd, 1, n_tok, n_used, y, wsg, gbytes, s);
+    // the down projection quantizes h to Q8_0 as it stages it
+    st = launch_matmul_routed(down, nullptr, nullptr, h, 1, n_tok, n_used, y, wsg, s);
     if (st != Q8_OK) return st;
     return launch_combine(y, route_w, n_tok, n_used, n_embd, out, s);
 }
 
 q8_status q8_check(const void *ws, void *stream) {
-    Q8_REQUIRE(ws != nullptr, Q8_E_NULL, "q8_check: ws is NULL");
     cudaStream_t s = (cudaStream_t)stream;
     int32_t flags = 0;
-    cudaError_t e = cudaMemcpyAsync(&flags, ws, sizeof flags, cudaMemcpyDeviceToHost, s);
+    cudaError_t e = cudaSuccess;
+    if (ws) e = cudaMemcpyAsync(&flags, ws, sizeof flags, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) Q8_FAIL(Q8_E_CUDA, "q8_check: %s", cudaGetErrorString(e));
+    int w1 = 0, w2 = 0;
+    if (read_wait_errors_matmul(&w1) != Q8_OK || read_wait_errors_moe(&w2) != Q8_OK)
+        Q8_FAIL(Q8_E_CUDA, "q8_check: reading the kernels' wait flags failed");
+    if (w1 | w2)
+        Q8_FAIL(Q8_E_CUDA, "q8_check: a kernel gave up waiting for a shared-memory stage");
     if (flags & ERR_ID_RANGE) Q8_FAIL(Q8_E_BAD_ID, "q8_check: a routing id is out of range");
     if (flags & ERR_ID_REPEAT)
         Q8_FAIL(Q8_E_BAD_ID, "q8_check: a routing id repeats within a token");

@@ -7,8 +7,13 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <mutex>
+#include <set>
+#include <utility>
+
 #include "q8_device.cuh"
 #include "q8_internal.h"
+#include "q8_ptx.cuh"
 
 namespace q8 {
 
@@ -19,6 +24,19 @@ void set_error_detail(const char *fmt, ...) {
     va_start(ap, fmt);
     vsnprintf(g_detail, sizeof g_detail, fmt, ap);
     va_end(ap);
+}
+
+static std::mutex g_optin_mu;
+static std::set<std::pair<const void *, int>> g_optin;
+
+bool smem_opted_in(const void *kernel, int device) {
+    std::lock_guard<std::mutex> lock(g_optin_mu);
+    return g_optin.count({kernel, device}) != 0;
+}
+
+void set_smem_opted_in(const void *kernel, int device) {
+    std::lock_guard<std::mutex> lock(g_optin_mu);
+    g_optin.insert({kernel, device});
 }
 
 q8_status check_tensor(const q8_tensor *W, const char *name, bool need_single) {
@@ -49,7 +67,12 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const float *__restr
                                                             int64_t n_rows, int k,
                                                             int8_t *__restrict__ qs,
                                                             uint16_t *__restrict__ d,
-                                                            int64_t ld_d) {
+                                                            int64_t ld_d, int early) {
+    // x may come from the previous kernel, which may also still read qs/d
+    griddep_wait();
+    // Activation rows (early != 0) let the next kernel launch at once.  Packed
+    // weights do not: a streaming kernel prefetches weights before it waits.
+    if (early) griddep_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int64_t nb = k / QK;
     const int64_t total8 = n_rows * nb * 8;
@@ -82,14 +105,14 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const float *__restr
     }
 }
 
-static q8_status launch_quantize(const float *x, int64_t n_rows, int64_t k, int8_t *qs,
-                                 uint16_t *d, int64_t ld_d, cudaStream_t s) {
+q8_status launch_quantize(const float *x, int64_t n_rows, int64_t k, int8_t *qs,
+                                 uint16_t *d, int64_t ld_d, cudaStream_t s, bool weights) {
     const int64_t total8 = n_rows * (k / QK) * 8;
     int64_t blocks = (total8 + 255) / 256;
     if (blocks > 148 * 16) blocks = 148 * 16;
     if (blocks < 1) blocks = 1;
-    quantize_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, n_rows, (int)k, qs, d, ld_d);
-    return launch_status("quantize_rows_kernel");
+    return launch_pdl("quantize_rows_kernel", quantize_rows_kernel, dim3((unsigned)blocks),
+                      dim3(256), 0, s, x, n_rows, (int)k, qs, d, ld_d, weights ? 0 : 1);
 }
 
 }  // namespace q8
@@ -114,7 +137,7 @@ q8_status q8_quantize_row(const float *x, int64_t n_rows, int64_t k, int8_t *qs,
     Q8_REQUIRE(aligned16(x), Q8_E_ALIGN, "q8_quantize_row: x must be 16-byte aligned");
     Q8_REQUIRE(((uintptr_t)qs & 3u) == 0, Q8_E_ALIGN, "q8_quantize_row: qs must be 4-byte aligned");
     Q8_REQUIRE(((uintptr_t)d & 1u) == 0, Q8_E_ALIGN, "q8_quantize_row: d must be 2-byte aligned");
-    return launch_quantize(x, n_rows, k, qs, d, k / QK, (cudaStream_t)stream);
+    return launch_quantize(x, n_rows, k, qs, d, k / QK, (cudaStream_t)stream, false);
 }
 
 q8_status q8_pack(const float *w, int64_t n_rows, int64_t k, int8_t *qs, uint16_t *d,
@@ -133,7 +156,7 @@ q8_status q8_pack(const float *w, int64_t n_rows, int64_t k, int8_t *qs, uint16_
         cudaError_t e = cudaMemsetAsync(d, 0, (size_t)n_rows * ld_d * sizeof(uint16_t), s);
         if (e != cudaSuccess) Q8_FAIL(Q8_E_CUDA, "q8_pack: memset: %s", cudaGetErrorString(e));
     }
-    return launch_quantize(w, n_rows, k, qs, d, ld_d, s);
+    return launch_quantize(w, n_rows, k, qs, d, ld_d, s, true);
 }
 
 const char *q8_status_string(q8_status st) {

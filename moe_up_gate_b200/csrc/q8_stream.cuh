@@ -1,0 +1,372 @@
+// q8_stream.cuh -- the weight-streaming engine shared by every Q8_0 matmul
+// kernel of libq8 (GEMV, batched GEMV, mul_mat_id, fused up/gate + SwiGLU).
+//
+// One persistent CTA per SM: warp 8 is the producer, warps 0-7 consume.
+//  * The work is a list of weight tiles: nr consecutive rows of one matrix
+//    (or nr/2 gate rows and the nr/2 matching up rows), nr fixed by the row
+//    length k.  A CTA takes a contiguous run of tiles.
+//  * The producer's elected lane streams each tile's quants and scales into a
+//    ring of shared-memory stages with 1-D bulk copies (cp.async.bulk, no
+//    multicast), several tiles ahead; a stage is refilled once the 8 consumer
+//    warps have released it (mbarrier "empty"), and consumers learn that a
+//    stage is full from its transaction-count mbarrier ("full").
+//  * Consumers stage the activation rows of the tile's matrix in shared memory
+//    (Q8_0 rows copied, or fp32 rows quantized on the way in) when the matrix
+//    changes, compute the exact int32 block dots with dp4a, scale by
+//    d_w * d_x in fp32, reduce each row with a fixed shuffle tree and hand
+//    the row sums to the kernel's epilogue through a double-buffered
+//    shared array.
+//  * Lane mapping: lane l of a warp takes block base + l of its rows (two
+//    16-byte shared loads per row and activation row, 8 dp4a per block dot,
+//    an exact int32).  The order of every floating-point sum depends only on
+//    k, so a row gives bitwise the same result in every kernel.
+//  * Programmatic dependent launch: weights never depend on earlier kernels,
+//    so a dense producer starts streaming at once; everything that reads
+//    activations or routing tables first waits for the preceding grid.
+#pragma once
+
+#include "q8_device.cuh"
+#include "q8_internal.h"
+#include "q8_ptx.cuh"
+
+namespace q8 {
+
+constexpr int kCW = 8;                  // consumer warps
+constexpr int kCT = kCW * 32;           // consumer threads
+constexpr int kThreadsStream = kCT + 32;
+constexpr int kStageQs = 32768;         // quant bytes per stage
+constexpr int kStageD = 2048;           // scale bytes per stage (nr * ld_d * 2 <= 2048 for every k)
+constexpr int kStageBytes = kStageQs + kStageD;
+constexpr int kMaxStages = 6;
+constexpr int kSmemLimit = 227 * 1024;
+constexpr int kBarConsumers = 1;        // named barrier of the consumer warps
+constexpr int kMaxXRows = 16;           // activation rows staged at once (at most)
+
+// Tile geometry, a function of k only: rows per tile, warps per row (the
+// row's blocks are split into wpr segments, one per warp), rows per warp
+// (kCW * rpw / wpr == nr).  A warp takes rpw rows at once, so each
+// activation block it loads from shared memory serves rpw weight rows.
+struct Geo {
+    int nr, wpr, rpw;
+};
+__host__ __device__ inline Geo geo_for_k(int k) {
+    if (k <= 1024) return {32, 1, 4};
+    if (k <= 2048) return {16, 2, 4};
+    if (k <= 4096) return {8, 4, 4};
+    if (k <= 8192) return {4, 8, 4};
+    return {2, 8, 2};
+}
+
+// Shared-memory plan of one launch (offsets in bytes from the dynamic base).
+struct Plan {
+    int stages;
+    int xmax;       // activation rows the stage holds
+    int max_nb;     // blocks per activation row the stage is sized for
+    int off_full, off_empty, off_ring, off_xq, off_xd, off_part;
+    int bytes;
+};
+
+__host__ inline int plan_part_floats(int nt) { return 2 * 32 * nt; }
+
+// CTAs per SM of a streaming kernel: two for one or two activation rows per
+// pass (the second CTA hides the first one's barrier and dependency stalls),
+// one otherwise (register use).
+__host__ __device__ constexpr int ctas_per_sm(int nt) { return nt <= 2 ? 2 : 1; }
+// Shared memory one CTA may use (the SM has 228 KB; 1 KB per CTA is reserved).
+__host__ inline int smem_budget(int nt) {
+    return ctas_per_sm(nt) == 2 ? (228 * 1024) / 2 - 1024 : kSmemLimit;
+}
+
+// xrows: activation rows wanted in shared memory at once.
+__host__ inline bool make_plan(int max_k, int xrows, int nt, Plan *out) {
+    const int budget = smem_budget(nt);
+    Plan p{};
+    p.max_nb = max_k / QK;
+    int xmax = xrows < kMaxXRows ? xrows : kMaxXRows;
+    if (xmax < nt) xmax = nt;
+    for (;; xmax -= nt) {
+        const int x_bytes = xmax * max_k + ((xmax * p.max_nb * 4 + 15) / 16) * 16;
+        const int part_bytes = plan_part_floats(nt) * 4;
+        const int fixed = 2 * kMaxStages * 8 + 128 + x_bytes + part_bytes;
+        int stages = (budget - fixed) / kStageBytes;
+        if (stages > kMaxStages) stages = kMaxStages;
+        if (stages >= 2 || xmax <= nt) {
+            if (stages < 2) return false;
+            p.stages = stages;
+            p.xmax = xmax;
+            p.off_full = 0;
+            p.off_empty = kMaxStages * 8;
+            p.off_ring = 128;
+            p.off_xq = p.off_ring + stages * kStageBytes;
+            p.off_xd = p.off_xq + xmax * max_k;
+            p.off_part = p.off_xd + ((xmax * p.max_nb * 4 + 15) / 16) * 16;
+            p.bytes = p.off_part + part_bytes;
+            *out = p;
+            return true;
+        }
+    }
+}
+
+// Contiguous run of tiles for this CTA.
+__device__ __forceinline__ void my_tiles(int64_t total, int64_t *b, int64_t *e) {
+    *b = total * blockIdx.x / gridDim.x;
+    *e = total * (blockIdx.x + 1) / gridDim.x;
+}
+
+// A tile's weight source: up to two row spans of one matrix.  Span 1 (if any)
+// lands at shared row row_off1.
+struct TileSrc {
+    const int8_t *q0;
+    const uint16_t *d0;
+    int rows0;
+    const int8_t *q1;
+    const uint16_t *d1;
+    int rows1;
+    int row_off1;
+    int k;
+    int ld_d;
+};
+
+struct Ring {
+    uint64_t *full;
+    uint64_t *empty;
+    unsigned char *base;
+    int stages;
+    __device__ __forceinline__ int8_t *qs(int s) const {
+        return reinterpret_cast<int8_t *>(base + (size_t)s * kStageBytes);
+    }
+    __device__ __forceinline__ uint16_t *d(int s) const {
+        return reinterpret_cast<uint16_t *>(base + (size_t)s * kStageBytes + kStageQs);
+    }
+};
+
+__device__ __forceinline__ Ring ring_init(unsigned char *smem, const Plan &pl) {
+    Ring R;
+    R.full = reinterpret_cast<uint64_t *>(smem + pl.off_full);
+    R.empty = reinterpret_cast<uint64_t *>(smem + pl.off_empty);
+    R.base = smem + pl.off_ring;
+    R.stages = pl.stages;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < pl.stages; ++s) {
+            mbar_init(&R.full[s], 1);
+            mbar_init(&R.empty[s], kCW);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+    return R;
+}
+
+// Producer (one lane): stream tiles [tb, te) through the ring.  src(t) gives a
+// tile's spans.  Ends after the last copies have landed.
+template <class SrcFn>
+__device__ __forceinline__ void produce(const Ring &R, int64_t tb, int64_t te, SrcFn src,
+                                        int *err) {
+    int it = 0;
+    for (int64_t t = tb; t < te; ++t, ++it) {
+        const int s = it % R.stages;
+        const int round = it / R.stages;
+        if (round > 0) mbar_wait(&R.empty[s], (round - 1) & 1, err);
+        const TileSrc ts = src(t);
+        const int k = ts.k;
+        const int ld_d = ts.ld_d;
+        const uint32_t qb0 = (uint32_t)ts.rows0 * k, qb1 = (uint32_t)ts.rows1 * k;
+        const uint32_t db0 = (uint32_t)(ts.rows0 * ld_d * 2), db1 = (uint32_t)(ts.rows1 * ld_d * 2);
+        mbar_arrive_expect_tx(&R.full[s], qb0 + qb1 + db0 + db1);
+        bulk_g2s(R.qs(s), ts.q0, qb0, &R.full[s]);
+        bulk_g2s(R.d(s), ts.d0, db0, &R.full[s]);
+        if (ts.rows1 > 0) {
+            bulk_g2s(R.qs(s) + (size_t)ts.row_off1 * k, ts.q1, qb1, &R.full[s]);
+            bulk_g2s(R.d(s) + (size_t)ts.row_off1 * ld_d, ts.d1, db1, &R.full[s]);
+        }
+    }
+    const int first = it > R.stages ? it - R.stages : 0;
+    for (int j = first; j < it; ++j) mbar_wait(&R.full[j % R.stages], (j / R.stages) & 1, err);
+}
+
+// ---------------------------------------------------------------------------
+// activation staging (consumer threads only: threadIdx.x < kCT)
+// ---------------------------------------------------------------------------
+struct XStage {
+    int8_t *q;   // [xmax][k]
+    float *dx;   // [xmax][nb]
+};
+
+// Copy Q8_0 rows arow(j) of aq/ad, j < n, into the stage.
+template <class RowFn>
+__device__ __forceinline__ void stage_q8(const XStage &xs, const int8_t *__restrict__ aq,
+                                         const uint16_t *__restrict__ ad, int k, int n,
+                                         RowFn arow) {
+    const int nb = k / QK;
+    const int v_per_row = k / 16;
+    for (int i = threadIdx.x; i < n * v_per_row; i += kCT) {
+        const int j = i / v_per_row;
+        const int c = i - j * v_per_row;
+        const uint4 v = *reinterpret_cast<const uint4 *>(aq + (int64_t)arow(j) * k + c * 16);
+        *reinterpret_cast<uint4 *>(xs.q + (size_t)j * k + c * 16) = v;
+    }
+    for (int i = threadIdx.x; i < n * nb; i += kCT) {
+        const int j = i / nb;
+        const int b = i - j * nb;
+        xs.dx[(size_t)j * nb + b] = scale_value(ad[(int64_t)arow(j) * nb + b]);
+    }
+}
+
+// Quantize fp32 rows arow(j) of af (k floats apart), j < n, into the stage,
+// one warp per 32-block, by the Q8_0 rule.
+template <class RowFn>
+__device__ __forceinline__ void stage_f32(const XStage &xs, const float *__restrict__ af, int k,
+                                          int n, RowFn arow) {
+    const int nb = k / QK;
+    const int lane = threadIdx.x & 31;
+    for (int blk = threadIdx.x >> 5; blk < n * nb; blk += kCW) {
+        const int j = blk / nb;
+        const int b = blk - j * nb;
+        const float v = af[(int64_t)arow(j) * k + b * QK + lane];
+        const float amax = warp_max_all(fabsf(v));
+        const float d32 = block_scale(amax);
+        const float id = block_inv_scale(d32);
+        xs.q[(size_t)j * k + b * QK + lane] = (int8_t)quantize_one(v, id);
+        if (lane == 0) xs.dx[(size_t)j * nb + b] = scale_value(scale_bits(d32));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// the dot engine
+// ---------------------------------------------------------------------------
+
+// Exact float of an int32 with |v| < 2^22: v + 1.5 * 2^23 is formed in the
+// float's bit pattern (ulp 1 in [2^23, 2^24)), then 1.5 * 2^23 is subtracted
+// exactly.  Keeps the conversion on the integer and FMA pipes.
+__device__ __forceinline__ float small_int_to_float(int v) {
+    return __int_as_float(v + 0x4B400000) - 12582912.0f;
+}
+
+// acc[r][t] = sum over this warp's blocks of row (row0 + r) of the stage with
+// activation row (xrow0 + t), t < n; every lane ends with the full sums.
+// Lane l takes block base + l (both 16-byte halves), so each block dot is
+// 8 dp4a in one lane; |isum| <= 32 * 128 * 128 < 2^22.
+template <int NT, int RPW>
+__device__ __forceinline__ void dot_rows(const int8_t *sq, const uint16_t *sd, int k, int ld_d,
+                                         int row0, int seg, int wpr, const XStage &xs, int xrow0,
+                                         int n, float (&acc)[RPW][NT]) {
+    const int lane = threadIdx.x & 31;
+    const int nb = k / QK;
+    // Lanes 4-7 of every quarter warp load the upper 16 bytes of their block
+    // first: a quarter warp's first (and second) loads then fall on 8 distinct
+    // 16-byte bank groups (no bank conflicts).  The int32 sum of the two
+    // halves does not depend on the order.
+    const int h0 = ((lane >> 2) & 1) * 16;
+    const int h1 = 16 - h0;
+#pragma unroll
+    for (int r = 0; r < RPW; ++r)
+#pragma unroll
+        for (int t = 0; t < NT; ++t) acc[r][t] = 0.0f;
+    for (int base = seg * 32; base < nb; base += 32 * wpr) {
+        const int kb = base + lane;
+        if (kb < nb) {
+            uint4 w0[RPW], w1[RPW];
+            float dw[RPW];
+#pragma unroll
+            for (int r = 0; r < RPW; ++r) {
+                const int8_t *p = sq + (size_t)(row0 + r) * k + kb * QK;
+                w0[r] = *reinterpret_cast<const uint4 *>(p + h0);
+                w1[r] = *reinterpret_cast<const uint4 *>(p + h1);
+                dw[r] = scale_value(sd[(size_t)(row0 + r) * ld_d + kb]);
+            }
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                if (t < n) {
+                    const int8_t *xp = xs.q + (size_t)(xrow0 + t) * k + kb * QK;
+                    const uint4 x0 = *reinterpret_cast<const uint4 *>(xp + h0);
+                    const uint4 x1 = *reinterpret_cast<const uint4 *>(xp + h1);
+                    const float dx = xs.dx[(size_t)(xrow0 + t) * nb + kb];
+#pragma unroll
+                    for (int r = 0; r < RPW; ++r) {
+                        const int s = block_dot(w0[r], w1[r], x0, x1);
+                        acc[r][t] = fmaf(dw[r] * dx, small_int_to_float(s), acc[r][t]);
+                    }
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < RPW; ++r)
+#pragma unroll
+        for (int t = 0; t < NT; ++t) acc[r][t] = warp_sum_all(acc[r][t]);
+}
+
+// Computes this warp's rows of a stage for activation rows [xrow0, xrow0+n)
+// and writes the warp partial sums to part[(row * wpr + seg) * NT + t].
+template <int NT>
+__device__ __forceinline__ void warp_rows_to_part(const int8_t *sq, const uint16_t *sd, int k,
+                                                  int ld_d, const Geo &g, const XStage &xs,
+                                                  int xrow0, int n, float *part) {
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int seg = warp % g.wpr;
+    const int row0 = (warp / g.wpr) * g.rpw;
+#define Q8_ROWS_CASE(RPW_)                                                                    \
+    {                                                                                         \
+        float acc[RPW_][NT];                                                                  \
+        dot_rows<NT, RPW_>(sq, sd, k, ld_d, row0, seg, g.wpr, xs, xrow0, n, acc);             \
+        _Pragma("unroll") for (int r = 0; r < RPW_; ++r)                                      \
+            _Pragma("unroll") for (int t = 0; t < NT; ++t) if (lane == ((r * NT + t) & 31))   \
+                part[((row0 + r) * g.wpr + seg) * NT + t] = acc[r][t];                        \
+    }
+    if (g.rpw == 4) Q8_ROWS_CASE(4)
+    else if (g.rpw == 2) Q8_ROWS_CASE(2)
+    else Q8_ROWS_CASE(1)
+#undef Q8_ROWS_CASE
+}
+
+// Row sum of tile row `row`, activation t, from the warp partials (seg order).
+template <int NT>
+__device__ __forceinline__ float part_sum(const float *part, const Geo &g, int row, int t) {
+    float v = part[(row * g.wpr) * NT + t];
+    for (int sgi = 1; sgi < g.wpr; ++sgi) v += part[(row * g.wpr + sgi) * NT + t];
+    return v;
+}
+
+// Launch a streaming kernel (kThreadsStream threads) with programmatic stream
+// serialization: the kernel itself waits for the preceding grid before it
+// reads anything that grid may write.
+template <class P>
+__host__ inline q8_status launch_stream(void (*kern)(P), int grid, size_t smem, cudaStream_t s,
+                                        const P &params, const char *what) {
+    // opt in to the full shared memory once per kernel and device (not per
+    // launch, so that launches inside a stream capture make no attribute calls)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        Q8_FAIL(Q8_E_CUDA, "%s: no current device", what);
+    if (!smem_opted_in((const void *)kern, dev)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSmemLimit);
+        if (e != cudaSuccess)
+            Q8_FAIL(Q8_E_CUDA, "%s: shared-memory attribute: %s", what, cudaGetErrorString(e));
+        set_smem_opted_in((const void *)kern, dev);
+    }
+    if (smem > (size_t)kSmemLimit) Q8_FAIL(Q8_E_UNSUPPORTED, "%s: plan exceeds shared memory", what);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreadsStream);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, params);
+    if (e != cudaSuccess) Q8_FAIL(Q8_E_CUDA, "%s: launch: %s", what, cudaGetErrorString(e));
+    return Q8_OK;
+}
+
+__host__ inline int pick_nt(int64_t rows_per_group) {
+    if (rows_per_group <= 1) return 1;
+    if (rows_per_group <= 2) return 2;
+    if (rows_per_group <= 4) return 4;
+    return 8;
+}
+
+}  // namespace q8
