@@ -386,7 +386,11 @@ class MoeWorkload:
             self.step_bytes.append(tot)
             self.up_gate_bytes.append(ug / layers)
         self.tokens_per_step = tokens
-        self.launches_per_step = layers * (5 if self.routed else 3)
+        self.small = P <= 1024 and E <= 512
+        if self.small:
+            self.launches_per_step = layers * (3 if self.routed else 2)
+        else:
+            self.launches_per_step = layers * (5 if self.routed else 3)
         self.dominant_launches = layers
         self.h2d_bytes = self.x_host[0].numel() * 4 + (
             (self.ids_host[0].numel() * 4 + self.p_host[0].numel() * 4) if self.routed else 0)
@@ -403,6 +407,25 @@ class MoeWorkload:
         s = i % self.sets if input_set is None else input_set
         layers = self.Lc[i % self.copies]
         T = self.T
+        if self.small:
+            # small batches: the fp32 calls (x and h quantized inside the
+            # kernels, routing grouped in every CTA), the same kernels
+            # q8_moe_ffn runs: routed 3 launches per layer, dense 2
+            for l, (UG, DN) in enumerate(layers):
+                x = self.x[s][l]
+                if self.routed:
+                    ids = self.ids[s][l]
+                    marks.begin()
+                    q8.moe_up_gate_swiglu_fp32(UG, x, ids, h=self.h)
+                    marks.end()
+                    q8.mul_mat_id_fp32(DN, self.h, ids, True, y=self.y)
+                    q8.moe_combine(self.y, self.p[s][l], out=self.out[l])
+                else:
+                    marks.begin()
+                    q8.moe_up_gate_swiglu_fp32(UG, x, None, h=self.h)
+                    marks.end()
+                    q8.gemv_batched([(DN, self.h, self.out[l])], n_tok=T)
+            return
         for l, (UG, DN) in enumerate(layers):
             x = self.x[s][l]
             q8._call("q8_quantize_row", q8._ptr(x), T, UG.k, q8._ptr(self.xq), q8._ptr(self.xd),

@@ -222,6 +222,38 @@ q8_status q8_mul_mat_id_pregrouped(const q8_tensor *W, const int8_t *aq, const u
                                    const void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * q8_moe_up_gate_swiglu_fp32 -- q8_moe_up_gate_swiglu for fp32 activations and
+ * small batches, with no workspace: each x row is quantized to Q8_0 inside
+ * the kernel (bit-exact with q8_quantize_row) and, when ids are given, every
+ * CTA groups the routed pairs itself.  One launch.
+ *  up_gate: as in q8_moe_up_gate_swiglu.  x: fp32 [n_tok][k], 16-byte aligned.
+ *  ids: [n_tok][n_used] or NULL (dense: n_mat == 1, n_used == 1).
+ *  Limits: n_tok * n_used <= Q8_SMALL_BATCH_PAIRS, n_mat <= Q8_SMALL_BATCH_MATS
+ *  (else Q8_E_UNSUPPORTED: use the workspace calls).
+ *  h: out fp32 [n_tok][n_used][n_ff].
+ *  err_word: optional device int32; receives the routing-id error flags
+ *  (nonzero: an id out of range or repeated in a token; pairs with an
+ *  out-of-range id are left unwritten).  Pass the first word of a routed
+ *  workspace to have q8_check report them.
+ */
+#define Q8_SMALL_BATCH_PAIRS 1024
+#define Q8_SMALL_BATCH_MATS 512
+q8_status q8_moe_up_gate_swiglu_fp32(const q8_tensor *up_gate, const float *x, int64_t n_tok,
+                                     const int32_t *ids, int32_t n_used, float *h,
+                                     int32_t *err_word, void *stream);
+
+/*
+ * q8_mul_mat_id_fp32 -- q8_mul_mat_id for fp32 activations and small
+ * batches, with no workspace (activation rows quantized to Q8_0 inside the
+ * kernel; routed pairs grouped in every CTA).  Arguments as in
+ * q8_mul_mat_id, a: fp32 rows (per slot or per token), 16-byte aligned; the
+ * limits and err_word of q8_moe_up_gate_swiglu_fp32.
+ */
+q8_status q8_mul_mat_id_fp32(const q8_tensor *W, const float *a, int32_t a_per_slot,
+                             int64_t n_tok, const int32_t *ids, int32_t n_used, float *y,
+                             int32_t *err_word, void *stream);
+
+/*
  * q8_moe_up_gate_swiglu_noalloc -- q8_moe_up_gate_swiglu for callers that
  * cannot allocate device memory (no counterpart on the pages: this is a
  * library convenience, not part of the method).  Some callers cannot call

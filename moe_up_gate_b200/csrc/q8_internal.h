@@ -116,6 +116,14 @@ q8_status launch_matmul_routed(const q8_tensor *W, const int8_t *aq, const uint1
                                float *y, const int32_t *ws, cudaStream_t s);
 q8_status launch_matmul_dense(const q8_tensor *W, const int8_t *aq, const uint16_t *ad,
                               const float *af, int64_t n_tok, float *y, cudaStream_t s);
+q8_status launch_matmul_routed_ids(const q8_tensor *W, const int8_t *aq, const uint16_t *ad,
+                                   const float *af, int a_per_slot, int64_t n_tok,
+                                   int32_t n_used, const int32_t *ids, float *y,
+                                   int32_t *err_out, cudaStream_t s);
+
+// Batches small enough for the grouping to be built inside each CTA.
+constexpr int64_t kCtaGroupMaxPairs = Q8_SMALL_BATCH_PAIRS;
+constexpr int64_t kCtaGroupMaxMats = Q8_SMALL_BATCH_MATS;
 
 // Wait-timeout flags latched by the streaming kernels of each file.
 q8_status read_wait_errors_matmul(int *flags);

@@ -44,11 +44,16 @@ struct MatmulParams {
     const float *af;
     float *y;
     const int32_t *ws;
-    int64_t lay_count, lay_offset, lay_list, lay_pairs;
+    int64_t lay_count, lay_offset, lay_list, lay_pairs, lay_big;
     int list_word;
     int n_dense;
     int a_per_slot;
     int n_used;
+    // routed with the grouping built in each CTA from ids (ws unused)
+    const int32_t *ids;
+    int n_tok;
+    int n_mat;
+    int32_t *err_out;
     Plan plan;
 };
 
@@ -59,10 +64,24 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     const Ring R = ring_init(smem, p.plan);
     const Geo g = geo_for_k(p.k);
     const int tpm = (p.rows + g.nr - 1) / g.nr;
-    const bool routed = p.ws != nullptr;
     griddep_launch_dependents();
-    if (routed) griddep_wait();
-    const int n_mat = routed ? p.ws[p.list_word] : 1;
+    const int32_t *tab = p.ws;
+    if (p.ids) {
+        griddep_wait();
+        int32_t *stab = reinterpret_cast<int32_t *>(smem + p.plan.off_tab);
+        GroupLayout L{};
+        L.count = p.lay_count;
+        L.offset = p.lay_offset;
+        L.list_small = p.lay_list;
+        L.list_big = p.lay_big;
+        L.pairs = p.lay_pairs;
+        cta_group(p.ids, p.n_tok, p.n_used, p.n_mat, L, stab, p.err_out);
+        tab = stab;
+    } else if (tab) {
+        griddep_wait();
+    }
+    const bool routed = tab != nullptr;
+    const int n_mat = routed ? tab[p.list_word] : 1;
     int64_t tb, te;
     my_tiles((int64_t)n_mat * tpm, &tb, &te);
     if ((threadIdx.x >> 5) == kCW) {  // producer warp
@@ -70,7 +89,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             auto src = [&](int64_t t) {
                 TileSrc ts{};
                 const int mi = (int)(t / tpm), ti = (int)(t % tpm);
-                const int e = routed ? p.ws[p.lay_list + mi] : 0;
+                const int e = routed ? tab[p.lay_list + mi] : 0;
                 const int r0 = ti * g.nr;
                 const int64_t row = (int64_t)e * p.mat_stride + r0;
                 ts.q0 = p.wq + row * p.k;
@@ -94,9 +113,9 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_matmul);
         const int mi = (int)(t / tpm), ti = (int)(t % tpm);
-        const int e = routed ? p.ws[p.lay_list + mi] : 0;
-        const int cnt = routed ? p.ws[p.lay_count + e] : p.n_dense;
-        const int32_t *plist = routed ? p.ws + p.lay_pairs + p.ws[p.lay_offset + e] : nullptr;
+        const int e = routed ? tab[p.lay_list + mi] : 0;
+        const int cnt = routed ? tab[p.lay_count + e] : p.n_dense;
+        const int32_t *plist = routed ? tab + p.lay_pairs + tab[p.lay_offset + e] : nullptr;
         const int r0 = ti * g.nr;
         const int rows_valid = min(g.nr, p.rows - r0);
         const int n_grp = (cnt + xmax - 1) / xmax;
@@ -122,7 +141,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             }
             for (int tg = 0; tg < nx; tg += NT) {
                 const int n = min(NT, nx - tg);
-                float *part = part0 + buf * 32 * NT;
+                float *part = part0 + buf * kPartRows * NT;
                 warp_rows_to_part<NT>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, xs, tg, n, part);
                 if (grp == n_grp - 1 && tg + NT >= nx) {  // last read of this stage
                     __syncwarp();
@@ -161,7 +180,12 @@ q8_status launch_matmul(const MatmulParams &base, int64_t max_group, int64_t max
                         cudaStream_t s) {
     MatmulParams p = base;
     const int nt = pick_nt(max_group);
-    if (!make_plan(p.k, (int)std::min<int64_t>(max_group, kMaxXRows), nt, &p.plan))
+    const int tab_words =
+        p.ids ? (int)group_layout((int64_t)p.n_tok * p.n_used, p.n_mat).words : 0;
+    int tq, td;
+    tile_bytes(geo_for_k(p.k), p.k, p.ld_d, &tq, &td);
+    if (!make_plan(tq, td, p.k, (int)std::min<int64_t>(max_group, kMaxXRows), nt, &p.plan,
+                   tab_words))
         Q8_FAIL(Q8_E_UNSUPPORTED, "matmul: k=%d does not fit the shared-memory plan", p.k);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * ctas_per_sm(nt), max_tiles));
     switch (nt) {
@@ -198,6 +222,43 @@ q8_status launch_matmul_routed(const q8_tensor *W, const int8_t *aq, const uint1
     p.list_word = WS_N_SMALL;
     p.a_per_slot = a_per_slot ? 1 : 0;
     p.n_used = n_used;
+    const Geo g = geo_for_k(p.k);
+    const int64_t tiles = std::min<int64_t>(W->n_mat, P) * ((p.rows + g.nr - 1) / g.nr);
+    return launch_matmul(p, n_tok, tiles, s);
+}
+
+// mul_mat_id with the grouping built in each CTA from ids (small batches);
+// routing-id errors go to *err_out.
+q8_status launch_matmul_routed_ids(const q8_tensor *W, const int8_t *aq, const uint16_t *ad,
+                                   const float *af, int a_per_slot, int64_t n_tok,
+                                   int32_t n_used, const int32_t *ids, float *y,
+                                   int32_t *err_out, cudaStream_t s) {
+    const int64_t P = n_tok * n_used;
+    const GroupLayout L = group_layout(P, W->n_mat);
+    MatmulParams p{};
+    p.wq = W->qs;
+    p.wd = W->d;
+    p.ld_d = W->ld_d;
+    p.mat_stride = W->mat_stride;
+    p.k = (int)W->k;
+    p.rows = (int)W->rows;
+    p.aq = aq;
+    p.ad = ad;
+    p.af = af;
+    p.y = y;
+    p.ws = nullptr;
+    p.lay_count = L.count;
+    p.lay_offset = L.offset;
+    p.lay_list = L.list_small;
+    p.lay_big = L.list_big;
+    p.lay_pairs = L.pairs;
+    p.list_word = WS_N_SMALL;
+    p.a_per_slot = a_per_slot ? 1 : 0;
+    p.n_used = n_used;
+    p.ids = ids;
+    p.n_tok = (int)n_tok;
+    p.n_mat = (int)W->n_mat;
+    p.err_out = err_out;
     const Geo g = geo_for_k(p.k);
     const int64_t tiles = std::min<int64_t>(W->n_mat, P) * ((p.rows + g.nr - 1) / g.nr);
     return launch_matmul(p, n_tok, tiles, s);
@@ -315,7 +376,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             }
             for (int tg = 0; tg < nx; tg += NT) {
                 const int n = min(NT, nx - tg);
-                float *part = part0 + buf * 32 * NT;
+                float *part = part0 + buf * kPartRows * NT;
                 warp_rows_to_part<NT>(R.qs(s), R.d(s), q.k, q.ld_d, g, xs, tg, n, part);
                 if (grp == n_grp - 1 && tg + NT >= nx) {
                     __syncwarp();
@@ -436,7 +497,7 @@ q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_t
     p.n_desc = n_desc;
     p.n_tok = (int)n_tok;
     int64_t tiles = 0;
-    int max_k = 32;
+    int max_k = 32, max_tq = 0, max_td = 0;
     for (int i = 0; i < n_desc; ++i) {
         const q8_gemv_desc &d = descs[i];
         q8_status st = check_tensor(&d.W, "q8_gemv_batched: W", true);
@@ -457,11 +518,15 @@ q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_t
         const Geo g = geo_for_k(q.k);
         tiles += (d.W.rows + g.nr - 1) / g.nr;
         max_k = std::max(max_k, q.k);
+        int tq, td;
+        tile_bytes(g, q.k, q.ld_d, &tq, &td);
+        max_tq = std::max(max_tq, tq);
+        max_td = std::max(max_td, td);
     }
     Q8_REQUIRE(tiles < (1LL << 31), Q8_E_SHAPE, "q8_gemv_batched: too many tiles");
     p.total_tiles = (int)tiles;
     const int nt = pick_nt(n_tok);
-    if (!make_plan(max_k, (int)std::min<int64_t>(n_tok, kMaxXRows), nt, &p.plan))
+    if (!make_plan(max_tq, max_td, max_k, (int)std::min<int64_t>(n_tok, kMaxXRows), nt, &p.plan))
         Q8_FAIL(Q8_E_UNSUPPORTED, "q8_gemv_batched: k=%d does not fit the plan", max_k);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * ctas_per_sm(nt), tiles));
     cudaStream_t s = (cudaStream_t)stream;

@@ -140,14 +140,20 @@ struct UpGateParams {
     int n_ff;
     const int8_t *xq;
     const uint16_t *xd;
+    const float *xf;  // fp32 x instead of xq/xd (quantized while staged)
     float *h;
     float *g_out;
     float *u_out;
     const int32_t *ws;
-    int64_t lay_count, lay_offset, lay_list, lay_pairs;
+    int64_t lay_count, lay_offset, lay_list, lay_pairs, lay_big;
     int list_word;
     int n_dense;
     int n_used;
+    // routed with the grouping built in each CTA from ids (ws unused)
+    const int32_t *ids;
+    int n_tok;
+    int n_mat;
+    int32_t *err_out;
     Plan plan;
 };
 
@@ -158,13 +164,27 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     up_gate_kernel(const __grid_constant__ UpGateParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
     const Ring R = ring_init(smem, p.plan);
-    const Geo g = geo_for_k(p.k);
+    const Geo g = geo_pair_for_k(p.k);
     const int half_rows = g.nr / 2;
     const int tpm = p.n_ff / half_rows;
-    const bool routed = p.ws != nullptr;
     griddep_launch_dependents();
-    if (routed) griddep_wait();
-    const int n_mat = routed ? p.ws[p.list_word] : 1;
+    const int32_t *tab = p.ws;
+    if (p.ids) {
+        griddep_wait();
+        int32_t *stab = reinterpret_cast<int32_t *>(smem + p.plan.off_tab);
+        GroupLayout L{};
+        L.count = p.lay_count;
+        L.offset = p.lay_offset;
+        L.list_small = p.lay_list;
+        L.list_big = p.lay_big;
+        L.pairs = p.lay_pairs;
+        cta_group(p.ids, p.n_tok, p.n_used, p.n_mat, L, stab, p.err_out);
+        tab = stab;
+    } else if (tab) {
+        griddep_wait();
+    }
+    const bool routed = tab != nullptr;
+    const int n_mat = routed ? tab[p.list_word] : 1;
     int64_t tb, te;
     my_tiles((int64_t)n_mat * tpm, &tb, &te);
     if ((threadIdx.x >> 5) == kCW) {  // producer warp
@@ -172,7 +192,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             auto src = [&](int64_t t) {
                 TileSrc ts{};
                 const int mi = (int)(t / tpm), ti = (int)(t % tpm);
-                const int e = routed ? p.ws[p.lay_list + mi] : 0;
+                const int e = routed ? tab[p.lay_list + mi] : 0;
                 const int64_t gate_row = (int64_t)e * p.mat_stride + (int64_t)ti * half_rows;
                 const int64_t up_row = gate_row + p.n_ff;
                 ts.q0 = p.wq + gate_row * p.k;
@@ -200,9 +220,9 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_moe);
         const int mi = (int)(t / tpm), ti = (int)(t % tpm);
-        const int e = routed ? p.ws[p.lay_list + mi] : 0;
-        const int cnt = routed ? p.ws[p.lay_count + e] : p.n_dense;
-        const int32_t *plist = routed ? p.ws + p.lay_pairs + p.ws[p.lay_offset + e] : nullptr;
+        const int e = routed ? tab[p.lay_list + mi] : 0;
+        const int cnt = routed ? tab[p.lay_count + e] : p.n_dense;
+        const int32_t *plist = routed ? tab + p.lay_pairs + tab[p.lay_offset + e] : nullptr;
         const int r0 = ti * half_rows;
         const int n_grp = (cnt + xmax - 1) / xmax;
         if (n_grp == 0) {
@@ -213,17 +233,21 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             const int x0 = grp * xmax;
             const int nx = min(xmax, cnt - x0);
             if (mi != staged_mi || grp != staged_grp) {
-                stage_q8(xs, p.xq, p.xd, p.k, nx, [&](int j) {
+                auto arow = [&](int j) {
                     const int pr = plist ? plist[x0 + j] : x0 + j;
                     return routed ? pr / p.n_used : pr;
-                });
+                };
+                if (p.xf)
+                    stage_f32(xs, p.xf, p.k, nx, arow);
+                else
+                    stage_q8(xs, p.xq, p.xd, p.k, nx, arow);
                 named_bar_sync(kBarConsumers, kCT);
                 staged_mi = mi;
                 staged_grp = grp;
             }
             for (int tg = 0; tg < nx; tg += NT) {
                 const int n = min(NT, nx - tg);
-                float *part = part0 + buf * 32 * NT;
+                float *part = part0 + buf * kPartRows * NT;
                 warp_rows_to_part<NT>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, xs, tg, n, part);
                 if (grp == n_grp - 1 && tg + NT >= nx) {
                     __syncwarp();
@@ -251,9 +275,14 @@ static q8_status launch_up_gate(const UpGateParams &base, int64_t max_group, int
                                 cudaStream_t s) {
     UpGateParams p = base;
     const int nt = pick_nt(max_group);
-    if (!make_plan(p.k, (int)std::min<int64_t>(max_group, kMaxXRows), nt, &p.plan))
+    const int tab_words =
+        p.ids ? (int)group_layout((int64_t)p.n_tok * p.n_used, p.n_mat).words : 0;
+    int tq, td;
+    tile_bytes(geo_pair_for_k(p.k), p.k, p.ld_d, &tq, &td);
+    if (!make_plan(tq, td, p.k, (int)std::min<int64_t>(max_group, kMaxXRows), nt, &p.plan,
+                   tab_words))
         Q8_FAIL(Q8_E_UNSUPPORTED, "up_gate: k=%d does not fit the shared-memory plan", p.k);
-    const Geo g = geo_for_k(p.k);
+    const Geo g = geo_pair_for_k(p.k);
     const int64_t tiles = slots * (p.n_ff / (g.nr / 2));
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * ctas_per_sm(nt), tiles));
     switch (nt) {
@@ -481,6 +510,76 @@ q8_status q8_moe_up_gate_swiglu_noalloc(const q8_tensor *up_gate, const int8_t *
                          u_out, scratch, Q8_NOALLOC_SCRATCH_BYTES, (cudaStream_t)stream);
 }
 
+q8_status q8_moe_up_gate_swiglu_fp32(const q8_tensor *up_gate, const float *x, int64_t n_tok,
+                                     const int32_t *ids, int32_t n_used, float *h,
+                                     int32_t *err_word, void *stream) {
+    const char *fn = "q8_moe_up_gate_swiglu_fp32";
+    q8_status st = check_tensor(up_gate, fn, false);
+    if (st != Q8_OK) return st;
+    Q8_REQUIRE(x && h, Q8_E_NULL, "%s: NULL pointer", fn);
+    Q8_REQUIRE(up_gate->rows % 64 == 0, Q8_E_SHAPE,
+               "%s: rows=%lld must be 2*n_ff with n_ff %% 32 == 0", fn, (long long)up_gate->rows);
+    Q8_REQUIRE(n_tok >= 1 && n_used >= 1 && n_used <= Q8_MAX_USED, Q8_E_SHAPE,
+               "%s: n_tok=%lld n_used=%d", fn, (long long)n_tok, n_used);
+    Q8_REQUIRE(aligned16(x), Q8_E_ALIGN, "%s: x must be 16-byte aligned", fn);
+    Q8_REQUIRE(((uintptr_t)ids & 3u) == 0 && ((uintptr_t)err_word & 3u) == 0, Q8_E_ALIGN,
+               "%s: ids/err_word misaligned", fn);
+    Q8_REQUIRE(n_tok * n_used <= kCtaGroupMaxPairs && up_gate->n_mat <= kCtaGroupMaxMats,
+               Q8_E_UNSUPPORTED, "%s: batch of %lld pairs over %lld matrices is above the "
+               "small-batch limits (%lld, %lld)", fn, (long long)(n_tok * n_used),
+               (long long)up_gate->n_mat, (long long)kCtaGroupMaxPairs,
+               (long long)kCtaGroupMaxMats);
+    const int64_t n_ff = up_gate->rows / 2;
+    UpGateParams p{};
+    p.wq = up_gate->qs;
+    p.wd = up_gate->d;
+    p.ld_d = up_gate->ld_d;
+    p.mat_stride = up_gate->mat_stride;
+    p.k = (int)up_gate->k;
+    p.n_ff = (int)n_ff;
+    p.xf = x;
+    p.h = h;
+    p.n_used = n_used;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (ids == nullptr) {
+        Q8_REQUIRE(up_gate->n_mat == 1 && n_used == 1, Q8_E_SHAPE,
+                   "%s: dense call (ids NULL) needs n_mat == 1, n_used == 1", fn);
+        p.n_dense = (int)n_tok;
+        return launch_up_gate(p, n_tok, 1, s);
+    }
+    const GroupLayout L = group_layout(n_tok * n_used, up_gate->n_mat);
+    p.lay_count = L.count;
+    p.lay_offset = L.offset;
+    p.lay_list = L.list_small;
+    p.lay_big = L.list_big;
+    p.lay_pairs = L.pairs;
+    p.list_word = WS_N_SMALL;
+    p.ids = ids;
+    p.n_tok = (int)n_tok;
+    p.n_mat = (int)up_gate->n_mat;
+    p.err_out = err_word;
+    return launch_up_gate(p, n_tok, std::min<int64_t>(up_gate->n_mat, n_tok * n_used), s);
+}
+
+q8_status q8_mul_mat_id_fp32(const q8_tensor *W, const float *a, int32_t a_per_slot,
+                             int64_t n_tok, const int32_t *ids, int32_t n_used, float *y,
+                             int32_t *err_word, void *stream) {
+    const char *fn = "q8_mul_mat_id_fp32";
+    q8_status st = check_tensor(W, fn, false);
+    if (st != Q8_OK) return st;
+    Q8_REQUIRE(a && ids && y, Q8_E_NULL, "%s: NULL pointer", fn);
+    Q8_REQUIRE(n_tok >= 1 && n_used >= 1 && n_used <= Q8_MAX_USED, Q8_E_SHAPE,
+               "%s: n_tok=%lld n_used=%d", fn, (long long)n_tok, n_used);
+    Q8_REQUIRE(W->rows < (1LL << 31), Q8_E_SHAPE, "%s: rows too large", fn);
+    Q8_REQUIRE(aligned16(a) && ((uintptr_t)y & 3u) == 0 && ((uintptr_t)ids & 3u) == 0 &&
+                   ((uintptr_t)err_word & 3u) == 0,
+               Q8_E_ALIGN, "%s: a must be 16-byte aligned; y/ids/err_word 4-byte", fn);
+    Q8_REQUIRE(n_tok * n_used <= kCtaGroupMaxPairs && W->n_mat <= kCtaGroupMaxMats,
+               Q8_E_UNSUPPORTED, "%s: batch above the small-batch limits", fn);
+    return launch_matmul_routed_ids(W, nullptr, nullptr, a, a_per_slot, n_tok, n_used, ids, y,
+                                    err_word, (cudaStream_t)stream);
+}
+
 q8_status q8_moe_combine(const float *y, const float *route_w, int64_t n_tok, int32_t n_used,
                          int64_t n_out, float *out, void *stream) {
     Q8_REQUIRE(y && route_w && out, Q8_E_NULL, "q8_moe_combine: NULL pointer");
@@ -523,6 +622,7 @@ q8_status q8_moe_ffn(const q8_tensor *up_gate, const q8_tensor *down, const floa
     else
         Q8_REQUIRE(up_gate->n_mat <= 4096, Q8_E_UNSUPPORTED, "q8_moe_ffn: n_mat > 4096");
     const FfnLayout F = ffn_layout(n_tok, n_used, up_gate->n_mat, n_embd, n_ff, routed);
+    const bool small = n_tok * n_used <= kCtaGroupMaxPairs && up_gate->n_mat <= kCtaGroupMaxMats;
     Q8_REQUIRE(ws != nullptr && aligned256(ws), Q8_E_WORKSPACE,
                "q8_moe_ffn: workspace NULL or not 256-byte aligned");
     Q8_REQUIRE(ws_bytes >= F.total, Q8_E_WORKSPACE, "q8_moe_ffn: workspace too small");
@@ -531,6 +631,19 @@ q8_status q8_moe_ffn(const q8_tensor *up_gate, const q8_tensor *down, const floa
     int8_t *xq = (int8_t *)(w8 + F.xq);
     uint16_t *xd = (uint16_t *)(w8 + F.xd);
     float *h = (float *)(w8 + F.h);
+    if (small) {
+        // Three launches: up/gate (x quantized as it is staged; routed: the
+        // grouping built in each CTA from ids), down (h quantized as it is
+        // staged), combine.
+        int32_t *err = routed ? (int32_t *)(w8 + F.group) : nullptr;
+        st = q8_moe_up_gate_swiglu_fp32(up_gate, x, n_tok, ids, n_used, h, err, s);
+        if (st != Q8_OK) return st;
+        if (!routed) return launch_matmul_dense(down, nullptr, nullptr, h, n_tok, out, s);
+        float *y = (float *)(w8 + F.y);
+        st = q8_mul_mat_id_fp32(down, h, 1, n_tok, ids, n_used, y, nullptr, s);
+        if (st != Q8_OK) return st;
+        return launch_combine(y, route_w, n_tok, n_used, n_embd, out, s);
+    }
     st = q8_quantize_row(x, n_tok, n_embd, xq, xd, s);
     if (st != Q8_OK) return st;
     if (!routed) {

@@ -34,39 +34,63 @@ namespace q8 {
 constexpr int kCW = 8;                  // consumer warps
 constexpr int kCT = kCW * 32;           // consumer threads
 constexpr int kThreadsStream = kCT + 32;
-constexpr int kStageQs = 32768;         // quant bytes per stage
-constexpr int kStageD = 2048;           // scale bytes per stage (nr * ld_d * 2 <= 2048 for every k)
-constexpr int kStageBytes = kStageQs + kStageD;
-constexpr int kMaxStages = 6;
+constexpr int kMaxTileQs = 32768;       // quant bytes of one tile at most (nr * k)
+constexpr int kMaxStages = 8;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kBarConsumers = 1;        // named barrier of the consumer warps
 constexpr int kMaxXRows = 16;           // activation rows staged at once (at most)
 
-// Tile geometry, a function of k only: rows per tile, warps per row (the
-// row's blocks are split into wpr segments, one per warp), rows per warp
-// (kCW * rpw / wpr == nr).  A warp takes rpw rows at once, so each
-// activation block it loads from shared memory serves rpw weight rows.
+// Tile geometry: rows per tile, warps per row (the row's blocks are split
+// into wpr segments, one per warp), rows per warp (kCW * rpw / wpr == nr).
+// A warp takes rpw rows at once, so each activation block it loads from
+// shared memory serves rpw weight rows.  A tile holds at most 32 KB of
+// quants.  The order of a row's floating-point sum depends on wpr and k
+// only, and wpr is a function of k, so every kernel sums a row the same way.
 struct Geo {
     int nr, wpr, rpw;
 };
+__host__ __device__ inline int wpr_for_k(int k) {
+    return k <= 1024 ? 1 : k <= 2048 ? 2 : k <= 4096 ? 4 : 8;
+}
+// Plain row tiles.
 __host__ __device__ inline Geo geo_for_k(int k) {
+    if (k <= 768) return {40, 1, 5};
     if (k <= 1024) return {32, 1, 4};
     if (k <= 2048) return {16, 2, 4};
     if (k <= 4096) return {8, 4, 4};
     if (k <= 8192) return {4, 8, 4};
     return {2, 8, 2};
 }
+// Gate/up tiles: nr/2 gate rows and the nr/2 matching up rows; nr/2 divides 32.
+__host__ __device__ inline Geo geo_pair_for_k(int k) {
+    if (k <= 1024) return {32, 1, 4};
+    return geo_for_k(k);
+}
+
+__host__ inline int round128(int v) { return (v + 127) / 128 * 128; }
+
+// Quant and scale bytes of a full tile.
+__host__ inline void tile_bytes(const Geo &g, int k, int64_t ld_d, int *qs, int *d) {
+    *qs = g.nr * k;
+    *d = (int)(g.nr * ld_d * 2);
+}
+
+// Partial-sum buffer stride (floats) of one of its two halves.
+constexpr int kPartRows = 40;
 
 // Shared-memory plan of one launch (offsets in bytes from the dynamic base).
 struct Plan {
     int stages;
+    int stage_qs;     // bytes of quants per stage (the scales follow)
+    int stage_bytes;  // bytes per stage
     int xmax;       // activation rows the stage holds
     int max_nb;     // blocks per activation row the stage is sized for
-    int off_full, off_empty, off_ring, off_xq, off_xd, off_part;
+    int off_full, off_empty, off_ring, off_xq, off_xd, off_part, off_tab;
+    int tab_words;  // routing tables built in shared memory (0: none)
     int bytes;
 };
 
-__host__ inline int plan_part_floats(int nt) { return 2 * 32 * nt; }
+__host__ inline int plan_part_floats(int nt) { return 2 * kPartRows * nt; }
 
 // CTAs per SM of a streaming kernel: two for one or two activation rows per
 // pass (the second CTA hides the first one's barrier and dependency stalls),
@@ -77,9 +101,15 @@ __host__ inline int smem_budget(int nt) {
     return ctas_per_sm(nt) == 2 ? (228 * 1024) / 2 - 1024 : kSmemLimit;
 }
 
-// xrows: activation rows wanted in shared memory at once.
-__host__ inline bool make_plan(int max_k, int xrows, int nt, Plan *out) {
+// tile_qs / tile_d: the largest tile's quant and scale bytes; xrows:
+// activation rows wanted in shared memory at once; tab_words: int32 words of
+// routing tables to build in shared memory.  As many stages as fit.
+__host__ inline bool make_plan(int tile_qs, int tile_d, int max_k, int xrows, int nt, Plan *out,
+                               int tab_words = 0) {
     const int budget = smem_budget(nt);
+    const int tab_bytes = ((tab_words * 4 + 15) / 16) * 16;
+    const int stage_qs = round128(tile_qs);
+    const int stage_bytes = stage_qs + round128(tile_d);
     Plan p{};
     p.max_nb = max_k / QK;
     int xmax = xrows < kMaxXRows ? xrows : kMaxXRows;
@@ -87,20 +117,24 @@ __host__ inline bool make_plan(int max_k, int xrows, int nt, Plan *out) {
     for (;; xmax -= nt) {
         const int x_bytes = xmax * max_k + ((xmax * p.max_nb * 4 + 15) / 16) * 16;
         const int part_bytes = plan_part_floats(nt) * 4;
-        const int fixed = 2 * kMaxStages * 8 + 128 + x_bytes + part_bytes;
-        int stages = (budget - fixed) / kStageBytes;
+        const int fixed = 2 * kMaxStages * 8 + 128 + x_bytes + part_bytes + tab_bytes;
+        int stages = (budget - fixed) / stage_bytes;
         if (stages > kMaxStages) stages = kMaxStages;
         if (stages >= 2 || xmax <= nt) {
             if (stages < 2) return false;
             p.stages = stages;
+            p.stage_qs = stage_qs;
+            p.stage_bytes = stage_bytes;
             p.xmax = xmax;
             p.off_full = 0;
             p.off_empty = kMaxStages * 8;
             p.off_ring = 128;
-            p.off_xq = p.off_ring + stages * kStageBytes;
+            p.off_xq = p.off_ring + stages * stage_bytes;
             p.off_xd = p.off_xq + xmax * max_k;
             p.off_part = p.off_xd + ((xmax * p.max_nb * 4 + 15) / 16) * 16;
-            p.bytes = p.off_part + part_bytes;
+            p.off_tab = p.off_part + part_bytes;
+            p.tab_words = tab_words;
+            p.bytes = p.off_tab + tab_bytes;
             *out = p;
             return true;
         }
@@ -132,11 +166,13 @@ struct Ring {
     uint64_t *empty;
     unsigned char *base;
     int stages;
+    int stage_bytes;
+    int stage_qs;
     __device__ __forceinline__ int8_t *qs(int s) const {
-        return reinterpret_cast<int8_t *>(base + (size_t)s * kStageBytes);
+        return reinterpret_cast<int8_t *>(base + (size_t)s * stage_bytes);
     }
     __device__ __forceinline__ uint16_t *d(int s) const {
-        return reinterpret_cast<uint16_t *>(base + (size_t)s * kStageBytes + kStageQs);
+        return reinterpret_cast<uint16_t *>(base + (size_t)s * stage_bytes + stage_qs);
     }
 };
 
@@ -146,6 +182,8 @@ __device__ __forceinline__ Ring ring_init(unsigned char *smem, const Plan &pl) {
     R.empty = reinterpret_cast<uint64_t *>(smem + pl.off_empty);
     R.base = smem + pl.off_ring;
     R.stages = pl.stages;
+    R.stage_bytes = pl.stage_bytes;
+    R.stage_qs = pl.stage_qs;
     if (threadIdx.x == 0) {
         for (int s = 0; s < pl.stages; ++s) {
             mbar_init(&R.full[s], 1);
@@ -185,6 +223,84 @@ __device__ __forceinline__ void produce(const Ring &R, int64_t tb, int64_t te, S
 }
 
 // ---------------------------------------------------------------------------
+// Expert grouping inside one CTA (all threads), for small batches: the tables
+// of GroupLayout L (counts, offsets, the ascending list of experts with
+// pairs, the pairs sorted by expert then by pair index) are built in shared
+// memory `tab` from ids [n_tok][n_used].  The same stable counting sort as
+// the grouping kernel; every CTA builds its own copy.  Routing-id errors are
+// recorded in tab[WS_ERR] and, by CTA 0, in *err_out (if given).  The
+// tensor-core list is not used here; its words serve as the scatter cursors.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cta_group(const int32_t *__restrict__ ids, int n_tok, int n_used,
+                                          int n_mat, const GroupLayout &L, int32_t *tab,
+                                          int32_t *err_out) {
+    const int P = n_tok * n_used;
+    int *cnt = tab + L.count;
+    int *cursor = tab + L.list_big;
+    for (int e = threadIdx.x; e < n_mat; e += blockDim.x) cnt[e] = 0;
+    if (threadIdx.x == 0) tab[WS_ERR] = 0;
+    __syncthreads();
+    int err = 0;
+    for (int p = threadIdx.x; p < P; p += blockDim.x) {
+        const int e = ids[p];
+        if (e < 0 || e >= n_mat) {
+            err |= ERR_ID_RANGE;
+            continue;
+        }
+        atomicAdd(&cnt[e], 1);
+        const int t = p / n_used;
+        for (int s2 = t * n_used; s2 < p; ++s2)
+            if (ids[s2] == e) err |= ERR_ID_REPEAT;
+    }
+    if (err) atomicOr(&tab[WS_ERR], err);
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x < 32) {
+        int running = 0, n_small = 0;
+        for (int base = 0; base < n_mat; base += 32) {
+            const int e = base + lane;
+            const int c = e < n_mat ? cnt[e] : 0;
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            const int off = running + incl - c;
+            if (e < n_mat) {
+                tab[L.offset + e] = off;
+                cursor[e] = off;
+            }
+            const unsigned bs = __ballot_sync(0xffffffffu, c > 0);
+            if (c > 0) tab[L.list_small + n_small + __popc(bs & ((1u << lane) - 1u))] = e;
+            n_small += __popc(bs);
+            running += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            tab[L.offset + n_mat] = running;
+            tab[WS_N_SMALL] = n_small;
+            tab[WS_N_BIG] = 0;
+            tab[WS_N_PAIRS] = P;
+        }
+        __syncwarp();
+        for (int base = 0; base < P; base += 32) {
+            const int p = base + lane;
+            const int e = p < P ? ids[p] : -1;
+            const bool valid = e >= 0 && e < n_mat;
+            const int key = valid ? e : n_mat + lane;
+            const unsigned m = __match_any_sync(0xffffffffu, key);
+            const int rank = __popc(m & ((1u << lane) - 1u));
+            if (valid) tab[L.pairs + cursor[e] + rank] = p;
+            __syncwarp();
+            if (valid && (__ffs(m) - 1) == lane) cursor[e] += __popc(m);
+            __syncwarp();
+        }
+        if (err_out && blockIdx.x == 0 && lane == 0) *err_out = tab[WS_ERR];
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
 // activation staging (consumer threads only: threadIdx.x < kCT)
 // ---------------------------------------------------------------------------
 struct XStage {
@@ -199,6 +315,7 @@ __device__ __forceinline__ void stage_q8(const XStage &xs, const int8_t *__restr
                                          RowFn arow) {
     const int nb = k / QK;
     const int v_per_row = k / 16;
+#pragma unroll 4
     for (int i = threadIdx.x; i < n * v_per_row; i += kCT) {
         const int j = i / v_per_row;
         const int c = i - j * v_per_row;
@@ -213,21 +330,40 @@ __device__ __forceinline__ void stage_q8(const XStage &xs, const int8_t *__restr
 }
 
 // Quantize fp32 rows arow(j) of af (k floats apart), j < n, into the stage,
-// one warp per 32-block, by the Q8_0 rule.
+// one warp per 32-block, by the Q8_0 rule.  Each warp first issues the loads
+// of up to 8 of its blocks, then quantizes them (one memory latency per 8
+// blocks instead of one per block).
 template <class RowFn>
 __device__ __forceinline__ void stage_f32(const XStage &xs, const float *__restrict__ af, int k,
                                           int n, RowFn arow) {
     const int nb = k / QK;
     const int lane = threadIdx.x & 31;
-    for (int blk = threadIdx.x >> 5; blk < n * nb; blk += kCW) {
-        const int j = blk / nb;
-        const int b = blk - j * nb;
-        const float v = af[(int64_t)arow(j) * k + b * QK + lane];
-        const float amax = warp_max_all(fabsf(v));
-        const float d32 = block_scale(amax);
-        const float id = block_inv_scale(d32);
-        xs.q[(size_t)j * k + b * QK + lane] = (int8_t)quantize_one(v, id);
-        if (lane == 0) xs.dx[(size_t)j * nb + b] = scale_value(scale_bits(d32));
+    const int total = n * nb;
+    for (int b0 = threadIdx.x >> 5; b0 < total; b0 += kCW * 8) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int blk = b0 + i * kCW;
+            v[i] = 0.0f;
+            if (blk < total) {
+                const int j = blk / nb;
+                const int b = blk - j * nb;
+                v[i] = af[(int64_t)arow(j) * k + b * QK + lane];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int blk = b0 + i * kCW;  // warp-uniform
+            if (blk < total) {
+                const int j = blk / nb;
+                const int b = blk - j * nb;
+                const float amax = warp_max_all(fabsf(v[i]));
+                const float d32 = block_scale(amax);
+                const float id = block_inv_scale(d32);
+                xs.q[(size_t)j * k + b * QK + lane] = (int8_t)quantize_one(v[i], id);
+                if (lane == 0) xs.dx[(size_t)j * nb + b] = scale_value(scale_bits(d32));
+            }
+        }
     }
 }
 
@@ -242,8 +378,8 @@ __device__ __forceinline__ float small_int_to_float(int v) {
     return __int_as_float(v + 0x4B400000) - 12582912.0f;
 }
 
-// acc[r][t] = sum over this warp's blocks of row (row0 + r) of the stage with
-// activation row (xrow0 + t), t < n; every lane ends with the full sums.
+// acc[r][t] = this lane's part of the sum over the warp's blocks of row
+// (row0 + r) of the stage with activation row (xrow0 + t), t < n.
 // Lane l takes block base + l (both 16-byte halves), so each block dot is
 // 8 dp4a in one lane; |isum| <= 32 * 128 * 128 < 2^22.
 template <int NT, int RPW>
@@ -290,10 +426,52 @@ __device__ __forceinline__ void dot_rows(const int8_t *sq, const uint16_t *sd, i
             }
         }
     }
+}
+
+// Sum each of V values (V a power of two, <= 32) over the 32 lanes of a warp
+// with a butterfly that halves the values a lane carries at each of the first
+// log2(V) levels (V - 1 + 5 - log2(V) shuffles instead of 5 V).  Every value
+// is summed over the same xor tree (offsets 16, 8, 4, 2, 1) as warp_sum_all,
+// so the results are bitwise those of warp_sum_all.  Lane l returns the sum
+// of value reduce_scatter_index<V>(l); the lanes with l % (32 / V) == 0 hold
+// the V distinct values.
+__host__ __device__ constexpr int pow2_ceil(int v) {
+    return v <= 1 ? 1 : v <= 2 ? 2 : v <= 4 ? 4 : v <= 8 ? 8 : v <= 16 ? 16 : 32;
+}
+
+template <int V>
+__device__ __forceinline__ float warp_reduce_scatter(float (&a)[V]) {
+    const int lane = threadIdx.x & 31;
+    int m = V;
 #pragma unroll
-    for (int r = 0; r < RPW; ++r)
+    for (int o = 16; o >= 1; o >>= 1) {
+        if (m > 1) {
+            const bool upper = (lane & o) != 0;
 #pragma unroll
-        for (int t = 0; t < NT; ++t) acc[r][t] = warp_sum_all(acc[r][t]);
+            for (int i = 0; i < V / 2; ++i) {
+                if (i < m / 2) {
+                    const float send = upper ? a[i] : a[i + m / 2];
+                    const float keep = upper ? a[i + m / 2] : a[i];
+                    a[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                }
+            }
+            m >>= 1;
+        } else {
+            a[0] += __shfl_xor_sync(0xffffffffu, a[0], o);
+        }
+    }
+    return a[0];
+}
+
+template <int V>
+__device__ __forceinline__ int reduce_scatter_index(int lane) {
+    int idx = 0, m = V;
+#pragma unroll
+    for (int o = 16; o >= 1 && m > 1; o >>= 1) {
+        if (lane & o) idx += m / 2;
+        m >>= 1;
+    }
+    return idx;
 }
 
 // Computes this warp's rows of a stage for activation rows [xrow0, xrow0+n)
@@ -310,11 +488,30 @@ __device__ __forceinline__ void warp_rows_to_part(const int8_t *sq, const uint16
     {                                                                                         \
         float acc[RPW_][NT];                                                                  \
         dot_rows<NT, RPW_>(sq, sd, k, ld_d, row0, seg, g.wpr, xs, xrow0, n, acc);             \
-        _Pragma("unroll") for (int r = 0; r < RPW_; ++r)                                      \
-            _Pragma("unroll") for (int t = 0; t < NT; ++t) if (lane == ((r * NT + t) & 31))   \
-                part[((row0 + r) * g.wpr + seg) * NT + t] = acc[r][t];                        \
+        constexpr int V = RPW_ * NT;                                                          \
+        if constexpr (V <= 32) {                                                              \
+            constexpr int VP = pow2_ceil(V);                                                  \
+            float a[VP];                                                                      \
+            _Pragma("unroll") for (int i = 0; i < VP; ++i)                                    \
+                a[i] = i < V ? reinterpret_cast<float(&)[V]>(acc)[i] : 0.0f;                  \
+            const float v = warp_reduce_scatter<VP>(a);                                       \
+            if ((lane & (32 / VP - 1)) == 0) {                                                \
+                const int idx = reduce_scatter_index<VP>(lane);                               \
+                if (idx < V) {                                                                \
+                    const int r = idx / NT, t = idx - (idx / NT) * NT;                        \
+                    part[((row0 + r) * g.wpr + seg) * NT + t] = v;                            \
+                }                                                                             \
+            }                                                                                 \
+        } else {                                                                              \
+            _Pragma("unroll") for (int r = 0; r < RPW_; ++r)                                  \
+                _Pragma("unroll") for (int t = 0; t < NT; ++t) {                              \
+                    const float v = warp_sum_all(acc[r][t]);                                  \
+                    if (lane == 0) part[((row0 + r) * g.wpr + seg) * NT + t] = v;             \
+                }                                                                             \
+        }                                                                                     \
     }
-    if (g.rpw == 4) Q8_ROWS_CASE(4)
+    if (g.rpw == 5) Q8_ROWS_CASE(5)
+    else if (g.rpw == 4) Q8_ROWS_CASE(4)
     else if (g.rpw == 2) Q8_ROWS_CASE(2)
     else Q8_ROWS_CASE(1)
 #undef Q8_ROWS_CASE

@@ -47,7 +47,7 @@ EXPORTS = ["q8_scale_stride", "q8_pack", "q8_quantize_row", "q8_gemv", "q8_gemv_
            "q8_moe_ffn_workspace_size", "q8_moe_ffn", "q8_check", "q8_debug_block_dots",
            "q8_status_string", "q8_last_error", "q8_moe_group",
            "q8_moe_up_gate_swiglu_pregrouped", "q8_mul_mat_id_pregrouped",
-           "q8_moe_up_gate_swiglu_noalloc"]
+           "q8_moe_up_gate_swiglu_noalloc", "q8_moe_up_gate_swiglu_fp32", "q8_mul_mat_id_fp32"]
 
 
 def lib_path() -> str:
@@ -91,6 +91,8 @@ def load(auto_build: bool = True):
                                               vp]),
             "q8_moe_up_gate_swiglu_noalloc": (st, [P(_Tensor), vp, vp, i64, vp, i32, vp, vp, vp,
                                                    vp, vp, vp]),
+            "q8_moe_up_gate_swiglu_fp32": (st, [P(_Tensor), vp, i64, vp, i32, vp, vp, vp]),
+            "q8_mul_mat_id_fp32": (st, [P(_Tensor), vp, i32, i64, vp, i32, vp, vp, vp]),
             "q8_status_string": (ctypes.c_char_p, [st]),
             "q8_last_error": (ctypes.c_char_p, []),
         }
@@ -255,6 +257,27 @@ def moe_up_gate_swiglu_noalloc(W: Q8Tensor, xq, xd, ids, h, hq=None, hd=None, g=
           xq.shape[0], _ptr(ids), ids.shape[1], _ptr(h), _ptr(hq), _ptr(hd), _ptr(g), _ptr(u),
           _stream(stream))
     return h
+
+
+def moe_up_gate_swiglu_fp32(W: Q8Tensor, x, ids=None, h=None, err_word=None, stream=None):
+    """Up/gate + SwiGLU from fp32 x (quantized in the kernel), small batches, no workspace."""
+    n_tok = x.shape[0]
+    n_used = 1 if ids is None else ids.shape[1]
+    if h is None:
+        h = torch.empty((n_tok, n_used, W.rows // 2), dtype=torch.float32, device=x.device)
+    _call("q8_moe_up_gate_swiglu_fp32", ctypes.byref(W.c()), _ptr(x), n_tok, _ptr(ids), n_used,
+          _ptr(h), _ptr(err_word), _stream(stream))
+    return h
+
+
+def mul_mat_id_fp32(W: Q8Tensor, a, ids, a_per_slot: bool, y=None, err_word=None, stream=None):
+    """mul_mat_id from fp32 activations (quantized in the kernel), small batches."""
+    n_tok, n_used = ids.shape
+    if y is None:
+        y = torch.empty((n_tok, n_used, W.rows), dtype=torch.float32, device=a.device)
+    _call("q8_mul_mat_id_fp32", ctypes.byref(W.c()), _ptr(a), 1 if a_per_slot else 0, n_tok,
+          _ptr(ids), n_used, _ptr(y), _ptr(err_word), _stream(stream))
+    return y
 
 
 def mul_mat_id(W: Q8Tensor, aq, ad, ids, a_per_slot: bool, ws=None, y=None, stream=None):

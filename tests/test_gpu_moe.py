@@ -244,3 +244,41 @@ def test_bad_ids_reported_without_fault():
     # the context is still usable, and a good call clears the report
     q8.moe_up_gate_swiglu(UG, xq, xd, ids, ws=ws)
     q8.check(ws)
+
+
+@pytest.mark.parametrize("n_exp,n_ff,n_embd,n_tok,n_used", [
+    (128, 704, 2816, 1, 8), (128, 704, 2816, 16, 8), (16, 64, 128, 5, 4), (1, 64, 256, 3, 1),
+    (32, 96, 2048, 33, 2)])
+def test_fp32_entry_points_match_workspace_path(n_exp, n_ff, n_embd, n_tok, n_used):
+    """The small-batch fp32 calls (quantize in the kernel, group in every CTA)
+    give bitwise the results of quantize + grouping + the Q8_0 calls."""
+    t, UG, DN, ids, p = _layer(n_exp, n_ff, n_embd, n_tok, n_used, seed=300 + n_tok + n_exp)
+    x = t["x"].to(DEV)
+    xq, xd = q8.quantize_row(x)
+    ref = q8.moe_up_gate_swiglu(UG, xq, xd, ids, want_hq=True)
+    h = q8.moe_up_gate_swiglu_fp32(UG, x, ids)
+    assert torch.equal(h, ref["h"])
+    if ids is not None:
+        y = q8.mul_mat_id_fp32(DN, h.reshape(-1, n_ff), ids, True)
+        y2 = q8.mul_mat_id(DN, ref["hq"].reshape(-1, n_ff), ref["hd"].reshape(-1, n_ff // 32),
+                           ids, True)
+        assert torch.equal(y, y2)
+        # the whole step through q8_moe_ffn takes the same kernels
+        out = q8.moe_ffn(UG, DN, x, ids, p)
+        assert torch.equal(out, q8.moe_combine(y2, p))
+
+
+def test_fp32_entry_reports_bad_ids():
+    t, UG, DN, ids, p = _layer(8, 32, 64, 4, 2, seed=97)
+    x = t["x"].to(DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    q8.moe_up_gate_swiglu_fp32(UG, x, ids, err_word=err)
+    assert int(err.item()) == 0
+    bad = ids.clone()
+    bad[3, 1] = -1
+    q8.moe_up_gate_swiglu_fp32(UG, x, bad, err_word=err)
+    assert int(err.item()) != 0
+    rep = ids.clone()
+    rep[0, 1] = rep[0, 0]
+    q8.mul_mat_id_fp32(DN, torch.zeros((8, 32), device=DEV), rep, True, err_word=err)
+    assert int(err.item()) != 0
