@@ -389,8 +389,12 @@ class MoeWorkload:
         self.small = P <= 1024 and E <= 512
         if self.small:
             self.launches_per_step = layers * (3 if self.routed else 2)
+        elif self.routed:
+            # quantize x, group, up/gate (dp4a + tensor cores), quantize h,
+            # down (dp4a + tensor cores), combine
+            self.launches_per_step = layers * 8
         else:
-            self.launches_per_step = layers * (5 if self.routed else 3)
+            self.launches_per_step = layers * 4
         self.dominant_launches = layers
         self.h2d_bytes = self.x_host[0].numel() * 4 + (
             (self.ids_host[0].numel() * 4 + self.p_host[0].numel() * 4) if self.routed else 0)

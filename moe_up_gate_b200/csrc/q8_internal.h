@@ -128,6 +128,16 @@ constexpr int64_t kCtaGroupMaxMats = Q8_SMALL_BATCH_MATS;
 // Wait-timeout flags latched by the streaming kernels of each file.
 q8_status read_wait_errors_matmul(int *flags);
 q8_status read_wait_errors_moe(int *flags);
+q8_status read_wait_errors_tc(int *flags);
+
+// Tensor-core path (q8_tc.cu) for experts with at least kTcMinPairs routed
+// rows: whether a weight view can take it, and the launch over the
+// tensor-core list of a grouping workspace.
+constexpr int kTcMinPairs = 16;
+bool tc_eligible(const q8_tensor *W, bool upgate);
+q8_status launch_tc(const q8_tensor *W, bool upgate, const int8_t *aq, const uint16_t *ad,
+                    const float *af, int a_per_slot, int64_t n_tok, int32_t n_used, float *out,
+                    const int32_t *ws, cudaStream_t s);
 
 // Launch the expert-grouping kernel (q8_moe.cu).  big_threshold: experts with
 // at least this many pairs go to the tensor-core list.

@@ -45,7 +45,7 @@ struct MatmulParams {
     float *y;
     const int32_t *ws;
     int64_t lay_count, lay_offset, lay_list, lay_pairs, lay_big;
-    int list_word;
+    int include_big;  // the dp4a kernel also takes the tensor-core list
     int n_dense;
     int a_per_slot;
     int n_used;
@@ -81,7 +81,11 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
         griddep_wait();
     }
     const bool routed = tab != nullptr;
-    const int n_mat = routed ? tab[p.list_word] : 1;
+    const int n_small = routed ? tab[WS_N_SMALL] : 1;
+    const int n_mat = n_small + ((routed && p.include_big) ? tab[WS_N_BIG] : 0);
+    auto expert = [&](int mi) {
+        return mi < n_small ? tab[p.lay_list + mi] : tab[p.lay_big + (mi - n_small)];
+    };
     int64_t tb, te;
     my_tiles((int64_t)n_mat * tpm, &tb, &te);
     if ((threadIdx.x >> 5) == kCW) {  // producer warp
@@ -89,7 +93,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             auto src = [&](int64_t t) {
                 TileSrc ts{};
                 const int mi = (int)(t / tpm), ti = (int)(t % tpm);
-                const int e = routed ? tab[p.lay_list + mi] : 0;
+                const int e = routed ? expert(mi) : 0;
                 const int r0 = ti * g.nr;
                 const int64_t row = (int64_t)e * p.mat_stride + r0;
                 ts.q0 = p.wq + row * p.k;
@@ -113,7 +117,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_matmul);
         const int mi = (int)(t / tpm), ti = (int)(t % tpm);
-        const int e = routed ? tab[p.lay_list + mi] : 0;
+        const int e = routed ? expert(mi) : 0;
         const int cnt = routed ? tab[p.lay_count + e] : p.n_dense;
         const int32_t *plist = routed ? tab + p.lay_pairs + tab[p.lay_offset + e] : nullptr;
         const int r0 = ti * g.nr;
@@ -218,13 +222,20 @@ q8_status launch_matmul_routed(const q8_tensor *W, const int8_t *aq, const uint1
     p.lay_count = L.count;
     p.lay_offset = L.offset;
     p.lay_list = L.list_small;
+    p.lay_big = L.list_big;
     p.lay_pairs = L.pairs;
-    p.list_word = WS_N_SMALL;
+    p.include_big = 0;
     p.a_per_slot = a_per_slot ? 1 : 0;
     p.n_used = n_used;
+    // experts with at least kTcMinPairs rows go to the tensor cores when the
+    // shape allows it; otherwise the dp4a kernel takes them too
+    const bool tc = tc_eligible(W, false) && P >= kTcMinPairs;
+    p.include_big = tc ? 0 : 1;
     const Geo g = geo_for_k(p.k);
     const int64_t tiles = std::min<int64_t>(W->n_mat, P) * ((p.rows + g.nr - 1) / g.nr);
-    return launch_matmul(p, n_tok, tiles, s);
+    q8_status st = launch_matmul(p, n_tok, tiles, s);
+    if (st != Q8_OK || !tc) return st;
+    return launch_tc(W, false, aq, ad, af, a_per_slot, n_tok, n_used, y, ws, s);
 }
 
 // mul_mat_id with the grouping built in each CTA from ids (small batches);
@@ -252,7 +263,7 @@ q8_status launch_matmul_routed_ids(const q8_tensor *W, const int8_t *aq, const u
     p.lay_list = L.list_small;
     p.lay_big = L.list_big;
     p.lay_pairs = L.pairs;
-    p.list_word = WS_N_SMALL;
+    p.include_big = 0;
     p.a_per_slot = a_per_slot ? 1 : 0;
     p.n_used = n_used;
     p.ids = ids;
@@ -464,7 +475,7 @@ static q8_status mul_mat_id_entry(const char *fn, const q8_tensor *W, const int8
     Q8_REQUIRE(ws_bytes >= q8_moe_workspace_size(n_tok, n_used, W->n_mat), Q8_E_WORKSPACE,
                "%s: workspace too small", fn);
     if (group) {
-        st = launch_group(ids, n_tok, n_used, W->n_mat, 1 << 30, (int32_t *)ws, s);
+        st = launch_group(ids, n_tok, n_used, W->n_mat, kTcMinPairs, (int32_t *)ws, s);
         if (st != Q8_OK) return st;
     }
     return launch_matmul_routed(W, aq, ad, nullptr, a_per_slot, n_tok, n_used, y,

@@ -146,7 +146,7 @@ struct UpGateParams {
     float *u_out;
     const int32_t *ws;
     int64_t lay_count, lay_offset, lay_list, lay_pairs, lay_big;
-    int list_word;
+    int include_big;  // the dp4a kernel also takes the tensor-core list
     int n_dense;
     int n_used;
     // routed with the grouping built in each CTA from ids (ws unused)
@@ -184,7 +184,11 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
         griddep_wait();
     }
     const bool routed = tab != nullptr;
-    const int n_mat = routed ? tab[p.list_word] : 1;
+    const int n_small = routed ? tab[WS_N_SMALL] : 1;
+    const int n_mat = n_small + ((routed && p.include_big) ? tab[WS_N_BIG] : 0);
+    auto expert = [&](int mi) {
+        return mi < n_small ? tab[p.lay_list + mi] : tab[p.lay_big + (mi - n_small)];
+    };
     int64_t tb, te;
     my_tiles((int64_t)n_mat * tpm, &tb, &te);
     if ((threadIdx.x >> 5) == kCW) {  // producer warp
@@ -192,7 +196,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             auto src = [&](int64_t t) {
                 TileSrc ts{};
                 const int mi = (int)(t / tpm), ti = (int)(t % tpm);
-                const int e = routed ? tab[p.lay_list + mi] : 0;
+                const int e = routed ? expert(mi) : 0;
                 const int64_t gate_row = (int64_t)e * p.mat_stride + (int64_t)ti * half_rows;
                 const int64_t up_row = gate_row + p.n_ff;
                 ts.q0 = p.wq + gate_row * p.k;
@@ -220,7 +224,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_moe);
         const int mi = (int)(t / tpm), ti = (int)(t % tpm);
-        const int e = routed ? tab[p.lay_list + mi] : 0;
+        const int e = routed ? expert(mi) : 0;
         const int cnt = routed ? tab[p.lay_count + e] : p.n_dense;
         const int32_t *plist = routed ? tab + p.lay_pairs + tab[p.lay_offset + e] : nullptr;
         const int r0 = ti * half_rows;
@@ -404,7 +408,7 @@ static q8_status up_gate_entry(const char *fn, const q8_tensor *up_gate, const i
                "%s: workspace too small", fn);
     const int64_t P = n_tok * n_used;
     if (group) {
-        st = launch_group(ids, n_tok, n_used, up_gate->n_mat, 1 << 30, (int32_t *)ws, s);
+        st = launch_group(ids, n_tok, n_used, up_gate->n_mat, kTcMinPairs, (int32_t *)ws, s);
         if (st != Q8_OK) return st;
     }
     const GroupLayout L = group_layout(P, up_gate->n_mat);
@@ -412,10 +416,20 @@ static q8_status up_gate_entry(const char *fn, const q8_tensor *up_gate, const i
     p.lay_count = L.count;
     p.lay_offset = L.offset;
     p.lay_list = L.list_small;
+    p.lay_big = L.list_big;
     p.lay_pairs = L.pairs;
-    p.list_word = WS_N_SMALL;
+    // experts with at least kTcMinPairs rows go to the tensor cores when the
+    // shape allows it; otherwise the dp4a kernel takes them too
+    // (the g/u debug taps come from the dp4a kernel only)
+    const bool tc = tc_eligible(up_gate, true) && P >= kTcMinPairs && !g_out && !u_out;
+    p.include_big = tc ? 0 : 1;
     st = launch_up_gate(p, n_tok, std::min<int64_t>(up_gate->n_mat, P), s);
-    if (st != Q8_OK || hq == nullptr) return st;
+    if (st != Q8_OK) return st;
+    if (tc) {
+        st = launch_tc(up_gate, true, xq, xd, nullptr, 0, n_tok, n_used, h, (const int32_t *)ws, s);
+        if (st != Q8_OK) return st;
+    }
+    if (hq == nullptr) return Q8_OK;
     return launch_quantize(h, P, n_ff, hq, hd, n_ff / QK, s);
 }
 
@@ -484,7 +498,7 @@ q8_status q8_moe_group(const int32_t *ids, int64_t n_tok, int32_t n_used, int64_
                "q8_moe_group: workspace NULL or not 256-byte aligned");
     Q8_REQUIRE(ws_bytes >= q8_moe_workspace_size(n_tok, n_used, n_mat), Q8_E_WORKSPACE,
                "q8_moe_group: workspace too small");
-    return launch_group(ids, n_tok, n_used, n_mat, 1 << 30, (int32_t *)ws, (cudaStream_t)stream);
+    return launch_group(ids, n_tok, n_used, n_mat, kTcMinPairs, (int32_t *)ws, (cudaStream_t)stream);
 }
 
 q8_status q8_moe_up_gate_swiglu_noalloc(const q8_tensor *up_gate, const int8_t *xq,
@@ -553,7 +567,7 @@ q8_status q8_moe_up_gate_swiglu_fp32(const q8_tensor *up_gate, const float *x, i
     p.lay_list = L.list_small;
     p.lay_big = L.list_big;
     p.lay_pairs = L.pairs;
-    p.list_word = WS_N_SMALL;
+    p.include_big = 0;
     p.ids = ids;
     p.n_tok = (int)n_tok;
     p.n_mat = (int)up_gate->n_mat;
@@ -675,10 +689,11 @@ q8_status q8_check(const void *ws, void *stream) {
     if (ws) e = cudaMemcpyAsync(&flags, ws, sizeof flags, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) Q8_FAIL(Q8_E_CUDA, "q8_check: %s", cudaGetErrorString(e));
-    int w1 = 0, w2 = 0;
-    if (read_wait_errors_matmul(&w1) != Q8_OK || read_wait_errors_moe(&w2) != Q8_OK)
+    int w1 = 0, w2 = 0, w3 = 0;
+    if (read_wait_errors_matmul(&w1) != Q8_OK || read_wait_errors_moe(&w2) != Q8_OK ||
+        read_wait_errors_tc(&w3) != Q8_OK)
         Q8_FAIL(Q8_E_CUDA, "q8_check: reading the kernels' wait flags failed");
-    if (w1 | w2)
+    if (w1 | w2 | w3)
         Q8_FAIL(Q8_E_CUDA, "q8_check: a kernel gave up waiting for a shared-memory stage");
     if (flags & ERR_ID_RANGE) Q8_FAIL(Q8_E_BAD_ID, "q8_check: a routing id is out of range");
     if (flags & ERR_ID_REPEAT)
