@@ -121,6 +121,23 @@ q8_status launch_matmul_routed_ids(const q8_tensor *W, const int8_t *aq, const u
                                    int32_t n_used, const int32_t *ids, float *y,
                                    int32_t *err_out, cudaStream_t s);
 
+// Rows per compute pass (the kernels' NT; a pass over fewer rows runs a
+// narrower variant at run time) and rows staged in shared memory at once
+// (every row of an expert where possible: restaging per tile costs a memory
+// latency each time).  An expert has at most n_tok rows.
+struct RowPlan {
+    int64_t nt_rows, x_rows;
+};
+inline RowPlan routed_rows(int64_t n_tok, int64_t n_used, int64_t n_mat) {
+    (void)n_used;
+    (void)n_mat;
+    RowPlan r;
+    r.nt_rows = n_tok;
+    r.x_rows = n_tok < 16 ? n_tok : 16;
+    return r;
+}
+inline RowPlan dense_rows(int64_t n_tok) { return RowPlan{n_tok, n_tok < 16 ? n_tok : 16}; }
+
 // Batches small enough for the grouping to be built inside each CTA.
 constexpr int64_t kCtaGroupMaxPairs = Q8_SMALL_BATCH_PAIRS;
 constexpr int64_t kCtaGroupMaxMats = Q8_SMALL_BATCH_MATS;

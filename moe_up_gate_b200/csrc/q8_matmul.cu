@@ -146,18 +146,21 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             for (int tg = 0; tg < nx; tg += NT) {
                 const int n = min(NT, nx - tg);
                 float *part = part0 + buf * kPartRows * NT;
-                warp_rows_to_part<NT>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, xs, tg, n, part);
-                if (grp == n_grp - 1 && tg + NT >= nx) {  // last read of this stage
-                    __syncwarp();
-                    if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
-                }
-                named_bar_sync(kBarConsumers, kCT);
-                for (int i = threadIdx.x; i < rows_valid * n; i += kCT) {
-                    const int row = i / n;
-                    const int tt = i - row * n;
-                    const int pr = plist ? plist[x0 + tg + tt] : x0 + tg + tt;
-                    p.y[(int64_t)pr * p.rows + r0 + row] = part_sum<NT>(part, g, row, tt);
-                }
+                with_nt<NT>(n, [&](auto ntc) {
+                    constexpr int NTC = decltype(ntc)::value;
+                    warp_rows_to_part<NTC>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, xs, tg, n, part);
+                    if (grp == n_grp - 1 && tg + NT >= nx) {  // last read of this stage
+                        __syncwarp();
+                        if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
+                    }
+                    named_bar_sync(kBarConsumers, kCT);
+                    for (int j = 0, i = epi_index(0); i < rows_valid * n; i = epi_index(++j)) {
+                        const int row = i / n;
+                        const int tt = i - row * n;
+                        const int pr = plist ? plist[x0 + tg + tt] : x0 + tg + tt;
+                        p.y[(int64_t)pr * p.rows + r0 + row] = part_sum<NTC>(part, g, row, tt);
+                    }
+                });
                 buf ^= 1;
             }
         }
@@ -178,20 +181,20 @@ int num_sms() {
     return g_num_sms[dev];
 }
 
-// max_group: the most activation rows any one matrix has (bounds NT);
+// rp: rows per compute pass (the kernel's NT) and rows staged at once;
 // max_tiles: an upper bound of the tile count (sizes the grid).
-q8_status launch_matmul(const MatmulParams &base, int64_t max_group, int64_t max_tiles,
+q8_status launch_matmul(const MatmulParams &base, RowPlan rp, int64_t max_tiles,
                         cudaStream_t s) {
     MatmulParams p = base;
-    const int nt = pick_nt(max_group);
+    const int nt = pick_nt(rp.nt_rows);
     const int tab_words =
         p.ids ? (int)group_layout((int64_t)p.n_tok * p.n_used, p.n_mat).words : 0;
     int tq, td;
     tile_bytes(geo_for_k(p.k), p.k, p.ld_d, &tq, &td);
-    if (!make_plan(tq, td, p.k, (int)std::min<int64_t>(max_group, kMaxXRows), nt, &p.plan,
+    if (!make_plan(tq, td, p.k, (int)std::min<int64_t>(rp.x_rows, kMaxXRows), nt, &p.plan,
                    tab_words))
         Q8_FAIL(Q8_E_UNSUPPORTED, "matmul: k=%d does not fit the shared-memory plan", p.k);
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * ctas_per_sm(nt), max_tiles));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * p.plan.ctas, max_tiles));
     switch (nt) {
         case 1: return launch_stream(stream_matmul_kernel<1>, grid, p.plan.bytes, s, p, "matmul");
         case 2: return launch_stream(stream_matmul_kernel<2>, grid, p.plan.bytes, s, p, "matmul");
@@ -233,7 +236,7 @@ q8_status launch_matmul_routed(const q8_tensor *W, const int8_t *aq, const uint1
     p.include_big = tc ? 0 : 1;
     const Geo g = geo_for_k(p.k);
     const int64_t tiles = std::min<int64_t>(W->n_mat, P) * ((p.rows + g.nr - 1) / g.nr);
-    q8_status st = launch_matmul(p, n_tok, tiles, s);
+    q8_status st = launch_matmul(p, routed_rows(n_tok, n_used, W->n_mat), tiles, s);
     if (st != Q8_OK || !tc) return st;
     return launch_tc(W, false, aq, ad, af, a_per_slot, n_tok, n_used, y, ws, s);
 }
@@ -272,7 +275,7 @@ q8_status launch_matmul_routed_ids(const q8_tensor *W, const int8_t *aq, const u
     p.err_out = err_out;
     const Geo g = geo_for_k(p.k);
     const int64_t tiles = std::min<int64_t>(W->n_mat, P) * ((p.rows + g.nr - 1) / g.nr);
-    return launch_matmul(p, n_tok, tiles, s);
+    return launch_matmul(p, routed_rows(n_tok, n_used, W->n_mat), tiles, s);
 }
 
 // Dense matmul of fp32 (af) or Q8_0 (aq/ad) activation rows: y = W a.
@@ -295,7 +298,7 @@ q8_status launch_matmul_dense(const q8_tensor *W, const int8_t *aq, const uint16
         p.y = y + t0 * W->rows;
         p.ws = nullptr;
         p.n_dense = (int)nt;
-        q8_status st = launch_matmul(p, nt, tiles, s);
+        q8_status st = launch_matmul(p, dense_rows(nt), tiles, s);
         if (st != Q8_OK) return st;
     }
     return Q8_OK;
@@ -388,17 +391,21 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             for (int tg = 0; tg < nx; tg += NT) {
                 const int n = min(NT, nx - tg);
                 float *part = part0 + buf * kPartRows * NT;
-                warp_rows_to_part<NT>(R.qs(s), R.d(s), q.k, q.ld_d, g, xs, tg, n, part);
-                if (grp == n_grp - 1 && tg + NT >= nx) {
-                    __syncwarp();
-                    if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
-                }
-                named_bar_sync(kBarConsumers, kCT);
-                for (int i = threadIdx.x; i < rows_valid * n; i += kCT) {
-                    const int row = i / n;
-                    const int tt = i - row * n;
-                    q.y[(int64_t)(x0 + tg + tt) * q.rows + r0 + row] = part_sum<NT>(part, g, row, tt);
-                }
+                with_nt<NT>(n, [&](auto ntc) {
+                    constexpr int NTC = decltype(ntc)::value;
+                    warp_rows_to_part<NTC>(R.qs(s), R.d(s), q.k, q.ld_d, g, xs, tg, n, part);
+                    if (grp == n_grp - 1 && tg + NT >= nx) {
+                        __syncwarp();
+                        if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
+                    }
+                    named_bar_sync(kBarConsumers, kCT);
+                    for (int j = 0, i = epi_index(0); i < rows_valid * n; i = epi_index(++j)) {
+                        const int row = i / n;
+                        const int tt = i - row * n;
+                        q.y[(int64_t)(x0 + tg + tt) * q.rows + r0 + row] =
+                            part_sum<NTC>(part, g, row, tt);
+                    }
+                });
                 buf ^= 1;
             }
         }
@@ -539,7 +546,7 @@ q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_t
     const int nt = pick_nt(n_tok);
     if (!make_plan(max_tq, max_td, max_k, (int)std::min<int64_t>(n_tok, kMaxXRows), nt, &p.plan))
         Q8_FAIL(Q8_E_UNSUPPORTED, "q8_gemv_batched: k=%d does not fit the plan", max_k);
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * ctas_per_sm(nt), tiles));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * p.plan.ctas, tiles));
     cudaStream_t s = (cudaStream_t)stream;
     switch (nt) {
         case 1: return launch_stream(gemv_batched_kernel<1>, grid, p.plan.bytes, s, p, "gemv_batched");

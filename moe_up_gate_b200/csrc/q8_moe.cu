@@ -252,43 +252,46 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             for (int tg = 0; tg < nx; tg += NT) {
                 const int n = min(NT, nx - tg);
                 float *part = part0 + buf * kPartRows * NT;
-                warp_rows_to_part<NT>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, xs, tg, n, part);
-                if (grp == n_grp - 1 && tg + NT >= nx) {
-                    __syncwarp();
-                    if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
-                }
-                named_bar_sync(kBarConsumers, kCT);
-                for (int i = threadIdx.x; i < half_rows * n; i += kCT) {
-                    const int row = i / n;
-                    const int tt = i - row * n;
-                    const int pr = plist ? plist[x0 + tg + tt] : x0 + tg + tt;
-                    const float gv = part_sum<NT>(part, g, row, tt);
-                    const float uv = part_sum<NT>(part, g, row + half_rows, tt);
-                    const int64_t o = (int64_t)pr * p.n_ff + r0 + row;
-                    p.h[o] = silu_f(gv) * uv;
-                    if (p.g_out) p.g_out[o] = gv;
-                    if (p.u_out) p.u_out[o] = uv;
-                }
+                with_nt<NT>(n, [&](auto ntc) {
+                    constexpr int NTC = decltype(ntc)::value;
+                    warp_rows_to_part<NTC>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, xs, tg, n, part);
+                    if (grp == n_grp - 1 && tg + NT >= nx) {
+                        __syncwarp();
+                        if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
+                    }
+                    named_bar_sync(kBarConsumers, kCT);
+                    for (int j = 0, i = epi_index(0); i < half_rows * n; i = epi_index(++j)) {
+                        const int row = i / n;
+                        const int tt = i - row * n;
+                        const int pr = plist ? plist[x0 + tg + tt] : x0 + tg + tt;
+                        const float gv = part_sum<NTC>(part, g, row, tt);
+                        const float uv = part_sum<NTC>(part, g, row + half_rows, tt);
+                        const int64_t o = (int64_t)pr * p.n_ff + r0 + row;
+                        p.h[o] = silu_f(gv) * uv;
+                        if (p.g_out) p.g_out[o] = gv;
+                        if (p.u_out) p.u_out[o] = uv;
+                    }
+                });
                 buf ^= 1;
             }
         }
     }
 }
 
-static q8_status launch_up_gate(const UpGateParams &base, int64_t max_group, int64_t slots,
+static q8_status launch_up_gate(const UpGateParams &base, RowPlan rp, int64_t slots,
                                 cudaStream_t s) {
     UpGateParams p = base;
-    const int nt = pick_nt(max_group);
+    const int nt = pick_nt(rp.nt_rows);
     const int tab_words =
         p.ids ? (int)group_layout((int64_t)p.n_tok * p.n_used, p.n_mat).words : 0;
     int tq, td;
     tile_bytes(geo_pair_for_k(p.k), p.k, p.ld_d, &tq, &td);
-    if (!make_plan(tq, td, p.k, (int)std::min<int64_t>(max_group, kMaxXRows), nt, &p.plan,
+    if (!make_plan(tq, td, p.k, (int)std::min<int64_t>(rp.x_rows, kMaxXRows), nt, &p.plan,
                    tab_words))
         Q8_FAIL(Q8_E_UNSUPPORTED, "up_gate: k=%d does not fit the shared-memory plan", p.k);
     const Geo g = geo_pair_for_k(p.k);
     const int64_t tiles = slots * (p.n_ff / (g.nr / 2));
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * ctas_per_sm(nt), tiles));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * p.plan.ctas, tiles));
     switch (nt) {
         case 1: return launch_stream(up_gate_kernel<1>, grid, p.plan.bytes, s, p, "up_gate");
         case 2: return launch_stream(up_gate_kernel<2>, grid, p.plan.bytes, s, p, "up_gate");
@@ -395,7 +398,7 @@ static q8_status up_gate_entry(const char *fn, const q8_tensor *up_gate, const i
                    "%s: dense call (ids NULL) needs n_mat == 1, n_used == 1", fn);
         p.ws = nullptr;
         p.n_dense = (int)n_tok;
-        st = launch_up_gate(p, n_tok, 1, s);
+        st = launch_up_gate(p, dense_rows(n_tok), 1, s);
         if (st != Q8_OK || hq == nullptr) return st;
         // h -> Q8_0 with the activation quantizer (a 32-block of h spans
         // several weight tiles, so it is not formed inside one tile)
@@ -423,7 +426,8 @@ static q8_status up_gate_entry(const char *fn, const q8_tensor *up_gate, const i
     // (the g/u debug taps come from the dp4a kernel only)
     const bool tc = tc_eligible(up_gate, true) && P >= kTcMinPairs && !g_out && !u_out;
     p.include_big = tc ? 0 : 1;
-    st = launch_up_gate(p, n_tok, std::min<int64_t>(up_gate->n_mat, P), s);
+    st = launch_up_gate(p, routed_rows(n_tok, n_used, up_gate->n_mat),
+                        std::min<int64_t>(up_gate->n_mat, P), s);
     if (st != Q8_OK) return st;
     if (tc) {
         st = launch_tc(up_gate, true, xq, xd, nullptr, 0, n_tok, n_used, h, (const int32_t *)ws, s);
@@ -559,7 +563,7 @@ q8_status q8_moe_up_gate_swiglu_fp32(const q8_tensor *up_gate, const float *x, i
         Q8_REQUIRE(up_gate->n_mat == 1 && n_used == 1, Q8_E_SHAPE,
                    "%s: dense call (ids NULL) needs n_mat == 1, n_used == 1", fn);
         p.n_dense = (int)n_tok;
-        return launch_up_gate(p, n_tok, 1, s);
+        return launch_up_gate(p, dense_rows(n_tok), 1, s);
     }
     const GroupLayout L = group_layout(n_tok * n_used, up_gate->n_mat);
     p.lay_count = L.count;
@@ -572,7 +576,8 @@ q8_status q8_moe_up_gate_swiglu_fp32(const q8_tensor *up_gate, const float *x, i
     p.n_tok = (int)n_tok;
     p.n_mat = (int)up_gate->n_mat;
     p.err_out = err_word;
-    return launch_up_gate(p, n_tok, std::min<int64_t>(up_gate->n_mat, n_tok * n_used), s);
+    return launch_up_gate(p, routed_rows(n_tok, n_used, up_gate->n_mat),
+                          std::min<int64_t>(up_gate->n_mat, n_tok * n_used), s);
 }
 
 q8_status q8_mul_mat_id_fp32(const q8_tensor *W, const float *a, int32_t a_per_slot,

@@ -25,6 +25,8 @@
 //    activations or routing tables first waits for the preceding grid.
 #pragma once
 
+#include <type_traits>
+
 #include "q8_device.cuh"
 #include "q8_internal.h"
 #include "q8_ptx.cuh"
@@ -88,6 +90,7 @@ struct Plan {
     int off_full, off_empty, off_ring, off_xq, off_xd, off_part, off_tab;
     int tab_words;  // routing tables built in shared memory (0: none)
     int bytes;
+    int ctas;       // CTAs per SM the plan is sized for
 };
 
 __host__ inline int plan_part_floats(int nt) { return 2 * kPartRows * nt; }
@@ -97,16 +100,14 @@ __host__ inline int plan_part_floats(int nt) { return 2 * kPartRows * nt; }
 // one otherwise (register use).
 __host__ __device__ constexpr int ctas_per_sm(int nt) { return nt <= 2 ? 2 : 1; }
 // Shared memory one CTA may use (the SM has 228 KB; 1 KB per CTA is reserved).
-__host__ inline int smem_budget(int nt) {
-    return ctas_per_sm(nt) == 2 ? (228 * 1024) / 2 - 1024 : kSmemLimit;
-}
+__host__ inline int smem_budget(int ctas) { return ctas == 2 ? (228 * 1024) / 2 - 1024 : kSmemLimit; }
 
 // tile_qs / tile_d: the largest tile's quant and scale bytes; xrows:
 // activation rows wanted in shared memory at once; tab_words: int32 words of
 // routing tables to build in shared memory.  As many stages as fit.
-__host__ inline bool make_plan(int tile_qs, int tile_d, int max_k, int xrows, int nt, Plan *out,
-                               int tab_words = 0) {
-    const int budget = smem_budget(nt);
+__host__ inline bool make_plan_ctas(int tile_qs, int tile_d, int max_k, int xrows, int nt,
+                                    int ctas, Plan *out, int tab_words) {
+    const int budget = smem_budget(ctas);
     const int tab_bytes = ((tab_words * 4 + 15) / 16) * 16;
     const int stage_qs = round128(tile_qs);
     const int stage_bytes = stage_qs + round128(tile_d);
@@ -135,10 +136,21 @@ __host__ inline bool make_plan(int tile_qs, int tile_d, int max_k, int xrows, in
             p.off_tab = p.off_part + part_bytes;
             p.tab_words = tab_words;
             p.bytes = p.off_tab + tab_bytes;
+            p.ctas = ctas;
             *out = p;
             return true;
         }
     }
+}
+
+// Two CTAs per SM where the kernel allows it and each still gets three ring
+// stages; else one CTA per SM with the whole shared memory.
+__host__ inline bool make_plan(int tile_qs, int tile_d, int max_k, int xrows, int nt, Plan *out,
+                               int tab_words = 0) {
+    if (ctas_per_sm(nt) == 2 &&
+        make_plan_ctas(tile_qs, tile_d, max_k, xrows, nt, 2, out, tab_words) && out->stages >= 3)
+        return true;
+    return make_plan_ctas(tile_qs, tile_d, max_k, xrows, nt, 1, out, tab_words);
 }
 
 // Contiguous run of tiles for this CTA.
@@ -237,12 +249,14 @@ __device__ __forceinline__ void cta_group(const int32_t *__restrict__ ids, int n
     const int P = n_tok * n_used;
     int *cnt = tab + L.count;
     int *cursor = tab + L.list_big;
+    int *sid = tab + L.pairs;  // the ids, read once; the pair list overwrites them below
     for (int e = threadIdx.x; e < n_mat; e += blockDim.x) cnt[e] = 0;
+    for (int p = threadIdx.x; p < P; p += blockDim.x) sid[p] = ids[p];
     if (threadIdx.x == 0) tab[WS_ERR] = 0;
     __syncthreads();
     int err = 0;
     for (int p = threadIdx.x; p < P; p += blockDim.x) {
-        const int e = ids[p];
+        const int e = sid[p];
         if (e < 0 || e >= n_mat) {
             err |= ERR_ID_RANGE;
             continue;
@@ -250,10 +264,13 @@ __device__ __forceinline__ void cta_group(const int32_t *__restrict__ ids, int n
         atomicAdd(&cnt[e], 1);
         const int t = p / n_used;
         for (int s2 = t * n_used; s2 < p; ++s2)
-            if (ids[s2] == e) err |= ERR_ID_REPEAT;
+            if (sid[s2] == e) err |= ERR_ID_REPEAT;
     }
     if (err) atomicOr(&tab[WS_ERR], err);
     __syncthreads();
+    // each thread keeps the ids of the pairs warp 0 will scatter, because the
+    // scatter writes the sorted pairs over sid
+    
     const int lane = threadIdx.x & 31;
     if (threadIdx.x < 32) {
         int running = 0, n_small = 0;
@@ -285,7 +302,7 @@ __device__ __forceinline__ void cta_group(const int32_t *__restrict__ ids, int n
         __syncwarp();
         for (int base = 0; base < P; base += 32) {
             const int p = base + lane;
-            const int e = p < P ? ids[p] : -1;
+            const int e = p < P ? ids[p] : -1;  // global (L1/L2 hit): sid is being overwritten
             const bool valid = e >= 0 && e < n_mat;
             const int key = valid ? e : n_mat + lane;
             const unsigned m = __match_any_sync(0xffffffffu, key);
@@ -331,18 +348,19 @@ __device__ __forceinline__ void stage_q8(const XStage &xs, const int8_t *__restr
 
 // Quantize fp32 rows arow(j) of af (k floats apart), j < n, into the stage,
 // one warp per 32-block, by the Q8_0 rule.  Each warp first issues the loads
-// of up to 8 of its blocks, then quantizes them (one memory latency per 8
-// blocks instead of one per block).
+// of up to 16 of its blocks, then quantizes them (one memory latency per 16
+// blocks, i.e. per row of up to 4096 for the whole CTA).
 template <class RowFn>
 __device__ __forceinline__ void stage_f32(const XStage &xs, const float *__restrict__ af, int k,
                                           int n, RowFn arow) {
+    constexpr int kBatch = 16;
     const int nb = k / QK;
     const int lane = threadIdx.x & 31;
     const int total = n * nb;
-    for (int b0 = threadIdx.x >> 5; b0 < total; b0 += kCW * 8) {
-        float v[8];
+    for (int b0 = threadIdx.x >> 5; b0 < total; b0 += kCW * kBatch) {
+        float v[kBatch];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < kBatch; ++i) {
             const int blk = b0 + i * kCW;
             v[i] = 0.0f;
             if (blk < total) {
@@ -352,7 +370,7 @@ __device__ __forceinline__ void stage_f32(const XStage &xs, const float *__restr
             }
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < kBatch; ++i) {
             const int blk = b0 + i * kCW;  // warp-uniform
             if (blk < total) {
                 const int j = blk / nb;
@@ -515,6 +533,41 @@ __device__ __forceinline__ void warp_rows_to_part(const int8_t *sq, const uint16
     else if (g.rpw == 2) Q8_ROWS_CASE(2)
     else Q8_ROWS_CASE(1)
 #undef Q8_ROWS_CASE
+}
+
+// Calls f(std::integral_constant<int, NTC>) with the smallest NTC in
+// {1, 2, 4, 8}, NTC <= NTMAX, that covers n activation rows (n warp-uniform),
+// so a pass over few rows pays for few rows.
+template <int NTMAX, class F>
+__device__ __forceinline__ void with_nt(int n, F &&f) {
+    if constexpr (NTMAX >= 8) {
+        if (n > 4) {
+            f(std::integral_constant<int, 8>{});
+            return;
+        }
+    }
+    if constexpr (NTMAX >= 4) {
+        if (n > 2) {
+            f(std::integral_constant<int, 4>{});
+            return;
+        }
+    }
+    if constexpr (NTMAX >= 2) {
+        if (n > 1) {
+            f(std::integral_constant<int, 2>{});
+            return;
+        }
+    }
+    f(std::integral_constant<int, 1>{});
+}
+
+// The i-th epilogue output of a pass is taken by consumer thread
+// epi_thread(i): outputs go round-robin over the 8 warps first, so that a
+// pass with few outputs spreads their latency instead of queueing it in one
+// warp.  epi_index inverts it for the calling thread (j-th round).
+__device__ __forceinline__ int epi_index(int j) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    return (j * 32 + lane) * kCW + warp;
 }
 
 // Row sum of tile row `row`, activation t, from the warp partials (seg order).
