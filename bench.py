@@ -94,6 +94,14 @@ class Dist:
             self.pg.destroy_process_group()
 
 
+def job_rate(dist, units_per_rank, local_ms):
+    """Whole-job rate of N replicas: the units every rank processed over the
+    slowest rank's device time (max over ranks).  Returns (rate per second,
+    that time in ms)."""
+    ms = dist.max(local_ms)
+    return units_per_rank * dist.world / (ms / 1e3), ms
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
@@ -699,12 +707,12 @@ def main():
             wl.e2e_post()
         e2e_ev[1].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = dist.max(e2e_ev[0].elapsed_time(e2e_ev[1]))
+    e2e_rate, e2e_ms = job_rate(dist, wl.tokens_per_step * K, e2e_ev[0].elapsed_time(e2e_ev[1]))
     dist.barrier()
 
     n = dist.world
-    tokens = wl.tokens_per_step * K * n
-    value = tokens / (total_ms / 1e3)
+    # total_ms is already the max over ranks of each round (one_round)
+    value, total_ms = job_rate(dist, wl.tokens_per_step * K, total_ms)
     step_bytes = statistics.mean(wl.unique_bytes(W + i) for i in range(K))
     peak, peak_kind = measured_peak()
     if isinstance(wl, LlamaDecode):
@@ -729,7 +737,7 @@ def main():
                      "bytes_per_launch": dom_bytes, "avg_launch_ms": dom_avg_ms,
                      "traffic": traffic},
         "clocks": clk,
-        "e2e": {"value": wl.tokens_per_step * K * n / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": e2e_rate, "unit": "tokens/s",
                 "h2d_bytes_per_step": wl.h2d_bytes, "d2h_bytes_per_step": wl.d2h_bytes},
         "gpu_launches": wl.launches_per_step * K,
     }

@@ -61,7 +61,9 @@ template <int NT>
 __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     stream_matmul_kernel(const __grid_constant__ MatmulParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
+    Q8_TRACE(0);
     const Ring R = ring_init(smem, p.plan);
+    Q8_TRACE(1);
     const Geo g = geo_for_k(p.k);
     const int tpm = (p.rows + g.nr - 1) / g.nr;
     griddep_launch_dependents();
@@ -77,6 +79,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
         L.pairs = p.lay_pairs;
         cta_group(p.ids, p.n_tok, p.n_used, p.n_mat, L, stab, p.err_out);
         tab = stab;
+        Q8_TRACE(3);
     } else if (tab) {
         griddep_wait();
     }
@@ -108,6 +111,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
         return;
     }
     if (!routed) griddep_wait();
+    Q8_TRACE(2);
     const XStage xs{reinterpret_cast<int8_t *>(smem + p.plan.off_xq),
                     reinterpret_cast<float *>(smem + p.plan.off_xd)};
     float *part0 = reinterpret_cast<float *>(smem + p.plan.off_part);
@@ -116,6 +120,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     for (int64_t t = tb; t < te; ++t, ++it) {
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_matmul);
+        Q8_TRACE(6);
         const int mi = (int)(t / tpm), ti = (int)(t % tpm);
         const int e = routed ? expert(mi) : 0;
         const int cnt = routed ? tab[p.lay_count + e] : p.n_dense;
@@ -140,6 +145,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                 else
                     stage_q8(xs, p.aq, p.ad, p.k, nx, arow);
                 named_bar_sync(kBarConsumers, kCT);
+                Q8_TRACE(7);
                 staged_mi = mi;
                 staged_grp = grp;
             }
@@ -149,17 +155,20 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                 with_nt<NT>(n, [&](auto ntc) {
                     constexpr int NTC = decltype(ntc)::value;
                     warp_rows_to_part<NTC>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, xs, tg, n, part);
+                    Q8_TRACE(8);
                     if (grp == n_grp - 1 && tg + NT >= nx) {  // last read of this stage
                         __syncwarp();
                         if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
                     }
                     named_bar_sync(kBarConsumers, kCT);
-                    for (int j = 0, i = epi_index(0); i < rows_valid * n; i = epi_index(++j)) {
+                    Q8_TRACE(9);
+                    for (int i = threadIdx.x; i < rows_valid * n; i += kCT) {
                         const int row = i / n;
                         const int tt = i - row * n;
                         const int pr = plist ? plist[x0 + tg + tt] : x0 + tg + tt;
                         p.y[(int64_t)pr * p.rows + r0 + row] = part_sum<NTC>(part, g, row, tt);
                     }
+                    Q8_TRACE(10);
                 });
                 buf ^= 1;
             }
@@ -339,7 +348,9 @@ template <int NT>
 __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     gemv_batched_kernel(const __grid_constant__ GemvBatchParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
+    Q8_TRACE(0);
     const Ring R = ring_init(smem, p.plan);
+    Q8_TRACE(1);
     griddep_launch_dependents();
     int64_t tb, te;
     my_tiles(p.total_tiles, &tb, &te);
@@ -364,6 +375,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
         return;
     }
     griddep_wait();
+    Q8_TRACE(2);
     const XStage xs{reinterpret_cast<int8_t *>(smem + p.plan.off_xq),
                     reinterpret_cast<float *>(smem + p.plan.off_xd)};
     float *part0 = reinterpret_cast<float *>(smem + p.plan.off_part);
@@ -376,6 +388,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
         const Geo g = geo_for_k(q.k);
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_matmul);
+        Q8_TRACE(6);
         const int r0 = (int)(t - q.tile_begin) * g.nr;
         const int rows_valid = min(g.nr, q.rows - r0);
         const int n_grp = (p.n_tok + xmax - 1) / xmax;
@@ -385,6 +398,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             if (cur != staged || grp != staged_grp) {
                 stage_f32(xs, q.x, q.k, nx, [&](int j) { return x0 + j; });
                 named_bar_sync(kBarConsumers, kCT);
+                Q8_TRACE(7);
                 staged = cur;
                 staged_grp = grp;
             }
@@ -394,17 +408,20 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                 with_nt<NT>(n, [&](auto ntc) {
                     constexpr int NTC = decltype(ntc)::value;
                     warp_rows_to_part<NTC>(R.qs(s), R.d(s), q.k, q.ld_d, g, xs, tg, n, part);
+                    Q8_TRACE(8);
                     if (grp == n_grp - 1 && tg + NT >= nx) {
                         __syncwarp();
                         if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
                     }
                     named_bar_sync(kBarConsumers, kCT);
-                    for (int j = 0, i = epi_index(0); i < rows_valid * n; i = epi_index(++j)) {
+                    Q8_TRACE(9);
+                    for (int i = threadIdx.x; i < rows_valid * n; i += kCT) {
                         const int row = i / n;
                         const int tt = i - row * n;
                         q.y[(int64_t)(x0 + tg + tt) * q.rows + r0 + row] =
                             part_sum<NTC>(part, g, row, tt);
                     }
+                    Q8_TRACE(10);
                 });
                 buf ^= 1;
             }

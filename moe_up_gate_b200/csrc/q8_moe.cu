@@ -163,7 +163,9 @@ template <int NT>
 __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     up_gate_kernel(const __grid_constant__ UpGateParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
+    Q8_TRACE(0);
     const Ring R = ring_init(smem, p.plan);
+    Q8_TRACE(1);
     const Geo g = geo_pair_for_k(p.k);
     const int half_rows = g.nr / 2;
     const int tpm = p.n_ff / half_rows;
@@ -180,6 +182,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
         L.pairs = p.lay_pairs;
         cta_group(p.ids, p.n_tok, p.n_used, p.n_mat, L, stab, p.err_out);
         tab = stab;
+        Q8_TRACE(3);
     } else if (tab) {
         griddep_wait();
     }
@@ -215,6 +218,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
         return;
     }
     if (!routed) griddep_wait();
+    Q8_TRACE(2);
     const XStage xs{reinterpret_cast<int8_t *>(smem + p.plan.off_xq),
                     reinterpret_cast<float *>(smem + p.plan.off_xd)};
     float *part0 = reinterpret_cast<float *>(smem + p.plan.off_part);
@@ -223,6 +227,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     for (int64_t t = tb; t < te; ++t, ++it) {
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_moe);
+        Q8_TRACE(6);
         const int mi = (int)(t / tpm), ti = (int)(t % tpm);
         const int e = routed ? expert(mi) : 0;
         const int cnt = routed ? tab[p.lay_count + e] : p.n_dense;
@@ -246,6 +251,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                 else
                     stage_q8(xs, p.xq, p.xd, p.k, nx, arow);
                 named_bar_sync(kBarConsumers, kCT);
+                Q8_TRACE(7);
                 staged_mi = mi;
                 staged_grp = grp;
             }
@@ -255,12 +261,14 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                 with_nt<NT>(n, [&](auto ntc) {
                     constexpr int NTC = decltype(ntc)::value;
                     warp_rows_to_part<NTC>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, xs, tg, n, part);
+                    Q8_TRACE(8);
                     if (grp == n_grp - 1 && tg + NT >= nx) {
                         __syncwarp();
                         if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
                     }
                     named_bar_sync(kBarConsumers, kCT);
-                    for (int j = 0, i = epi_index(0); i < half_rows * n; i = epi_index(++j)) {
+                    Q8_TRACE(9);
+                    for (int i = threadIdx.x; i < half_rows * n; i += kCT) {
                         const int row = i / n;
                         const int tt = i - row * n;
                         const int pr = plist ? plist[x0 + tg + tt] : x0 + tg + tt;
@@ -271,6 +279,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                         if (p.g_out) p.g_out[o] = gv;
                         if (p.u_out) p.u_out[o] = uv;
                     }
+                    Q8_TRACE(10);
                 });
                 buf ^= 1;
             }

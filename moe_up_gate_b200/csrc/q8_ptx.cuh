@@ -11,6 +11,13 @@
 
 #include <stdint.h>
 
+// Trace points of the kernels (numbered phases of a CTA's timeline).  They
+// compile to nothing unless the build defines Q8_TRACE(id) to a recorder
+// before this header is included.
+#ifndef Q8_TRACE
+#define Q8_TRACE(id) ((void)0)
+#endif
+
 namespace q8 {
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

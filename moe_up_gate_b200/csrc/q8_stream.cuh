@@ -213,10 +213,12 @@ template <class SrcFn>
 __device__ __forceinline__ void produce(const Ring &R, int64_t tb, int64_t te, SrcFn src,
                                         int *err) {
     int it = 0;
+    Q8_TRACE(20);
     for (int64_t t = tb; t < te; ++t, ++it) {
         const int s = it % R.stages;
         const int round = it / R.stages;
         if (round > 0) mbar_wait(&R.empty[s], (round - 1) & 1, err);
+        Q8_TRACE(21);
         const TileSrc ts = src(t);
         const int k = ts.k;
         const int ld_d = ts.ld_d;
@@ -230,8 +232,10 @@ __device__ __forceinline__ void produce(const Ring &R, int64_t tb, int64_t te, S
             bulk_g2s(R.d(s) + (size_t)ts.row_off1 * ld_d, ts.d1, db1, &R.full[s]);
         }
     }
+    Q8_TRACE(22);
     const int first = it > R.stages ? it - R.stages : 0;
     for (int j = first; j < it; ++j) mbar_wait(&R.full[j % R.stages], (j / R.stages) & 1, err);
+    Q8_TRACE(23);
 }
 
 // ---------------------------------------------------------------------------
@@ -348,12 +352,12 @@ __device__ __forceinline__ void stage_q8(const XStage &xs, const int8_t *__restr
 
 // Quantize fp32 rows arow(j) of af (k floats apart), j < n, into the stage,
 // one warp per 32-block, by the Q8_0 rule.  Each warp first issues the loads
-// of up to 16 of its blocks, then quantizes them (one memory latency per 16
-// blocks, i.e. per row of up to 4096 for the whole CTA).
+// of up to 8 of its blocks, then quantizes them (one memory latency per 8
+// blocks).
 template <class RowFn>
 __device__ __forceinline__ void stage_f32(const XStage &xs, const float *__restrict__ af, int k,
                                           int n, RowFn arow) {
-    constexpr int kBatch = 16;
+    constexpr int kBatch = 8;
     const int nb = k / QK;
     const int lane = threadIdx.x & 31;
     const int total = n * nb;
@@ -559,15 +563,6 @@ __device__ __forceinline__ void with_nt(int n, F &&f) {
         }
     }
     f(std::integral_constant<int, 1>{});
-}
-
-// The i-th epilogue output of a pass is taken by consumer thread
-// epi_thread(i): outputs go round-robin over the 8 warps first, so that a
-// pass with few outputs spreads their latency instead of queueing it in one
-// warp.  epi_index inverts it for the calling thread (j-th round).
-__device__ __forceinline__ int epi_index(int j) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    return (j * 32 + lane) * kCW + warp;
 }
 
 // Row sum of tile row `row`, activation t, from the warp partials (seg order).
