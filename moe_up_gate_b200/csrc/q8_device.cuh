@@ -37,6 +37,26 @@ __device__ __forceinline__ float scale_value(uint16_t bits) {
     return __half2float(__ushort_as_half(bits));
 }
 
+// One 32-block held by one thread (v[0..31]) quantized by the rule above:
+// the codes packed four per word (byte i of word w is element 4w + i);
+// returns d32.  amax is the exact maximum of |v|, as in the warp form.
+__device__ __forceinline__ float quantize_block_thread(const float (&v)[32], uint32_t (&q)[8]) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const float d32 = block_scale(amax);
+    const float id = block_inv_scale(d32);
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            word |= ((uint32_t)quantize_one(v[4 * w + b], id) & 0xffu) << (8 * b);
+        q[w] = word;
+    }
+    return d32;
+}
+
 // ---------------------------------------------------------------------------
 // warp helpers
 // ---------------------------------------------------------------------------

@@ -106,7 +106,28 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                 ts.ld_d = (int)p.ld_d;
                 return ts;
             };
-            produce(R, tb, te, src, &g_err_matmul);
+            if (p.af && R.raw_rows > 0) {
+                XJobs J;
+                const int xmax = p.plan.xmax;
+                auto jobs = [&](int64_t t, int when) {
+                    const int mi = (int)(t / tpm);
+                    const int e = routed ? expert(mi) : 0;
+                    const int cnt = routed ? tab[p.lay_count + e] : p.n_dense;
+                    const int32_t *plist = routed ? tab + p.lay_pairs + tab[p.lay_offset + e] : nullptr;
+                    const int n_grp = (cnt + xmax - 1) / xmax;
+                    for (int grp = when; grp < (when == 0 ? min(1, n_grp) : n_grp); ++grp) {
+                        const int x0 = grp * xmax;
+                        produce_job(R, J, mi, grp, min(xmax, cnt - x0), p.k, [&](int j) {
+                            const int pr = plist ? plist[x0 + j] : x0 + j;
+                            const int r = (!routed || p.a_per_slot) ? pr : pr / p.n_used;
+                            return p.af + (int64_t)r * p.k;
+                        }, &g_err_matmul);
+                    }
+                };
+                produce(R, tb, te, src, &g_err_matmul, jobs);
+            } else {
+                produce(R, tb, te, src, &g_err_matmul);
+            }
         }
         return;
     }
@@ -117,6 +138,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     float *part0 = reinterpret_cast<float *>(smem + p.plan.off_part);
     const int xmax = p.plan.xmax;
     int buf = 0, staged_mi = -1, staged_grp = -1, it = 0;
+    XJobs J;
     for (int64_t t = tb; t < te; ++t, ++it) {
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_matmul);
@@ -136,12 +158,15 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             const int x0 = grp * xmax;
             const int nx = min(xmax, cnt - x0);
             if (mi != staged_mi || grp != staged_grp) {
+                // after passes without a barrier every warp must be done
+                // with the staged rows before they are replaced
+                if (g.wpr == 1 && staged_mi >= 0) named_bar_sync(kBarConsumers, kCT);
                 auto arow = [&](int j) {
                     const int pr = plist ? plist[x0 + j] : x0 + j;
                     return (!routed || p.a_per_slot) ? pr : pr / p.n_used;
                 };
                 if (p.af)
-                    stage_f32(xs, p.af, p.k, nx, arow);
+                    stage_job_f32(R, J, xs, p.af, p.k, nx, arow, &g_err_matmul);
                 else
                     stage_q8(xs, p.aq, p.ad, p.k, nx, arow);
                 named_bar_sync(kBarConsumers, kCT);
@@ -154,6 +179,24 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                 float *part = part0 + buf * kPartRows * NT;
                 with_nt<NT>(n, [&](auto ntc) {
                     constexpr int NTC = decltype(ntc)::value;
+                    if (g.wpr == 1) {
+                        // whole rows per warp: each sum is final, written
+                        // by the lane that holds it (no barrier)
+                        warp_rows<NTC>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, xs, tg, n,
+                                       [&](int row, int tt, float v) {
+                                           if (row < rows_valid && tt < n) {
+                                               const int pr = plist ? plist[x0 + tg + tt]
+                                                                    : x0 + tg + tt;
+                                               p.y[(int64_t)pr * p.rows + r0 + row] = v;
+                                           }
+                                       });
+                        Q8_TRACE(8);
+                        if (grp == n_grp - 1 && tg + NT >= nx) {
+                            __syncwarp();
+                            if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
+                        }
+                        return;
+                    }
                     warp_rows_to_part<NTC>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, xs, tg, n, part);
                     Q8_TRACE(8);
                     if (grp == n_grp - 1 && tg + NT >= nx) {  // last read of this stage
@@ -201,7 +244,7 @@ q8_status launch_matmul(const MatmulParams &base, RowPlan rp, int64_t max_tiles,
     int tq, td;
     tile_bytes(geo_for_k(p.k), p.k, p.ld_d, &tq, &td);
     if (!make_plan(tq, td, p.k, (int)std::min<int64_t>(rp.x_rows, kMaxXRows), nt, &p.plan,
-                   tab_words))
+                   tab_words, p.af != nullptr && aligned16(p.af)))
         Q8_FAIL(Q8_E_UNSUPPORTED, "matmul: k=%d does not fit the shared-memory plan", p.k);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * p.plan.ctas, max_tiles));
     switch (nt) {
@@ -370,7 +413,25 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                 ts.ld_d = q.ld_d;
                 return ts;
             };
-            produce(R, tb, te, src, &g_err_matmul);
+            if (R.raw_rows > 0) {
+                XJobs J;
+                int jc = cur;
+                const int xmax = p.plan.xmax;
+                const int n_grp = (p.n_tok + xmax - 1) / xmax;
+                auto jobs = [&](int64_t t, int when) {
+                    while (jc + 1 < p.n_desc && p.pr[jc + 1].tile_begin <= t) ++jc;
+                    const GemvProblem &q = p.pr[jc];
+                    for (int grp = when; grp < (when == 0 ? min(1, n_grp) : n_grp); ++grp) {
+                        const int x0 = grp * xmax;
+                        produce_job(R, J, jc, grp, min(xmax, p.n_tok - x0), q.k,
+                                    [&](int j) { return q.x + (int64_t)(x0 + j) * q.k; },
+                                    &g_err_matmul);
+                    }
+                };
+                produce(R, tb, te, src, &g_err_matmul, jobs);
+            } else {
+                produce(R, tb, te, src, &g_err_matmul);
+            }
         }
         return;
     }
@@ -382,6 +443,8 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     const int xmax = p.plan.xmax;
     int buf = 0, staged = -1, staged_grp = -1, it = 0;
     int cur = tb < te ? find_problem(p, tb) : 0;
+    XJobs J;
+    bool unsynced = false;  // passes without a barrier since the last one
     for (int64_t t = tb; t < te; ++t, ++it) {
         while (cur + 1 < p.n_desc && p.pr[cur + 1].tile_begin <= t) ++cur;
         const GemvProblem &q = p.pr[cur];
@@ -396,7 +459,12 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             const int x0 = grp * xmax;
             const int nx = min(xmax, p.n_tok - x0);
             if (cur != staged || grp != staged_grp) {
-                stage_f32(xs, q.x, q.k, nx, [&](int j) { return x0 + j; });
+                // after passes without a barrier every warp must be done
+                // with the staged rows before they are replaced
+                if (unsynced) named_bar_sync(kBarConsumers, kCT);
+                unsynced = false;
+                stage_job_f32(R, J, xs, q.x, q.k, nx, [&](int j) { return x0 + j; },
+                              &g_err_matmul);
                 named_bar_sync(kBarConsumers, kCT);
                 Q8_TRACE(7);
                 staged = cur;
@@ -407,6 +475,22 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                 float *part = part0 + buf * kPartRows * NT;
                 with_nt<NT>(n, [&](auto ntc) {
                     constexpr int NTC = decltype(ntc)::value;
+                    if (g.wpr == 1) {
+                        // whole rows per warp: each sum is final, written
+                        // by the lane that holds it (no barrier)
+                        warp_rows<NTC>(R.qs(s), R.d(s), q.k, q.ld_d, g, xs, tg, n,
+                                       [&](int row, int tt, float v) {
+                                           if (row < rows_valid && tt < n)
+                                               q.y[(int64_t)(x0 + tg + tt) * q.rows + r0 + row] = v;
+                                       });
+                        Q8_TRACE(8);
+                        if (grp == n_grp - 1 && tg + NT >= nx) {
+                            __syncwarp();
+                            if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
+                        }
+                        unsynced = true;
+                        return;
+                    }
                     warp_rows_to_part<NTC>(R.qs(s), R.d(s), q.k, q.ld_d, g, xs, tg, n, part);
                     Q8_TRACE(8);
                     if (grp == n_grp - 1 && tg + NT >= nx) {
@@ -561,7 +645,8 @@ q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_t
     Q8_REQUIRE(tiles < (1LL << 31), Q8_E_SHAPE, "q8_gemv_batched: too many tiles");
     p.total_tiles = (int)tiles;
     const int nt = pick_nt(n_tok);
-    if (!make_plan(max_tq, max_td, max_k, (int)std::min<int64_t>(n_tok, kMaxXRows), nt, &p.plan))
+    if (!make_plan(max_tq, max_td, max_k, (int)std::min<int64_t>(n_tok, kMaxXRows), nt, &p.plan,
+                   0, true))
         Q8_FAIL(Q8_E_UNSUPPORTED, "q8_gemv_batched: k=%d does not fit the plan", max_k);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * p.plan.ctas, tiles));
     cudaStream_t s = (cudaStream_t)stream;

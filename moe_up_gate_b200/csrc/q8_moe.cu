@@ -213,7 +213,27 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                 ts.ld_d = (int)p.ld_d;
                 return ts;
             };
-            produce(R, tb, te, src, &g_err_moe);
+            if (p.xf && R.raw_rows > 0) {
+                XJobs J;
+                const int xmax = p.plan.xmax;
+                auto jobs = [&](int64_t t, int when) {
+                    const int mi = (int)(t / tpm);
+                    const int e = routed ? expert(mi) : 0;
+                    const int cnt = routed ? tab[p.lay_count + e] : p.n_dense;
+                    const int32_t *plist = routed ? tab + p.lay_pairs + tab[p.lay_offset + e] : nullptr;
+                    const int n_grp = (cnt + xmax - 1) / xmax;
+                    for (int grp = when; grp < (when == 0 ? min(1, n_grp) : n_grp); ++grp) {
+                        const int x0 = grp * xmax;
+                        produce_job(R, J, mi, grp, min(xmax, cnt - x0), p.k, [&](int j) {
+                            const int pr = plist ? plist[x0 + j] : x0 + j;
+                            return p.xf + (int64_t)(routed ? pr / p.n_used : pr) * p.k;
+                        }, &g_err_moe);
+                    }
+                };
+                produce(R, tb, te, src, &g_err_moe, jobs);
+            } else {
+                produce(R, tb, te, src, &g_err_moe);
+            }
         }
         return;
     }
@@ -224,6 +244,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     float *part0 = reinterpret_cast<float *>(smem + p.plan.off_part);
     const int xmax = p.plan.xmax;
     int buf = 0, staged_mi = -1, staged_grp = -1, it = 0;
+    XJobs J;
     for (int64_t t = tb; t < te; ++t, ++it) {
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_moe);
@@ -242,12 +263,15 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             const int x0 = grp * xmax;
             const int nx = min(xmax, cnt - x0);
             if (mi != staged_mi || grp != staged_grp) {
+                // after passes without a barrier every warp must be done
+                // with the staged rows before they are replaced
+                if (g.wpr == 1 && staged_mi >= 0) named_bar_sync(kBarConsumers, kCT);
                 auto arow = [&](int j) {
                     const int pr = plist ? plist[x0 + j] : x0 + j;
                     return routed ? pr / p.n_used : pr;
                 };
                 if (p.xf)
-                    stage_f32(xs, p.xf, p.k, nx, arow);
+                    stage_job_f32(R, J, xs, p.xf, p.k, nx, arow, &g_err_moe);
                 else
                     stage_q8(xs, p.xq, p.xd, p.k, nx, arow);
                 named_bar_sync(kBarConsumers, kCT);
@@ -260,6 +284,26 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                 float *part = part0 + buf * kPartRows * NT;
                 with_nt<NT>(n, [&](auto ntc) {
                     constexpr int NTC = decltype(ntc)::value;
+                    if (g.wpr == 1) {
+                        // whole rows per warp: each warp forms h of its rows
+                        warp_pairs<NTC>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, half_rows, xs, tg,
+                                        n, [&](int row, int tt, float gv, float uv) {
+                                            if (tt < n) {
+                                                const int pr = plist ? plist[x0 + tg + tt]
+                                                                     : x0 + tg + tt;
+                                                const int64_t o = (int64_t)pr * p.n_ff + r0 + row;
+                                                p.h[o] = silu_f(gv) * uv;
+                                                if (p.g_out) p.g_out[o] = gv;
+                                                if (p.u_out) p.u_out[o] = uv;
+                                            }
+                                        });
+                        Q8_TRACE(8);
+                        if (grp == n_grp - 1 && tg + NT >= nx) {
+                            __syncwarp();
+                            if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
+                        }
+                        return;
+                    }
                     warp_rows_to_part<NTC>(R.qs(s), R.d(s), p.k, (int)p.ld_d, g, xs, tg, n, part);
                     Q8_TRACE(8);
                     if (grp == n_grp - 1 && tg + NT >= nx) {
@@ -296,7 +340,7 @@ static q8_status launch_up_gate(const UpGateParams &base, RowPlan rp, int64_t sl
     int tq, td;
     tile_bytes(geo_pair_for_k(p.k), p.k, p.ld_d, &tq, &td);
     if (!make_plan(tq, td, p.k, (int)std::min<int64_t>(rp.x_rows, kMaxXRows), nt, &p.plan,
-                   tab_words))
+                   tab_words, p.xf != nullptr && aligned16(p.xf)))
         Q8_FAIL(Q8_E_UNSUPPORTED, "up_gate: k=%d does not fit the shared-memory plan", p.k);
     const Geo g = geo_pair_for_k(p.k);
     const int64_t tiles = slots * (p.n_ff / (g.nr / 2));

@@ -25,6 +25,7 @@
 //    activations or routing tables first waits for the preceding grid.
 #pragma once
 
+#include <algorithm>
 #include <type_traits>
 
 #include "q8_device.cuh"
@@ -45,27 +46,29 @@ constexpr int kMaxXRows = 16;           // activation rows staged at once (at mo
 // Tile geometry: rows per tile, warps per row (the row's blocks are split
 // into wpr segments, one per warp), rows per warp (kCW * rpw / wpr == nr).
 // A warp takes rpw rows at once, so each activation block it loads from
-// shared memory serves rpw weight rows.  A tile holds at most 32 KB of
-// quants.  The order of a row's floating-point sum depends on wpr and k
-// only, and wpr is a function of k, so every kernel sums a row the same way.
+// shared memory serves rpw weight rows.  Up to k = 4096 a warp owns whole
+// rows (wpr = 1): its sums are final and need no exchange between warps.
+// The order of a row's floating-point sum depends on wpr and k only, and wpr
+// is a function of k, so every kernel sums a row the same way.
 struct Geo {
     int nr, wpr, rpw;
 };
-__host__ __device__ inline int wpr_for_k(int k) {
-    return k <= 1024 ? 1 : k <= 2048 ? 2 : k <= 4096 ? 4 : 8;
-}
-// Plain row tiles.
+__host__ __device__ inline int wpr_for_k(int k) { return k <= 4096 ? 1 : 8; }
+// Plain row tiles (at most 32 KB of quants).
 __host__ __device__ inline Geo geo_for_k(int k) {
     if (k <= 768) return {40, 1, 5};
     if (k <= 1024) return {32, 1, 4};
-    if (k <= 2048) return {16, 2, 4};
-    if (k <= 4096) return {8, 4, 4};
+    if (k <= 2048) return {16, 1, 2};
+    if (k <= 4096) return {8, 1, 1};
     if (k <= 8192) return {4, 8, 4};
     return {2, 8, 2};
 }
-// Gate/up tiles: nr/2 gate rows and the nr/2 matching up rows; nr/2 divides 32.
+// Gate/up tiles: nr/2 gate rows and the nr/2 matching up rows; nr/2 divides
+// 32.  With whole rows per warp, warp w owns gate rows w*rpw/2 .. and the
+// matching up rows, so it forms h itself.
 __host__ __device__ inline Geo geo_pair_for_k(int k) {
     if (k <= 1024) return {32, 1, 4};
+    if (k <= 4096) return {16, 1, 2};
     return geo_for_k(k);
 }
 
@@ -91,7 +94,14 @@ struct Plan {
     int tab_words;  // routing tables built in shared memory (0: none)
     int bytes;
     int ctas;       // CTAs per SM the plan is sized for
+    // fp32 activation rows the producer copies ahead into the raw slot
+    // (0: the consumers load them from global memory themselves)
+    int raw_rows;
+    int off_xfull, off_xempty, off_raw;
 };
+
+// Bytes of the raw activation slot at most (fp32 rows copied by the producer).
+constexpr int kRawSlotBytes = 16 * 1024;
 
 __host__ inline int plan_part_floats(int nt) { return 2 * kPartRows * nt; }
 
@@ -106,7 +116,7 @@ __host__ inline int smem_budget(int ctas) { return ctas == 2 ? (228 * 1024) / 2 
 // activation rows wanted in shared memory at once; tab_words: int32 words of
 // routing tables to build in shared memory.  As many stages as fit.
 __host__ inline bool make_plan_ctas(int tile_qs, int tile_d, int max_k, int xrows, int nt,
-                                    int ctas, Plan *out, int tab_words) {
+                                    int ctas, Plan *out, int tab_words, bool raw) {
     const int budget = smem_budget(ctas);
     const int tab_bytes = ((tab_words * 4 + 15) / 16) * 16;
     const int stage_qs = round128(tile_qs);
@@ -118,7 +128,9 @@ __host__ inline bool make_plan_ctas(int tile_qs, int tile_d, int max_k, int xrow
     for (;; xmax -= nt) {
         const int x_bytes = xmax * max_k + ((xmax * p.max_nb * 4 + 15) / 16) * 16;
         const int part_bytes = plan_part_floats(nt) * 4;
-        const int fixed = 2 * kMaxStages * 8 + 128 + x_bytes + part_bytes + tab_bytes;
+        const int raw_rows = raw ? std::min(xmax, kRawSlotBytes / (4 * max_k)) : 0;
+        const int raw_bytes = raw_rows * 4 * max_k;
+        const int fixed = 256 + x_bytes + part_bytes + tab_bytes + raw_bytes;
         int stages = (budget - fixed) / stage_bytes;
         if (stages > kMaxStages) stages = kMaxStages;
         if (stages >= 2 || xmax <= nt) {
@@ -129,13 +141,17 @@ __host__ inline bool make_plan_ctas(int tile_qs, int tile_d, int max_k, int xrow
             p.xmax = xmax;
             p.off_full = 0;
             p.off_empty = kMaxStages * 8;
-            p.off_ring = 128;
+            p.off_xfull = 2 * kMaxStages * 8;
+            p.off_xempty = p.off_xfull + 8;
+            p.off_ring = 256;
             p.off_xq = p.off_ring + stages * stage_bytes;
             p.off_xd = p.off_xq + xmax * max_k;
             p.off_part = p.off_xd + ((xmax * p.max_nb * 4 + 15) / 16) * 16;
             p.off_tab = p.off_part + part_bytes;
             p.tab_words = tab_words;
-            p.bytes = p.off_tab + tab_bytes;
+            p.raw_rows = raw_rows;
+            p.off_raw = p.off_tab + tab_bytes;
+            p.bytes = p.off_raw + raw_bytes;
             p.ctas = ctas;
             *out = p;
             return true;
@@ -144,13 +160,24 @@ __host__ inline bool make_plan_ctas(int tile_qs, int tile_d, int max_k, int xrow
 }
 
 // Two CTAs per SM where the kernel allows it and each still gets three ring
-// stages; else one CTA per SM with the whole shared memory.
+// stages (or two of 44 KB and more); else one CTA per SM with the whole
+// shared memory.  raw: fp32
+// activations that the producer may copy ahead (a raw slot is reserved when
+// one row of max_k floats fits kRawSlotBytes and the ring keeps its stages).
 __host__ inline bool make_plan(int tile_qs, int tile_d, int max_k, int xrows, int nt, Plan *out,
-                               int tab_words = 0) {
-    if (ctas_per_sm(nt) == 2 &&
-        make_plan_ctas(tile_qs, tile_d, max_k, xrows, nt, 2, out, tab_words) && out->stages >= 3)
-        return true;
-    return make_plan_ctas(tile_qs, tile_d, max_k, xrows, nt, 1, out, tab_words);
+                               int tab_words = 0, bool raw = false) {
+    raw = raw && 4 * max_k <= kRawSlotBytes;
+    for (int use_raw = raw ? 1 : 0; use_raw >= 0; --use_raw) {
+        if (ctas_per_sm(nt) == 2 &&
+            make_plan_ctas(tile_qs, tile_d, max_k, xrows, nt, 2, out, tab_words, use_raw) &&
+            (out->stages >= 3 || out->stages * out->stage_bytes >= 88 * 1024))
+            return true;
+    }
+    for (int use_raw = raw ? 1 : 0; use_raw >= 0; --use_raw)
+        if (make_plan_ctas(tile_qs, tile_d, max_k, xrows, nt, 1, out, tab_words, use_raw) &&
+            (out->stages >= 3 || !use_raw))
+            return true;
+    return false;
 }
 
 // Contiguous run of tiles for this CTA.
@@ -180,6 +207,11 @@ struct Ring {
     int stages;
     int stage_bytes;
     int stage_qs;
+    // raw activation slot: fp32 rows copied by the producer (raw_rows == 0: none)
+    uint64_t *xfull;
+    uint64_t *xempty;
+    float *raw;
+    int raw_rows;
     __device__ __forceinline__ int8_t *qs(int s) const {
         return reinterpret_cast<int8_t *>(base + (size_t)s * stage_bytes);
     }
@@ -196,27 +228,74 @@ __device__ __forceinline__ Ring ring_init(unsigned char *smem, const Plan &pl) {
     R.stages = pl.stages;
     R.stage_bytes = pl.stage_bytes;
     R.stage_qs = pl.stage_qs;
+    R.xfull = reinterpret_cast<uint64_t *>(smem + pl.off_xfull);
+    R.xempty = reinterpret_cast<uint64_t *>(smem + pl.off_xempty);
+    R.raw = reinterpret_cast<float *>(smem + pl.off_raw);
+    R.raw_rows = pl.raw_rows;
     if (threadIdx.x == 0) {
         for (int s = 0; s < pl.stages; ++s) {
             mbar_init(&R.full[s], 1);
             mbar_init(&R.empty[s], kCW);
         }
+        mbar_init(R.xfull, 1);
+        mbar_init(R.xempty, kCW);
         fence_barrier_init();
     }
     __syncthreads();
     return R;
 }
 
+// Activation jobs: the consumers stage a new set of activation rows whenever
+// the (key, group) of the rows a pass needs changes.  When the rows are fp32
+// and fit the raw slot, the producer copies them into the slot in stream
+// order (right before the first weight tile that needs them), so they arrive
+// behind the weights already in flight instead of being loaded by the
+// consumers behind the whole stream; the consumers quantize them from shared
+// memory and release the slot.
+struct XJobs {
+    int key = -1, grp = -1;  // the job last seen
+    int n = 0;               // jobs that went through the raw slot
+    // true when (key, grp) starts a new job
+    __device__ __forceinline__ bool next(int k, int g) {
+        if (k == key && g == grp) return false;
+        key = k;
+        grp = g;
+        return true;
+    }
+};
+
+// Producer side of a job of nx fp32 rows of k floats, row j at row(j).
+// bulk copies of 16-byte aligned rows; no L2 eviction hint (other CTAs read
+// the same rows).
+template <class RowFn>
+__device__ __forceinline__ void produce_job(const Ring &R, XJobs &J, int key, int grp, int nx,
+                                            int k, RowFn row, int *err) {
+    if (!J.next(key, grp) || nx > R.raw_rows) return;
+    if (J.n > 0) mbar_wait(R.xempty, (J.n - 1) & 1, err);
+    const uint32_t bytes = (uint32_t)k * 4;
+    mbar_arrive_expect_tx(R.xfull, bytes * (uint32_t)nx);
+    for (int j = 0; j < nx; ++j) bulk_g2s_keep(R.raw + (size_t)j * k, row(j), bytes, R.xfull);
+    ++J.n;
+}
+
+// No activation jobs (activations staged by the consumers).
+struct NoJobs {
+    __device__ __forceinline__ void operator()(int64_t, int) const {}
+};
+
 // Producer (one lane): stream tiles [tb, te) through the ring.  src(t) gives a
-// tile's spans.  Ends after the last copies have landed.
-template <class SrcFn>
+// tile's spans; jobs(t, when) issues the activation jobs of tile t: when == 0
+// before its weights (the job of its first group), when == 1 after them (the
+// jobs of its other groups).  Ends after the last copies have landed.
+template <class SrcFn, class JobFn = NoJobs>
 __device__ __forceinline__ void produce(const Ring &R, int64_t tb, int64_t te, SrcFn src,
-                                        int *err) {
+                                        int *err, JobFn jobs = JobFn{}) {
     int it = 0;
     Q8_TRACE(20);
     for (int64_t t = tb; t < te; ++t, ++it) {
         const int s = it % R.stages;
         const int round = it / R.stages;
+        jobs(t, 0);
         if (round > 0) mbar_wait(&R.empty[s], (round - 1) & 1, err);
         Q8_TRACE(21);
         const TileSrc ts = src(t);
@@ -231,6 +310,7 @@ __device__ __forceinline__ void produce(const Ring &R, int64_t tb, int64_t te, S
             bulk_g2s(R.qs(s) + (size_t)ts.row_off1 * k, ts.q1, qb1, &R.full[s]);
             bulk_g2s(R.d(s) + (size_t)ts.row_off1 * ld_d, ts.d1, db1, &R.full[s]);
         }
+        jobs(t, 1);
     }
     Q8_TRACE(22);
     const int first = it > R.stages ? it - R.stages : 0;
@@ -251,6 +331,56 @@ __device__ __forceinline__ void cta_group(const int32_t *__restrict__ ids, int n
                                           int n_mat, const GroupLayout &L, int32_t *tab,
                                           int32_t *err_out) {
     const int P = n_tok * n_used;
+    if (P <= 32) {
+        // one warp, one load: each lane is a pair; ranks by shuffles
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            const bool live = lane < P;
+            const int e = live ? ids[lane] : -1;
+            const bool valid = live && e >= 0 && e < n_mat;
+            int err = (live && !valid) ? ERR_ID_RANGE : 0;
+            const int tok0 = live ? (lane / n_used) * n_used : 0;
+            int rank = 0, cnt_e = 0, dpos = 0;
+            bool first = true;
+            for (int s2 = 0; s2 < 32; ++s2) {
+                const int e2 = __shfl_sync(0xffffffffu, e, s2);
+                const bool v2 = __shfl_sync(0xffffffffu, valid ? 1 : 0, s2) != 0;
+                if (!valid || !v2) continue;
+                if (e2 < e || (e2 == e && s2 < lane)) ++rank;
+                if (e2 == e) {
+                    ++cnt_e;
+                    if (s2 < lane) {
+                        first = false;
+                        if (s2 >= tok0) err |= ERR_ID_REPEAT;
+                    }
+                }
+            }
+            const unsigned firsts = __ballot_sync(0xffffffffu, valid && first);
+            for (int s2 = 0; s2 < 32; ++s2) {
+                const int e2 = __shfl_sync(0xffffffffu, e, s2);
+                if (((firsts >> s2) & 1u) && e2 < e) ++dpos;
+            }
+            if (valid) tab[L.pairs + rank] = lane;
+            if (valid && first) {
+                tab[L.list_small + dpos] = e;
+                tab[L.count + e] = cnt_e;
+                tab[L.offset + e] = rank;
+            }
+            const unsigned vb = __ballot_sync(0xffffffffu, valid);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) err |= __shfl_xor_sync(0xffffffffu, err, o);
+            if (lane == 0) {
+                tab[WS_ERR] = err;
+                tab[WS_N_SMALL] = __popc(firsts);
+                tab[WS_N_BIG] = 0;
+                tab[WS_N_PAIRS] = P;
+                tab[L.offset + n_mat] = __popc(vb);
+                if (err_out && blockIdx.x == 0) *err_out = err;
+            }
+        }
+        __syncthreads();
+        return;
+    }
     int *cnt = tab + L.count;
     int *cursor = tab + L.list_big;
     int *sid = tab + L.pairs;  // the ids, read once; the pair list overwrites them below
@@ -361,6 +491,31 @@ __device__ __forceinline__ void stage_f32(const XStage &xs, const float *__restr
     const int nb = k / QK;
     const int lane = threadIdx.x & 31;
     const int total = n * nb;
+    if (total <= kCT && ((uintptr_t)af & 15u) == 0) {
+        // one block per thread: every load of the stage in flight at once
+        if ((int)threadIdx.x < total) {
+            const int j = threadIdx.x / nb;
+            const int b = threadIdx.x - j * nb;
+            const float4 *src =
+                reinterpret_cast<const float4 *>(af + (int64_t)arow(j) * k + b * QK);
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 f = src[i];
+                v[4 * i] = f.x;
+                v[4 * i + 1] = f.y;
+                v[4 * i + 2] = f.z;
+                v[4 * i + 3] = f.w;
+            }
+            uint32_t q[8];
+            const float d32 = quantize_block_thread(v, q);
+            uint4 *dst = reinterpret_cast<uint4 *>(xs.q + (size_t)j * k + b * QK);
+            dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
+            dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+            xs.dx[(size_t)j * nb + b] = scale_value(scale_bits(d32));
+        }
+        return;
+    }
     for (int b0 = threadIdx.x >> 5; b0 < total; b0 += kCW * kBatch) {
         float v[kBatch];
 #pragma unroll
@@ -389,6 +544,51 @@ __device__ __forceinline__ void stage_f32(const XStage &xs, const float *__restr
     }
 }
 
+// Quantize the n fp32 rows of the raw slot (row j at raw + j * k) into the
+// stage: stage_f32's rule, from shared memory, one consumer thread per block
+// (no cross-lane steps, so a thread's blocks are independent chains).
+__device__ __forceinline__ void stage_f32_raw(const XStage &xs, const float *raw, int k, int n) {
+    const int nb = k / QK;
+    for (int blk = threadIdx.x; blk < n * nb; blk += kCT) {
+        const int j = blk / nb;
+        const int b = blk - j * nb;
+        const float4 *src = reinterpret_cast<const float4 *>(raw + (size_t)j * k + b * QK);
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 f = src[i];
+            v[4 * i] = f.x;
+            v[4 * i + 1] = f.y;
+            v[4 * i + 2] = f.z;
+            v[4 * i + 3] = f.w;
+        }
+        uint32_t q[8];
+        const float d32 = quantize_block_thread(v, q);
+        uint4 *dst = reinterpret_cast<uint4 *>(xs.q + (size_t)j * k + b * QK);
+        dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
+        dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+        xs.dx[(size_t)j * nb + b] = scale_value(scale_bits(d32));
+    }
+}
+
+// Consumer side of an activation job of nx rows (fp32 af, rows arow(j)):
+// from the raw slot when the producer copied them, else from global memory.
+// The caller synchronizes the consumer warps afterwards.
+template <class RowFn>
+__device__ __forceinline__ void stage_job_f32(const Ring &R, XJobs &J, const XStage &xs,
+                                              const float *af, int k, int nx, RowFn arow,
+                                              int *err) {
+    if (nx <= R.raw_rows) {
+        mbar_wait(R.xfull, J.n & 1, err);
+        stage_f32_raw(xs, R.raw, k, nx);
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(R.xempty);
+        ++J.n;
+    } else {
+        stage_f32(xs, af, k, nx, arow);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // the dot engine
 // ---------------------------------------------------------------------------
@@ -400,14 +600,16 @@ __device__ __forceinline__ float small_int_to_float(int v) {
     return __int_as_float(v + 0x4B400000) - 12582912.0f;
 }
 
-// acc[r][t] = this lane's part of the sum over the warp's blocks of row
-// (row0 + r) of the stage with activation row (xrow0 + t), t < n.
+// acc[r][t] = this lane's part of the sum over the warp's blocks of stage row
+// srow(r) with activation row (xrow0 + t), t < n; srow(r) = row0 + r for
+// r < split, row1 + (r - split) after.
 // Lane l takes block base + l (both 16-byte halves), so each block dot is
 // 8 dp4a in one lane; |isum| <= 32 * 128 * 128 < 2^22.
 template <int NT, int RPW>
 __device__ __forceinline__ void dot_rows(const int8_t *sq, const uint16_t *sd, int k, int ld_d,
-                                         int row0, int seg, int wpr, const XStage &xs, int xrow0,
-                                         int n, float (&acc)[RPW][NT]) {
+                                         int row0, int row1, int split, int seg, int wpr,
+                                         const XStage &xs, int xrow0, int n,
+                                         float (&acc)[RPW][NT]) {
     const int lane = threadIdx.x & 31;
     const int nb = k / QK;
     // Lanes 4-7 of every quarter warp load the upper 16 bytes of their block
@@ -427,10 +629,11 @@ __device__ __forceinline__ void dot_rows(const int8_t *sq, const uint16_t *sd, i
             float dw[RPW];
 #pragma unroll
             for (int r = 0; r < RPW; ++r) {
-                const int8_t *p = sq + (size_t)(row0 + r) * k + kb * QK;
+                const int srow = r < split ? row0 + r : row1 + (r - split);
+                const int8_t *p = sq + (size_t)srow * k + kb * QK;
                 w0[r] = *reinterpret_cast<const uint4 *>(p + h0);
                 w1[r] = *reinterpret_cast<const uint4 *>(p + h1);
-                dw[r] = scale_value(sd[(size_t)(row0 + r) * ld_d + kb]);
+                dw[r] = scale_value(sd[(size_t)srow * ld_d + kb]);
             }
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
@@ -496,12 +699,29 @@ __device__ __forceinline__ int reduce_scatter_index(int lane) {
     return idx;
 }
 
+// The lowest lane that holds value idx after warp_reduce_scatter<V>: the
+// inverse of reduce_scatter_index (bit j of idx, from the top, is lane bit
+// 4 - j).
+template <int V>
+__device__ __forceinline__ int reduce_scatter_lane(int idx) {
+    int lane = 0, m = V, o = 16;
+#pragma unroll
+    for (int j = 0; j < 5 && m > 1; ++j) {
+        if (idx & (m / 2)) lane |= o;
+        idx &= m / 2 - 1;
+        m >>= 1;
+        o >>= 1;
+    }
+    return lane;
+}
+
 // Computes this warp's rows of a stage for activation rows [xrow0, xrow0+n)
-// and writes the warp partial sums to part[(row * wpr + seg) * NT + t].
-template <int NT>
-__device__ __forceinline__ void warp_rows_to_part(const int8_t *sq, const uint16_t *sd, int k,
-                                                  int ld_d, const Geo &g, const XStage &xs,
-                                                  int xrow0, int n, float *part) {
+// and hands each warp sum to emit(row, t, v) (row within the tile, t < NT;
+// called by the one lane that holds the sum).
+template <int NT, class EmitFn>
+__device__ __forceinline__ void warp_rows(const int8_t *sq, const uint16_t *sd, int k, int ld_d,
+                                          const Geo &g, const XStage &xs, int xrow0, int n,
+                                          EmitFn emit) {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int seg = warp % g.wpr;
@@ -509,7 +729,7 @@ __device__ __forceinline__ void warp_rows_to_part(const int8_t *sq, const uint16
 #define Q8_ROWS_CASE(RPW_)                                                                    \
     {                                                                                         \
         float acc[RPW_][NT];                                                                  \
-        dot_rows<NT, RPW_>(sq, sd, k, ld_d, row0, seg, g.wpr, xs, xrow0, n, acc);             \
+        dot_rows<NT, RPW_>(sq, sd, k, ld_d, row0, 0, RPW_, seg, g.wpr, xs, xrow0, n, acc);    \
         constexpr int V = RPW_ * NT;                                                          \
         if constexpr (V <= 32) {                                                              \
             constexpr int VP = pow2_ceil(V);                                                  \
@@ -521,14 +741,14 @@ __device__ __forceinline__ void warp_rows_to_part(const int8_t *sq, const uint16
                 const int idx = reduce_scatter_index<VP>(lane);                               \
                 if (idx < V) {                                                                \
                     const int r = idx / NT, t = idx - (idx / NT) * NT;                        \
-                    part[((row0 + r) * g.wpr + seg) * NT + t] = v;                            \
+                    emit(row0 + r, t, v);                                                     \
                 }                                                                             \
             }                                                                                 \
         } else {                                                                              \
             _Pragma("unroll") for (int r = 0; r < RPW_; ++r)                                  \
                 _Pragma("unroll") for (int t = 0; t < NT; ++t) {                              \
                     const float v = warp_sum_all(acc[r][t]);                                  \
-                    if (lane == 0) part[((row0 + r) * g.wpr + seg) * NT + t] = v;             \
+                    if (lane == 0) emit(row0 + r, t, v);                                      \
                 }                                                                             \
         }                                                                                     \
     }
@@ -537,6 +757,54 @@ __device__ __forceinline__ void warp_rows_to_part(const int8_t *sq, const uint16
     else if (g.rpw == 2) Q8_ROWS_CASE(2)
     else Q8_ROWS_CASE(1)
 #undef Q8_ROWS_CASE
+}
+
+// Gate/up tile with whole rows per warp (wpr == 1, rpw even): warp w owns
+// gate stage rows w*rpw/2 + i and the matching up rows half + w*rpw/2 + i
+// (i < rpw/2).  emit(i_row, t, g, u) gets each (gate row within the tile, t)
+// with its two final sums, called by one lane.
+template <int NT, class EmitFn>
+__device__ __forceinline__ void warp_pairs(const int8_t *sq, const uint16_t *sd, int k, int ld_d,
+                                           const Geo &g, int half, const XStage &xs, int xrow0,
+                                           int n, EmitFn emit) {
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+#define Q8_PAIRS_CASE(RPW_)                                                                   \
+    {                                                                                         \
+        constexpr int H = RPW_ / 2;                                                           \
+        const int row0 = warp * H;                                                            \
+        float acc[RPW_][NT];                                                                  \
+        dot_rows<NT, RPW_>(sq, sd, k, ld_d, row0, half + row0, H, 0, 1, xs, xrow0, n, acc);   \
+        constexpr int V = RPW_ * NT;                                                          \
+        constexpr int VP = pow2_ceil(V);                                                      \
+        static_assert(V <= 32, "pair tile too wide");                                         \
+        float a[VP];                                                                          \
+        _Pragma("unroll") for (int i = 0; i < VP; ++i)                                        \
+            a[i] = i < V ? reinterpret_cast<float(&)[V]>(acc)[i] : 0.0f;                      \
+        const float v = warp_reduce_scatter<VP>(a);                                           \
+        const int idx = reduce_scatter_index<VP>(lane);                                       \
+        const int up_idx = idx + H * NT;                                                      \
+        const float u = __shfl_sync(0xffffffffu, v,                                           \
+                                    reduce_scatter_lane<VP>(up_idx < VP ? up_idx : 0));       \
+        if ((lane & (32 / VP - 1)) == 0 && idx < H * NT) {                                    \
+            const int i = idx / NT, t = idx - (idx / NT) * NT;                                \
+            emit(row0 + i, t, v, u);                                                          \
+        }                                                                                     \
+    }
+    if (g.rpw == 4) Q8_PAIRS_CASE(4)
+    else Q8_PAIRS_CASE(2)
+#undef Q8_PAIRS_CASE
+}
+
+// The warp partial sums of a K-split tile go to part[(row * wpr + seg) * NT + t].
+template <int NT>
+__device__ __forceinline__ void warp_rows_to_part(const int8_t *sq, const uint16_t *sd, int k,
+                                                  int ld_d, const Geo &g, const XStage &xs,
+                                                  int xrow0, int n, float *part) {
+    const int seg = (threadIdx.x >> 5) % g.wpr;
+    warp_rows<NT>(sq, sd, k, ld_d, g, xs, xrow0, n, [&](int row, int t, float v) {
+        part[(row * g.wpr + seg) * NT + t] = v;
+    });
 }
 
 // Calls f(std::integral_constant<int, NTC>) with the smallest NTC in
