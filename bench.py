@@ -392,10 +392,20 @@ class MoeWorkload:
                 tot += ne * self.expert_bytes
                 ug += ne * q8_bytes(2 * F, D)
             self.step_bytes.append(tot)
-            self.up_gate_bytes.append(ug / layers)
+            # bytes of one launch of the dominant kernel (a layer's up/gate, or
+            # the whole layer when it is fused)
+            self.up_gate_bytes.append((tot if self.routed and P <= 32 and D <= 4096 and F <= 2048
+                                       else ug) / layers)
         self.tokens_per_step = tokens
         self.small = P <= 1024 and E <= 512
-        if self.small:
+        # routed batches of at most 32 pairs: q8_moe_ffn runs the whole layer
+        # as one kernel (the dominant kernel is then the layer kernel)
+        self.fused = self.routed and P <= 32 and D <= 4096 and F <= 2048
+        if self.fused:
+            self.kernel = "moe_layer_kernel"
+            self.ffn_ws = q8.moe_ffn_workspace(tokens, U, E, D, F, dev)
+            self.launches_per_step = layers
+        elif self.small:
             self.launches_per_step = layers * (3 if self.routed else 2)
         elif self.routed:
             # quantize x, group, up/gate (dp4a + tensor cores), quantize h,
@@ -419,6 +429,14 @@ class MoeWorkload:
         s = i % self.sets if input_set is None else input_set
         layers = self.Lc[i % self.copies]
         T = self.T
+        if self.fused:
+            # the public whole-step call: one fused kernel per layer
+            for l, (UG, DN) in enumerate(layers):
+                marks.begin()
+                q8.moe_ffn(UG, DN, self.x[s][l], self.ids[s][l], self.p[s][l], ws=self.ffn_ws,
+                           out=self.out[l])
+                marks.end()
+            return
         if self.small:
             # small batches: the fp32 calls (x and h quantized inside the
             # kernels, routing grouped in every CTA), the same kernels

@@ -304,7 +304,14 @@ q8_status q8_moe_combine(const float *y, const float *route_w, int64_t n_tok, in
  *  n_used == 1), where out = down . quantize(h).
  *  out: fp32 [n_tok][n_embd].
  *  ws: q8_moe_ffn_workspace_size(...) bytes, 256-byte aligned; it also holds
- *      the intermediates (xq, h, hq, per-slot y).
+ *      the intermediates (xq, h, hq, per-slot y) and the grid-barrier words
+ *      of the fused layer kernel.  Zero-fill it before its first use; the
+ *      calls leave those words at zero (after a wait timeout reported by
+ *      q8_check, zero it again).
+ * Routed batches of at most 32 pairs (n_tok * n_used) with n_embd <= 4096
+ * and n_ff <= 2048 run as ONE cooperative kernel (grouping, up/gate +
+ * SwiGLU, a grid barrier, down + combine); the result is bitwise that of
+ * the separate calls.
  */
 size_t q8_moe_ffn_workspace_size(int64_t n_tok, int32_t n_used, int64_t n_mat, int64_t n_embd,
                                  int64_t n_ff);

@@ -143,6 +143,15 @@ constexpr int64_t kCtaGroupMaxPairs = Q8_SMALL_BATCH_PAIRS;
 constexpr int64_t kCtaGroupMaxMats = Q8_SMALL_BATCH_MATS;
 
 // Wait-timeout flags latched by the streaming kernels of each file.
+// The fused MoE layer kernel (q8_layer.cu) for small routed batches.
+constexpr int64_t kLayerMaxPairs = 32;
+bool layer_eligible(const q8_tensor *up_gate, const q8_tensor *down, int64_t n_tok,
+                    int32_t n_used);
+q8_status launch_layer(const q8_tensor *up_gate, const q8_tensor *down, const float *x,
+                       int64_t n_tok, const int32_t *ids, const float *route_w, int32_t n_used,
+                       float *out, float *h, unsigned *bar, int32_t *err_out, cudaStream_t s);
+q8_status read_wait_errors_layer(int *flags);
+
 q8_status read_wait_errors_matmul(int *flags);
 q8_status read_wait_errors_moe(int *flags);
 q8_status read_wait_errors_tc(int *flags);

@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                         }, &g_err_matmul);
                     }
                 };
-                produce(R, tb, te, src, &g_err_matmul, jobs);
+                produce(R, tb, te, src, &g_err_matmul, jobs, !routed);
             } else {
                 produce(R, tb, te, src, &g_err_matmul);
             }
@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                                     &g_err_matmul);
                     }
                 };
-                produce(R, tb, te, src, &g_err_matmul, jobs);
+                produce(R, tb, te, src, &g_err_matmul, jobs, true);
             } else {
                 produce(R, tb, te, src, &g_err_matmul);
             }

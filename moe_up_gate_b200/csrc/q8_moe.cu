@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                         }, &g_err_moe);
                     }
                 };
-                produce(R, tb, te, src, &g_err_moe, jobs);
+                produce(R, tb, te, src, &g_err_moe, jobs, !routed);
             } else {
                 produce(R, tb, te, src, &g_err_moe);
             }
@@ -382,7 +382,7 @@ static q8_status launch_combine(const float *y, const float *w, int64_t n_tok, i
 
 // moe_ffn workspace regions
 struct FfnLayout {
-    size_t group, xq, xd, h, y, total;
+    size_t group, bar, xq, xd, h, y, total;
 };
 
 static FfnLayout ffn_layout(int64_t n_tok, int32_t n_used, int64_t n_mat, int64_t n_embd,
@@ -392,6 +392,8 @@ static FfnLayout ffn_layout(int64_t n_tok, int32_t n_used, int64_t n_mat, int64_
     size_t o = 0;
     L.group = o;
     o += routed ? group_bytes(P, n_mat) : 0;
+    L.bar = o;  // grid barrier words of the fused layer kernel
+    o += 256;
     L.xq = o;
     o += round_up((size_t)n_tok * n_embd, 256);
     L.xd = o;
@@ -708,6 +710,9 @@ q8_status q8_moe_ffn(const q8_tensor *up_gate, const q8_tensor *down, const floa
         // grouping built in each CTA from ids), down (h quantized as it is
         // staged), combine.
         int32_t *err = routed ? (int32_t *)(w8 + F.group) : nullptr;
+        if (routed && layer_eligible(up_gate, down, n_tok, n_used))
+            return launch_layer(up_gate, down, x, n_tok, ids, route_w, n_used, out, h,
+                                (unsigned *)(w8 + F.bar), err, s);
         st = q8_moe_up_gate_swiglu_fp32(up_gate, x, n_tok, ids, n_used, h, err, s);
         if (st != Q8_OK) return st;
         if (!routed) return launch_matmul_dense(down, nullptr, nullptr, h, n_tok, out, s);
@@ -747,11 +752,11 @@ q8_status q8_check(const void *ws, void *stream) {
     if (ws) e = cudaMemcpyAsync(&flags, ws, sizeof flags, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) Q8_FAIL(Q8_E_CUDA, "q8_check: %s", cudaGetErrorString(e));
-    int w1 = 0, w2 = 0, w3 = 0;
+    int w1 = 0, w2 = 0, w3 = 0, w4 = 0;
     if (read_wait_errors_matmul(&w1) != Q8_OK || read_wait_errors_moe(&w2) != Q8_OK ||
-        read_wait_errors_tc(&w3) != Q8_OK)
+        read_wait_errors_tc(&w3) != Q8_OK || read_wait_errors_layer(&w4) != Q8_OK)
         Q8_FAIL(Q8_E_CUDA, "q8_check: reading the kernels' wait flags failed");
-    if (w1 | w2 | w3)
+    if (w1 | w2 | w3 | w4)
         Q8_FAIL(Q8_E_CUDA, "q8_check: a kernel gave up waiting for a shared-memory stage");
     if (flags & ERR_ID_RANGE) Q8_FAIL(Q8_E_BAD_ID, "q8_check: a routing id is out of range");
     if (flags & ERR_ID_REPEAT)

@@ -287,15 +287,28 @@ struct NoJobs {
 // tile's spans; jobs(t, when) issues the activation jobs of tile t: when == 0
 // before its weights (the job of its first group), when == 1 after them (the
 // jobs of its other groups).  Ends after the last copies have landed.
+// gated: the activations may be written by the preceding grid and this
+// thread has not waited for it yet.  The weights do not depend on that grid,
+// so the first ring's worth of tiles is issued at once; the producer then
+// waits for the grid and issues the jobs of those tiles (their consumers wait
+// for them), and goes on in stream order.
 template <class SrcFn, class JobFn = NoJobs>
 __device__ __forceinline__ void produce(const Ring &R, int64_t tb, int64_t te, SrcFn src,
-                                        int *err, JobFn jobs = JobFn{}) {
+                                        int *err, JobFn jobs = JobFn{}, bool gated = false) {
     int it = 0;
     Q8_TRACE(20);
+    const int64_t pre = gated ? min(te, tb + (int64_t)R.stages) : tb;
     for (int64_t t = tb; t < te; ++t, ++it) {
         const int s = it % R.stages;
         const int round = it / R.stages;
-        jobs(t, 0);
+        if (t == pre && gated) {
+            griddep_wait();
+            for (int64_t j = tb; j < pre; ++j) {
+                jobs(j, 0);
+                jobs(j, 1);
+            }
+        }
+        if (t >= pre) jobs(t, 0);
         if (round > 0) mbar_wait(&R.empty[s], (round - 1) & 1, err);
         Q8_TRACE(21);
         const TileSrc ts = src(t);
@@ -310,7 +323,14 @@ __device__ __forceinline__ void produce(const Ring &R, int64_t tb, int64_t te, S
             bulk_g2s(R.qs(s) + (size_t)ts.row_off1 * k, ts.q1, qb1, &R.full[s]);
             bulk_g2s(R.d(s) + (size_t)ts.row_off1 * ld_d, ts.d1, db1, &R.full[s]);
         }
-        jobs(t, 1);
+        if (t >= pre) jobs(t, 1);
+    }
+    if (gated && pre == te) {  // every tile went out before the wait
+        griddep_wait();
+        for (int64_t j = tb; j < te; ++j) {
+            jobs(j, 0);
+            jobs(j, 1);
+        }
     }
     Q8_TRACE(22);
     const int first = it > R.stages ? it - R.stages : 0;

@@ -243,25 +243,43 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             float acc[16];
 #pragma unroll
             for (int t = 0; t < 16; ++t) acc[t] = 0.0f;
-            for (int b = 0; b < nb; ++b, ++bg) {
-                const int slot = bg % kTcSlots;
-                mbar_wait(&sfull[slot], (bg / kTcSlots) & 1, &g_err_tc);
+            // blocks in groups of up to 4 (one K chunk): the MMA thread's
+            // commit on the group's last slot covers the group's earlier
+            // MMAs too, so one wait and one tensor-memory load round trip
+            // serve four blocks
+            for (int b = 0; b < nb; b += 4) {
+                const int gn = min(4, nb - b);
+                const int slot_last = (bg + gn - 1) % kTcSlots;
+                mbar_wait(&sfull[slot_last], ((bg + gn - 1) / kTcSlots) & 1, &g_err_tc);
                 tc_fence_after();
-                uint32_t v[16];
+                uint32_t v[4][16];
                 if (active) {
-                    tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * kTcN + half * 16), v);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (i < gn)
+                            tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) +
+                                          (uint32_t)(((bg + i) % kTcSlots) * kTcN + half * 16),
+                                      v[i]);
                     tmem_ld_wait();
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sempty[slot]);
+                if (lane == 0)
+                    for (int i = 0; i < gn; ++i) mbar_arrive(&sempty[(bg + i) % kTcSlots]);
                 if (active) {
-                    const float dw = row_ok ? scale_value(drow[b]) : 0.0f;
-                    const float *dxb = dxs + (half * 16) * nb + b;
 #pragma unroll
-                    for (int t = 0; t < 16; ++t)
-                        acc[t] = fmaf(dw * dxb[t * nb], small_int_to_float((int)v[t]), acc[t]);
+                    for (int i = 0; i < 4; ++i) {
+                        if (i < gn) {
+                            const float dw = row_ok ? scale_value(drow[b + i]) : 0.0f;
+                            const float *dxb = dxs + (half * 16) * nb + b + i;
+#pragma unroll
+                            for (int t = 0; t < 16; ++t)
+                                acc[t] = fmaf(dw * dxb[t * nb], small_int_to_float((int)v[i][t]),
+                                              acc[t]);
+                        }
+                    }
                 }
+                bg += gn;
             }
             // ---- outputs
             if (upgate) {

@@ -327,7 +327,7 @@ def moe_combine(y, route_w, out=None, stream=None):
 
 def moe_ffn_workspace(n_tok, n_used, n_mat, n_embd, n_ff, device="cuda") -> torch.Tensor:
     nbytes = int(load().q8_moe_ffn_workspace_size(n_tok, n_used, n_mat, n_embd, n_ff))
-    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)  # zero before first use
 
 
 def moe_ffn(up_gate: Q8Tensor, down: Q8Tensor, x, ids=None, route_w=None, ws=None, out=None,
