@@ -17,7 +17,7 @@
 //           expert (k <= 4096: whole rows per warp); x rows are copied by the
 //           producer and quantized in shared memory; h goes to global memory.
 //  barrier  all CTAs' h is written (bounded wait).
-//  phase B  units of kLayerNrb down rows; a stage holds those rows of up to 8
+//  phase B  units of kLayerNrb (8) down rows; a stage holds those rows of up to 8
 //           experts (one per warp).  Every CTA stages all pairs' h as Q8_0,
 //           computes y for its rows, then forms out[t] = sum_s p[t][s] y[t][s]
 //           in s order for the unit's rows (the combine_kernel fma chain).
@@ -37,7 +37,7 @@ q8_status read_wait_errors_layer(int *flags) {
     return e == cudaSuccess ? Q8_OK : Q8_E_CUDA;
 }
 
-constexpr int kLayerNrb = 4;  // down rows per unit (rows per warp in phase B)
+constexpr int kLayerNrb = 8;  // down rows per unit (rows per warp in phase B)
 constexpr int kLayerNT = 4;   // activation rows per pass (template bound)
 
 struct LayerParams {
@@ -181,6 +181,7 @@ __global__ void __launch_bounds__(kThreadsStream, 1) moe_layer_kernel(const __gr
                 const int ti = (int)(t % tpm);
                 const int64_t grow = (int64_t)e * p.ug_stride + (int64_t)ti * half;
                 const int64_t urow = grow + p.n_ff;
+                Q8_TRACE(21);
                 const uint32_t qb = (uint32_t)(half * p.k), db = (uint32_t)(half * p.ug_ld_d * 2);
                 mbar_arrive_expect_tx(&R.full[s], 2 * (qb + db));
                 bulk_g2s(R.qs(s), p.ug_q + grow * p.k, qb, &R.full[s]);
@@ -265,6 +266,7 @@ __global__ void __launch_bounds__(kThreadsStream, 1) moe_layer_kernel(const __gr
 
     // ---------------- every CTA's h is written
     named_bar_sync(kBarConsumers, kCT);
+    Q8_TRACE(12);
     if (threadIdx.x == 0) grid_barrier(p.bar, gridDim.x, &g_err_layer);
     named_bar_sync(kBarConsumers, kCT);
     Q8_TRACE(11);
@@ -297,9 +299,10 @@ __global__ void __launch_bounds__(kThreadsStream, 1) moe_layer_kernel(const __gr
                 const int e = expert(mi);
                 const int cnt = tab[p.lay_count + e];
                 const int off = tab[p.lay_offset + e];
-                for (int tg = 0; tg < cnt; tg += NT) {
-                    const int n = min(NT, cnt - tg);
-                    with_nt<NT>(n, [&](auto ntc) {
+                // at most 2 activation rows per pass here: 8 rows per warp
+                for (int tg = 0; tg < cnt; tg += 2) {
+                    const int n = min(2, cnt - tg);
+                    with_nt<2>(n, [&](auto ntc) {
                         constexpr int NTC = decltype(ntc)::value;
                         warp_rows<NTC>(R.qs(s), R.d(s), p.n_ff, (int)p.dn_ld_d, gb, hs, off + tg, n,
                                        [&](int row, int tt, float v) {

@@ -370,22 +370,18 @@ struct GemvProblem {
     int tile_begin;
 };
 
+constexpr int kGemvMaxGrid = 1024;
+
 struct GemvBatchParams {
     int n_desc;
     int n_tok;
     int total_tiles;
+    int grid;
     Plan plan;
     GemvProblem pr[Q8_MAX_GEMV_DESC];
+    uint8_t first_problem[kGemvMaxGrid];  // problem of each CTA's first tile
 };
 
-__device__ __forceinline__ int find_problem(const GemvBatchParams &p, int64_t t) {
-    int lo = 0, hi = p.n_desc - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (p.pr[mid].tile_begin <= t) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-}
 
 template <int NT>
 __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
@@ -399,7 +395,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     my_tiles(p.total_tiles, &tb, &te);
     if ((threadIdx.x >> 5) == kCW) {
         if ((threadIdx.x & 31) == 0 && tb < te) {
-            int cur = find_problem(p, tb);
+            int cur = p.first_problem[blockIdx.x];
             auto src = [&](int64_t t) {
                 while (cur + 1 < p.n_desc && p.pr[cur + 1].tile_begin <= t) ++cur;
                 const GemvProblem &q = p.pr[cur];
@@ -442,7 +438,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     float *part0 = reinterpret_cast<float *>(smem + p.plan.off_part);
     const int xmax = p.plan.xmax;
     int buf = 0, staged = -1, staged_grp = -1, it = 0;
-    int cur = tb < te ? find_problem(p, tb) : 0;
+    int cur = p.first_problem[blockIdx.x];
     XJobs J;
     bool unsynced = false;  // passes without a barrier since the last one
     for (int64_t t = tb; t < te; ++t, ++it) {
@@ -648,7 +644,17 @@ q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_t
     if (!make_plan(max_tq, max_td, max_k, (int)std::min<int64_t>(n_tok, kMaxXRows), nt, &p.plan,
                    0, true))
         Q8_FAIL(Q8_E_UNSUPPORTED, "q8_gemv_batched: k=%d does not fit the plan", max_k);
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * p.plan.ctas, tiles));
+    const int grid = (int)std::max<int64_t>(
+        1, std::min<int64_t>(std::min<int64_t>((int64_t)num_sms() * p.plan.ctas, tiles),
+                             kGemvMaxGrid));
+    p.grid = grid;
+    // the problem of each CTA's first tile (the kernel's my_tiles split),
+    // so that no thread searches the problem list at start
+    for (int b = 0, cur = 0; b < grid; ++b) {
+        const int64_t tb = tiles * b / grid;
+        while (cur + 1 < n_desc && p.pr[cur + 1].tile_begin <= tb) ++cur;
+        p.first_problem[b] = (uint8_t)cur;
+    }
     cudaStream_t s = (cudaStream_t)stream;
     switch (nt) {
         case 1: return launch_stream(gemv_batched_kernel<1>, grid, p.plan.bytes, s, p, "gemv_batched");

@@ -362,6 +362,7 @@ __device__ __forceinline__ void cta_group(const int32_t *__restrict__ ids, int n
             const int tok0 = live ? (lane / n_used) * n_used : 0;
             int rank = 0, cnt_e = 0, dpos = 0;
             bool first = true;
+#pragma unroll
             for (int s2 = 0; s2 < 32; ++s2) {
                 const int e2 = __shfl_sync(0xffffffffu, e, s2);
                 const bool v2 = __shfl_sync(0xffffffffu, valid ? 1 : 0, s2) != 0;
@@ -376,6 +377,7 @@ __device__ __forceinline__ void cta_group(const int32_t *__restrict__ ids, int n
                 }
             }
             const unsigned firsts = __ballot_sync(0xffffffffu, valid && first);
+#pragma unroll
             for (int s2 = 0; s2 < 32; ++s2) {
                 const int e2 = __shfl_sync(0xffffffffu, e, s2);
                 if (((firsts >> s2) & 1u) && e2 < e) ++dpos;
@@ -642,6 +644,8 @@ __device__ __forceinline__ void dot_rows(const int8_t *sq, const uint16_t *sd, i
     for (int r = 0; r < RPW; ++r)
 #pragma unroll
         for (int t = 0; t < NT; ++t) acc[r][t] = 0.0f;
+    // two K steps in flight when a warp takes few rows (long rows)
+#pragma unroll(RPW <= 2 ? 2 : 1)
     for (int base = seg * 32; base < nb; base += 32 * wpr) {
         const int kb = base + lane;
         if (kb < nb) {
@@ -772,7 +776,8 @@ __device__ __forceinline__ void warp_rows(const int8_t *sq, const uint16_t *sd, 
                 }                                                                             \
         }                                                                                     \
     }
-    if (g.rpw == 5) Q8_ROWS_CASE(5)
+    if (g.rpw == 8) Q8_ROWS_CASE(8)
+    else if (g.rpw == 5) Q8_ROWS_CASE(5)
     else if (g.rpw == 4) Q8_ROWS_CASE(4)
     else if (g.rpw == 2) Q8_ROWS_CASE(2)
     else Q8_ROWS_CASE(1)
