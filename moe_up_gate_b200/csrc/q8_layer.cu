@@ -13,11 +13,13 @@
 //
 // Grid: one CTA per SM, all co-resident (cooperative launch), each with the
 // streaming engine of q8_stream.cuh (one producer warp, 8 consumer warps).
+// The raw x slot and the phase-B areas share one region: x is staged before
+// phase B starts.
 //  phase A  tiles of 8 gate rows + the 8 matching up rows of one routed
 //           expert (k <= 4096: whole rows per warp); x rows are copied by the
 //           producer and quantized in shared memory; h goes to global memory.
 //  barrier  all CTAs' h is written (bounded wait).
-//  phase B  units of kLayerNrb (8) down rows; a stage holds those rows of up to 8
+//  phase B  units of nrb (8) down rows; a stage holds those rows of up to 8
 //           experts (one per warp).  Every CTA stages all pairs' h as Q8_0,
 //           computes y for its rows, then forms out[t] = sum_s p[t][s] y[t][s]
 //           in s order for the unit's rows (the combine_kernel fma chain).
@@ -37,8 +39,7 @@ q8_status read_wait_errors_layer(int *flags) {
     return e == cudaSuccess ? Q8_OK : Q8_E_CUDA;
 }
 
-constexpr int kLayerNrb = 8;  // down rows per unit (rows per warp in phase B)
-constexpr int kLayerNT = 4;   // activation rows per pass (template bound)
+constexpr int kLayerNT = 4;   // activation rows per pass (template bound), several tokens
 
 struct LayerParams {
     const int8_t *ug_q;
@@ -59,6 +60,7 @@ struct LayerParams {
     int n_tok, n_used, n_mat;
     int64_t lay_count, lay_offset, lay_list, lay_big, lay_pairs;
     int off_hq, off_hd, off_y, off_inv;  // phase-B areas
+    int nrb;                             // down rows per unit
     Plan plan;
 };
 
@@ -125,14 +127,23 @@ __device__ __forceinline__ void stage_f32_l2(const XStage &xs, const float *src,
     }
 }
 
-template <int NT>
-__global__ void __launch_bounds__(kThreadsStream, 1) moe_layer_kernel(const __grid_constant__ LayerParams p) {
+template <int NT, int MINB>
+__global__ void __launch_bounds__(kThreadsStream, MINB)
+    moe_layer_kernel(const __grid_constant__ LayerParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
     Q8_TRACE(0);
     const Ring R = ring_init(smem, p.plan);
     Q8_TRACE(1);
     griddep_wait();  // x, ids and route_w may come from the preceding kernel
     griddep_launch_dependents();
+    // One token (the NT == 1 variant): every routed expert reads the same x
+    // row, so the producer fetches it before the grouping and it is staged
+    // once for the whole of phase A.
+    const bool x_once = NT == 1 && R.raw_rows > 0;
+    if (x_once && threadIdx.x == kCT) {
+        mbar_arrive_expect_tx(R.xfull, (uint32_t)p.k * 4);
+        bulk_g2s_keep(R.raw, p.x, (uint32_t)p.k * 4, R.xfull);
+    }
     int32_t *tab = reinterpret_cast<int32_t *>(smem + p.plan.off_tab);
     {
         GroupLayout L{};
@@ -149,7 +160,8 @@ __global__ void __launch_bounds__(kThreadsStream, 1) moe_layer_kernel(const __gr
     const Geo ga = geo_pair_for_k(p.k);
     const int half = ga.nr / 2;
     const int tpm = p.n_ff / half;
-    const int units = (p.k + kLayerNrb - 1) / kLayerNrb;
+    const int nrb = p.nrb;
+    const int units = (p.k + nrb - 1) / nrb;
     const int sg_per_unit = (n_exp + kCW - 1) / kCW;
     const int xmax = p.plan.xmax;
     int64_t ta0, ta1, ub0, ub1;
@@ -175,7 +187,7 @@ __global__ void __launch_bounds__(kThreadsStream, 1) moe_layer_kernel(const __gr
             };
             for (int64_t t = ta0; t < ta1; ++t, ++it) {  // phase A: gate/up tiles
                 const int s = it % R.stages;
-                if (R.raw_rows > 0) jobs(t, 0);
+                if (R.raw_rows > 0 && !x_once) jobs(t, 0);
                 if (it >= R.stages) mbar_wait(&R.empty[s], (it / R.stages - 1) & 1, &g_err_layer);
                 const int e = expert((int)(t / tpm));
                 const int ti = (int)(t % tpm);
@@ -189,11 +201,11 @@ __global__ void __launch_bounds__(kThreadsStream, 1) moe_layer_kernel(const __gr
                 bulk_g2s(R.qs(s) + (size_t)half * p.k, p.ug_q + urow * p.k, qb, &R.full[s]);
                 bulk_g2s(R.d(s) + (size_t)half * p.ug_ld_d, p.ug_d + urow * p.ug_ld_d, db,
                          &R.full[s]);
-                if (R.raw_rows > 0) jobs(t, 1);
+                if (R.raw_rows > 0 && !x_once) jobs(t, 1);
             }
             for (int64_t u = ub0; u < ub1; ++u) {  // phase B: down rows of every expert
-                const int r0 = (int)u * kLayerNrb;
-                const int nrv = min(kLayerNrb, p.k - r0);
+                const int r0 = (int)u * nrb;
+                const int nrv = min(nrb, p.k - r0);
                 for (int sg = 0; sg < sg_per_unit; ++sg, ++it) {
                     const int s = it % R.stages;
                     if (it >= R.stages)
@@ -203,9 +215,9 @@ __global__ void __launch_bounds__(kThreadsStream, 1) moe_layer_kernel(const __gr
                     mbar_arrive_expect_tx(&R.full[s], (uint32_t)ne * (qb + db));
                     for (int j = 0; j < ne; ++j) {
                         const int64_t row = (int64_t)expert(sg * kCW + j) * p.dn_stride + r0;
-                        bulk_g2s(R.qs(s) + (size_t)j * kLayerNrb * p.n_ff, p.dn_q + row * p.n_ff,
+                        bulk_g2s(R.qs(s) + (size_t)j * nrb * p.n_ff, p.dn_q + row * p.n_ff,
                                  qb, &R.full[s]);
-                        bulk_g2s(R.d(s) + (size_t)j * kLayerNrb * p.dn_ld_d,
+                        bulk_g2s(R.d(s) + (size_t)j * nrb * p.dn_ld_d,
                                  p.dn_d + row * p.dn_ld_d, db, &R.full[s]);
                     }
                 }
@@ -222,6 +234,12 @@ __global__ void __launch_bounds__(kThreadsStream, 1) moe_layer_kernel(const __gr
                     reinterpret_cast<float *>(smem + p.plan.off_xd)};
     int it = 0, staged_mi = -1, staged_grp = -1;
     XJobs J;
+    if (x_once) {
+        mbar_wait(R.xfull, 0, &g_err_layer);
+        stage_f32_raw(xs, R.raw, p.k, 1);
+        named_bar_sync(kBarConsumers, kCT);
+        Q8_TRACE(7);
+    }
     for (int64_t t = ta0; t < ta1; ++t, ++it) {
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_layer);
@@ -235,7 +253,7 @@ __global__ void __launch_bounds__(kThreadsStream, 1) moe_layer_kernel(const __gr
         for (int grp = 0; grp < n_grp; ++grp) {
             const int x0 = grp * xmax;
             const int nx = min(xmax, cnt - x0);
-            if (mi != staged_mi || grp != staged_grp) {
+            if (!x_once && (mi != staged_mi || grp != staged_grp)) {
                 if (staged_mi >= 0) named_bar_sync(kBarConsumers, kCT);
                 stage_job_f32(R, J, xs, p.x, p.k, nx,
                               [&](int j) { return plist[x0 + j] / p.n_used; }, &g_err_layer);
@@ -286,10 +304,10 @@ __global__ void __launch_bounds__(kThreadsStream, 1) moe_layer_kernel(const __gr
     Q8_TRACE(7);
 
     // ---------------- phase B: y = down . hq, out = sum_s p y
-    const Geo gb{kLayerNrb * kCW, 1, kLayerNrb};
+    const Geo gb{nrb * kCW, 1, nrb};
     for (int64_t u = ub0; u < ub1; ++u) {
-        const int r0 = (int)u * kLayerNrb;
-        const int nrv = min(kLayerNrb, p.k - r0);
+        const int r0 = (int)u * nrb;
+        const int nrv = min(nrb, p.k - r0);
         for (int sg = 0; sg < sg_per_unit; ++sg, ++it) {
             const int s = it % R.stages;
             mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_layer);
@@ -299,17 +317,23 @@ __global__ void __launch_bounds__(kThreadsStream, 1) moe_layer_kernel(const __gr
                 const int e = expert(mi);
                 const int cnt = tab[p.lay_count + e];
                 const int off = tab[p.lay_offset + e];
-                // at most 2 activation rows per pass here: 8 rows per warp
-                for (int tg = 0; tg < cnt; tg += 2) {
-                    const int n = min(2, cnt - tg);
-                    with_nt<2>(n, [&](auto ntc) {
+                // at most 2 activation rows per pass here (up to 8 rows per
+                // warp); one at one token (an expert then has one pair)
+                constexpr int NB = NT == 1 ? 1 : 2;
+                for (int tg = 0; tg < cnt; tg += NB) {
+                    const int n = min(NB, cnt - tg);
+                    with_nt<NB>(n, [&](auto ntc) {
                         constexpr int NTC = decltype(ntc)::value;
-                        warp_rows<NTC>(R.qs(s), R.d(s), p.n_ff, (int)p.dn_ld_d, gb, hs, off + tg, n,
-                                       [&](int row, int tt, float v) {
-                                           const int rr = row - warp * kLayerNrb;
-                                           if (tt < n && rr < nrv)
-                                               ybuf[(off + tg + tt) * kLayerNrb + rr] = v;
-                                       });
+                        auto emit = [&](int row, int tt, float v) {
+                            const int rr = row - warp * nrb;
+                            if (tt < n && rr < nrv) ybuf[(off + tg + tt) * nrb + rr] = v;
+                        };
+                        if (nrb == 8)
+                            warp_rows<NTC, 8>(R.qs(s), R.d(s), p.n_ff, (int)p.dn_ld_d, gb, hs,
+                                              off + tg, n, emit);
+                        else
+                            warp_rows<NTC, 4>(R.qs(s), R.d(s), p.n_ff, (int)p.dn_ld_d, gb, hs,
+                                              off + tg, n, emit);
                     });
                 }
             }
@@ -324,8 +348,7 @@ __global__ void __launch_bounds__(kThreadsStream, 1) moe_layer_kernel(const __gr
             float acc = 0.0f;
             for (int s2 = 0; s2 < p.n_used; ++s2) {
                 const int q = inv[t * p.n_used + s2];
-                acc = fmaf(p.route_w[t * p.n_used + s2], q >= 0 ? ybuf[q * kLayerNrb + rr] : 0.0f,
-                           acc);
+                acc = fmaf(p.route_w[t * p.n_used + s2], q >= 0 ? ybuf[q * nrb + rr] : 0.0f, acc);
             }
             p.out[(int64_t)t * p.k + r0 + rr] = acc;
         }
@@ -341,6 +364,67 @@ bool layer_eligible(const q8_tensor *up_gate, const q8_tensor *down, int64_t n_t
     const int64_t n_ff = up_gate->rows / 2;
     return n_tok * n_used <= kLayerMaxPairs && up_gate->n_mat <= kCtaGroupMaxMats &&
            up_gate->k <= 4096 && n_ff <= 2048 && n_ff % 16 == 0 && down->k == n_ff;
+}
+
+// Shared-memory plan of the layer kernel: barriers, the ring (stages sized
+// for the larger of a gate/up tile and a phase-B stage), the x stage, the
+// grouping tables, then one region that holds the raw x slot during phase A
+// and the phase-B areas (all pairs' hq and scales, y, the pair inverse)
+// afterwards.
+static bool layer_plan(LayerParams &p, int64_t P, int n_ff, int tq, int td, int xrows, int ctas,
+                       int nrb, bool raw, int group_words) {
+    const int budget = smem_budget(ctas);
+    const int nb_ff = n_ff / QK;
+    const int xmax = xrows;
+    const int x_bytes = xmax * p.k + ((xmax * (p.k / QK) * 4 + 15) / 16) * 16;
+    const int tab_bytes = ((group_words * 4 + 15) / 16) * 16;
+    const int raw_rows = raw ? std::min(xmax, kRawSlotBytes / (4 * p.k)) : 0;
+    const int raw_bytes = raw_rows * 4 * p.k;
+    int o = 0;
+    const int hq = o;
+    o += (int)(P * n_ff);
+    o = (o + 15) / 16 * 16;
+    const int hd = o;
+    o += (int)(P * nb_ff * 4);
+    const int y = o;
+    o += (int)(P * nrb * 4);
+    const int inv = o;
+    o += (int)(P * 4);
+    const int union_bytes = (std::max(o, raw_bytes) + 127) / 128 * 128;
+    const int stage_qs = round128(tq);
+    const int stage_bytes = stage_qs + round128(td);
+    const int fixed = 256 + x_bytes + tab_bytes + union_bytes;
+    int stages = (budget - fixed) / stage_bytes;
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages < 2) return false;
+    Plan &pl = p.plan;
+    pl = Plan{};
+    pl.stages = stages;
+    pl.stage_qs = stage_qs;
+    pl.stage_bytes = stage_bytes;
+    pl.xmax = xmax;
+    pl.max_nb = p.k / QK;
+    pl.off_full = 0;
+    pl.off_empty = kMaxStages * 8;
+    pl.off_xfull = 2 * kMaxStages * 8;
+    pl.off_xempty = pl.off_xfull + 8;
+    pl.off_ring = 256;
+    pl.off_xq = pl.off_ring + stages * stage_bytes;
+    pl.off_xd = pl.off_xq + xmax * p.k;
+    pl.off_part = pl.off_xd + ((xmax * (p.k / QK) * 4 + 15) / 16) * 16;  // unused
+    pl.off_tab = pl.off_part;
+    pl.tab_words = group_words;
+    const int off_union = pl.off_tab + tab_bytes;
+    pl.raw_rows = raw_rows;
+    pl.off_raw = off_union;
+    pl.bytes = off_union + union_bytes;
+    pl.ctas = ctas;
+    p.off_hq = off_union + hq;
+    p.off_hd = off_union + hd;
+    p.off_y = off_union + y;
+    p.off_inv = off_union + inv;
+    p.nrb = nrb;
+    return pl.bytes <= budget;
 }
 
 q8_status launch_layer(const q8_tensor *up_gate, const q8_tensor *down, const float *x,
@@ -375,45 +459,30 @@ q8_status launch_layer(const q8_tensor *up_gate, const q8_tensor *down, const fl
     p.lay_list = L.list_small;
     p.lay_big = L.list_big;
     p.lay_pairs = L.pairs;
-    // phase-B areas after the grouping tables (all in the plan's table region)
-    const int nb_ff = (int)(n_ff / QK);
-    int o = (int)L.words * 4;
-    o = (o + 15) / 16 * 16;
-    const int hq_off = o;
-    o += (int)(P * n_ff);
-    const int hd_off = o;
-    o += (int)(P * nb_ff * 4);
-    const int y_off = o;
-    o += (int)(P * kLayerNrb * 4);
-    const int inv_off = o;
-    o += (int)(P * 4);
-    const int tab_words = (o + 3) / 4;
     const Geo ga = geo_pair_for_k(p.k);
-    int tq = ga.nr * p.k, td = (int)(ga.nr * up_gate->ld_d * 2);
-    tq = std::max(tq, kLayerNrb * kCW * p.n_ff);
-    td = std::max(td, (int)(kLayerNrb * kCW * down->ld_d * 2));
-    if (!make_plan_ctas(tq, td, p.k, (int)std::min<int64_t>(n_tok, kMaxXRows), kLayerNT, 1,
-                        &p.plan, tab_words, aligned16(x)) ||
-        p.plan.stages < 2)
-        Q8_FAIL(Q8_E_UNSUPPORTED, "moe layer: does not fit the shared-memory plan");
-    p.off_hq = p.plan.off_tab + hq_off;
-    p.off_hd = p.plan.off_tab + hd_off;
-    p.off_y = p.plan.off_tab + y_off;
-    p.off_inv = p.plan.off_tab + inv_off;
-
+    const int tq = std::max<int>(ga.nr * p.k, 8 * kCW * p.n_ff);
+    const int td = std::max<int>((int)(ga.nr * up_gate->ld_d * 2), (int)(8 * kCW * down->ld_d * 2));
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         Q8_FAIL(Q8_E_CUDA, "moe layer: no current device");
-    auto kern = moe_layer_kernel<kLayerNT>;
-    if (!smem_opted_in((const void *)kern, dev)) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kSmemLimit);
-        if (e != cudaSuccess)
-            Q8_FAIL(Q8_E_CUDA, "moe layer: shared-memory attribute: %s", cudaGetErrorString(e));
+    auto opt_in = [&](void (*kern)(LayerParams)) -> bool {
+        if (smem_opted_in((const void *)kern, dev)) return true;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
+            cudaSuccess)
+            return false;
         set_smem_opted_in((const void *)kern, dev);
-    }
+        return true;
+    };
+    // one CTA per SM with 8-row down units (two CTAs per SM, with half the
+    // ring each, measured slower: the ring then holds too little of the
+    // stream); one token runs the variant without multi-row passes
+    const int xrows = (int)std::min<int64_t>(n_tok, kMaxXRows);
+    if (!layer_plan(p, P, (int)n_ff, tq, td, xrows, 1, 8, aligned16(x), (int)L.words))
+        Q8_FAIL(Q8_E_UNSUPPORTED, "moe layer: does not fit the shared-memory plan");
+    void (*kern)(LayerParams) = n_tok == 1 ? moe_layer_kernel<1, 1> : moe_layer_kernel<kLayerNT, 1>;
+    if (!opt_in(kern)) Q8_FAIL(Q8_E_CUDA, "moe layer: shared-memory attribute refused");
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)num_sms());
+    cfg.gridDim = dim3((unsigned)(num_sms() * p.plan.ctas));
     cfg.blockDim = dim3(kThreadsStream);
     cfg.dynamicSmemBytes = (size_t)p.plan.bytes;
     cfg.stream = s;

@@ -644,8 +644,6 @@ __device__ __forceinline__ void dot_rows(const int8_t *sq, const uint16_t *sd, i
     for (int r = 0; r < RPW; ++r)
 #pragma unroll
         for (int t = 0; t < NT; ++t) acc[r][t] = 0.0f;
-    // two K steps in flight when a warp takes few rows (long rows)
-#pragma unroll(RPW <= 2 ? 2 : 1)
     for (int base = seg * 32; base < nb; base += 32 * wpr) {
         const int kb = base + lane;
         if (kb < nb) {
@@ -742,7 +740,8 @@ __device__ __forceinline__ int reduce_scatter_lane(int idx) {
 // Computes this warp's rows of a stage for activation rows [xrow0, xrow0+n)
 // and hands each warp sum to emit(row, t, v) (row within the tile, t < NT;
 // called by the one lane that holds the sum).
-template <int NT, class EmitFn>
+// RPW_ONLY != 0 compiles only that rows-per-warp case (g.rpw must equal it).
+template <int NT, int RPW_ONLY = 0, class EmitFn>
 __device__ __forceinline__ void warp_rows(const int8_t *sq, const uint16_t *sd, int k, int ld_d,
                                           const Geo &g, const XStage &xs, int xrow0, int n,
                                           EmitFn emit) {
@@ -776,11 +775,14 @@ __device__ __forceinline__ void warp_rows(const int8_t *sq, const uint16_t *sd, 
                 }                                                                             \
         }                                                                                     \
     }
-    if (g.rpw == 8) Q8_ROWS_CASE(8)
-    else if (g.rpw == 5) Q8_ROWS_CASE(5)
-    else if (g.rpw == 4) Q8_ROWS_CASE(4)
-    else if (g.rpw == 2) Q8_ROWS_CASE(2)
-    else Q8_ROWS_CASE(1)
+    if constexpr (RPW_ONLY != 0) {
+        Q8_ROWS_CASE(RPW_ONLY)
+    } else {
+        if (g.rpw == 5) Q8_ROWS_CASE(5)
+        else if (g.rpw == 4) Q8_ROWS_CASE(4)
+        else if (g.rpw == 2) Q8_ROWS_CASE(2)
+        else Q8_ROWS_CASE(1)
+    }
 #undef Q8_ROWS_CASE
 }
 
