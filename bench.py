@@ -534,10 +534,23 @@ def gpu_id(local_rank: int) -> str:
         return str(local_rank)
 
 
-def kernel_source_hash():
+# the sources each kernel is built from (its traffic record is void once any
+# of them changes)
+KERNEL_SOURCES = {
+    "gemv_batched_kernel": ["q8_matmul.cu"],
+    "up_gate_kernel": ["q8_moe.cu"],
+    "moe_layer_kernel": ["q8_layer.cu"],
+    "tc_kernel": ["q8_tc.cu", "q8_tc.cuh"],
+}
+SHARED_SOURCES = ["q8_stream.cuh", "q8_device.cuh", "q8_ptx.cuh", "q8_internal.h"]
+
+
+def kernel_source_hash(kernel=None):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "moe_up_gate_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    files = (sorted(os.listdir(csrc)) if kernel not in KERNEL_SOURCES else
+             sorted(KERNEL_SOURCES[kernel] + SHARED_SOURCES))
+    for fn in files:
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode())
             h.update(f.read())
@@ -552,7 +565,7 @@ def recorded_traffic(workload, kernel):
     except (OSError, ValueError):
         return None
     ent = rec.get(f"{workload}:{kernel}")
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
         return None
     return ent.get("dram_bytes_per_launch")
 

@@ -8,6 +8,7 @@
 // 26B-A4B Q8_0 (section 「3段階で構成された修正」), applied per routed expert.
 // All of them run on the streaming engine of q8_stream.cuh.
 #include <algorithm>
+#include <vector>
 
 #include "q8_internal.h"
 #include "q8_stream.cuh"
@@ -379,6 +380,7 @@ struct GemvBatchParams {
     int grid;
     Plan plan;
     GemvProblem pr[Q8_MAX_GEMV_DESC];
+    int cta_begin[kGemvMaxGrid + 1];      // CTA b takes tiles [cta_begin[b], cta_begin[b+1])
     uint8_t first_problem[kGemvMaxGrid];  // problem of each CTA's first tile
 };
 
@@ -391,8 +393,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     const Ring R = ring_init(smem, p.plan);
     Q8_TRACE(1);
     griddep_launch_dependents();
-    int64_t tb, te;
-    my_tiles(p.total_tiles, &tb, &te);
+    const int64_t tb = p.cta_begin[blockIdx.x], te = p.cta_begin[blockIdx.x + 1];
     if ((threadIdx.x >> 5) == kCW) {
         if ((threadIdx.x & 31) == 0 && tb < te) {
             int cur = p.first_problem[blockIdx.x];
@@ -648,12 +649,42 @@ q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_t
         1, std::min<int64_t>(std::min<int64_t>((int64_t)num_sms() * p.plan.ctas, tiles),
                              kGemvMaxGrid));
     p.grid = grid;
-    // the problem of each CTA's first tile (the kernel's my_tiles split),
-    // so that no thread searches the problem list at start
-    for (int b = 0, cur = 0; b < grid; ++b) {
-        const int64_t tb = tiles * b / grid;
-        while (cur + 1 < n_desc && p.pr[cur + 1].tile_begin <= tb) ++cur;
-        p.first_problem[b] = (uint8_t)cur;
+    // Contiguous runs of tiles of equal cost: a tile costs its bytes, and the
+    // first tile of a problem also the restaging of the activations that it
+    // makes a CTA pay (about 0.7 of a tile's time).  Also the problem of each
+    // CTA's first tile, so that no thread searches the problem list.
+    {
+        std::vector<double> cost((size_t)tiles);
+        double total = 0.0;
+        for (int i = 0; i < n_desc; ++i) {
+            const GemvProblem &q = p.pr[i];
+            const Geo g = geo_for_k(q.k);
+            const int64_t nt = (q.rows + g.nr - 1) / g.nr;
+            const double tb_bytes = (double)g.nr * q.k * 1.0625;
+            for (int64_t t = 0; t < nt; ++t) {
+                cost[(size_t)(q.tile_begin + t)] = tb_bytes * (t == 0 ? 1.7 : 1.0);
+                total += cost[(size_t)(q.tile_begin + t)];
+            }
+        }
+        double acc = 0.0;
+        int64_t t = 0;
+        p.cta_begin[0] = 0;
+        for (int b = 1; b < grid; ++b) {
+            const double target = total * b / grid;
+            while (t < tiles && acc + 0.5 * cost[(size_t)t] < target) acc += cost[(size_t)t++];
+            // keep at least one tile for each remaining CTA
+            const int64_t max_t = tiles - (grid - b);
+            if (t > max_t) {
+                while (t > max_t) acc -= cost[(size_t)--t];
+            }
+            if (t < p.cta_begin[b - 1] + 1) acc += cost[(size_t)t++];
+            p.cta_begin[b] = (int)t;
+        }
+        p.cta_begin[grid] = (int)tiles;
+        for (int b = 0, cur = 0; b < grid; ++b) {
+            while (cur + 1 < n_desc && p.pr[cur + 1].tile_begin <= p.cta_begin[b]) ++cur;
+            p.first_problem[b] = (uint8_t)cur;
+        }
     }
     cudaStream_t s = (cudaStream_t)stream;
     switch (nt) {

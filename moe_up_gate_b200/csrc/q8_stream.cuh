@@ -289,15 +289,15 @@ struct NoJobs {
 // jobs of its other groups).  Ends after the last copies have landed.
 // gated: the activations may be written by the preceding grid and this
 // thread has not waited for it yet.  The weights do not depend on that grid,
-// so the first ring's worth of tiles is issued at once; the producer then
-// waits for the grid and issues the jobs of those tiles (their consumers wait
-// for them), and goes on in stream order.
+// so the first tile is issued at once; the producer then waits for the grid,
+// issues that tile's jobs (its consumers wait for them) and goes on in stream
+// order.
 template <class SrcFn, class JobFn = NoJobs>
 __device__ __forceinline__ void produce(const Ring &R, int64_t tb, int64_t te, SrcFn src,
                                         int *err, JobFn jobs = JobFn{}, bool gated = false) {
     int it = 0;
     Q8_TRACE(20);
-    const int64_t pre = gated ? min(te, tb + (int64_t)R.stages) : tb;
+    const int64_t pre = gated ? min(te, tb + 1) : tb;
     for (int64_t t = tb; t < te; ++t, ++it) {
         const int s = it % R.stages;
         const int round = it / R.stages;
