@@ -103,9 +103,9 @@ __device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned n, int *err
 // stage, one thread per 32-block.
 template <class RowFn>
 __device__ __forceinline__ void stage_f32_l2(const XStage &xs, const float *src, int k, int n,
-                                             RowFn arow) {
+                                             RowFn arow, int tid, int nthr) {
     const int nb = k / QK;
-    for (int blk = threadIdx.x; blk < n * nb; blk += kCT) {
+    for (int blk = tid; blk < n * nb; blk += nthr) {
         const int j = blk / nb;
         const int b = blk - j * nb;
         const float4 *p = reinterpret_cast<const float4 *>(src + (int64_t)arow(j) * k + b * QK);
@@ -127,9 +127,16 @@ __device__ __forceinline__ void stage_f32_l2(const XStage &xs, const float *src,
     }
 }
 
-template <int NT, int MINB>
-__global__ void __launch_bounds__(kThreadsStream, MINB)
+// G consumer groups of kCW warps share one ring: group g takes every G-th
+// tile of phase A and every G-th unit of phase B (G = 2 doubles the warps
+// that hide each other's latency, at one CTA per SM).  G > 1 needs the
+// one-token variant (x staged once, shared by the groups).
+template <int NT, int G>
+__global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
     moe_layer_kernel(const __grid_constant__ LayerParams p) {
+    static_assert(G == 1 || NT == 1, "several consumer groups need the one-token variant");
+    constexpr int kProd = G * kCW;  // the producer warp
+    constexpr int kAll = G * kCT;   // consumer threads
     extern __shared__ __align__(128) unsigned char smem[];
     Q8_TRACE(0);
     const Ring R = ring_init(smem, p.plan);
@@ -140,7 +147,7 @@ __global__ void __launch_bounds__(kThreadsStream, MINB)
     // row, so the producer fetches it before the grouping and it is staged
     // once for the whole of phase A.
     const bool x_once = NT == 1 && R.raw_rows > 0;
-    if (x_once && threadIdx.x == kCT) {
+    if (x_once && threadIdx.x == kProd * 32) {
         mbar_arrive_expect_tx(R.xfull, (uint32_t)p.k * 4);
         bulk_g2s_keep(R.raw, p.x, (uint32_t)p.k * 4, R.xfull);
     }
@@ -169,7 +176,7 @@ __global__ void __launch_bounds__(kThreadsStream, MINB)
     my_tiles(units, &ub0, &ub1);
     auto expert = [&](int i) { return tab[p.lay_list + i]; };
 
-    if (warp == kCW) {  // ---------------- producer
+    if (warp == kProd) {  // ---------------- producer
         if (lane == 0) {
             int it = 0;
             XJobs J;
@@ -229,18 +236,27 @@ __global__ void __launch_bounds__(kThreadsStream, MINB)
         return;
     }
 
-    // ---------------- consumers, phase A: h = silu(gate . x) * (up . x)
+    // ---------------- consumers
+    const int grp = warp / kCW;  // consumer group
+    const int w8 = warp % kCW;   // warp within the group
+    const int bar_grp = kBarConsumers + grp;
+    const int bar_all = kBarConsumers + G;
+    auto sync_grp = [&]() { named_bar_sync(bar_grp, kCT); };
+    auto sync_all = [&]() { named_bar_sync(G == 1 ? kBarConsumers : bar_all, kAll); };
+
+    // phase A: h = silu(gate . x) * (up . x)
     const XStage xs{reinterpret_cast<int8_t *>(smem + p.plan.off_xq),
                     reinterpret_cast<float *>(smem + p.plan.off_xd)};
-    int it = 0, staged_mi = -1, staged_grp = -1;
+    int staged_mi = -1, staged_grp = -1;
     XJobs J;
     if (x_once) {
         mbar_wait(R.xfull, 0, &g_err_layer);
-        stage_f32_raw(xs, R.raw, p.k, 1);
-        named_bar_sync(kBarConsumers, kCT);
+        stage_f32_raw(xs, R.raw, p.k, 1, threadIdx.x, kAll);
+        sync_all();
         Q8_TRACE(7);
     }
-    for (int64_t t = ta0; t < ta1; ++t, ++it) {
+    for (int64_t t = ta0 + grp; t < ta1; t += G) {
+        const int it = (int)(t - ta0);
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_layer);
         Q8_TRACE(6);
@@ -250,17 +266,18 @@ __global__ void __launch_bounds__(kThreadsStream, MINB)
         const int32_t *plist = tab + p.lay_pairs + tab[p.lay_offset + e];
         const int r0 = ti * half;
         const int n_grp = (cnt + xmax - 1) / xmax;
-        for (int grp = 0; grp < n_grp; ++grp) {
-            const int x0 = grp * xmax;
+        for (int xg = 0; xg < n_grp; ++xg) {
+            const int x0 = xg * xmax;
             const int nx = min(xmax, cnt - x0);
-            if (!x_once && (mi != staged_mi || grp != staged_grp)) {
-                if (staged_mi >= 0) named_bar_sync(kBarConsumers, kCT);
+            if (!x_once && (mi != staged_mi || xg != staged_grp)) {
+                // (G == 1 here)
+                if (staged_mi >= 0) sync_grp();
                 stage_job_f32(R, J, xs, p.x, p.k, nx,
                               [&](int j) { return plist[x0 + j] / p.n_used; }, &g_err_layer);
-                named_bar_sync(kBarConsumers, kCT);
+                sync_grp();
                 Q8_TRACE(7);
                 staged_mi = mi;
-                staged_grp = grp;
+                staged_grp = xg;
             }
             for (int tg = 0; tg < nx; tg += NT) {
                 const int n = min(NT, nx - tg);
@@ -273,7 +290,8 @@ __global__ void __launch_bounds__(kThreadsStream, MINB)
                                             p.h[(int64_t)pr * p.n_ff + r0 + row] =
                                                 gv / (1.0f + expf(-gv)) * uv;
                                         }
-                                    });
+                                    },
+                                    w8);
                 });
                 Q8_TRACE(8);
             }
@@ -283,10 +301,10 @@ __global__ void __launch_bounds__(kThreadsStream, MINB)
     }
 
     // ---------------- every CTA's h is written
-    named_bar_sync(kBarConsumers, kCT);
+    sync_all();
     Q8_TRACE(12);
     if (threadIdx.x == 0) grid_barrier(p.bar, gridDim.x, &g_err_layer);
-    named_bar_sync(kBarConsumers, kCT);
+    sync_all();
     Q8_TRACE(11);
 
     // every pair's h as Q8_0, in grouped (expert, pair) order
@@ -295,24 +313,28 @@ __global__ void __launch_bounds__(kThreadsStream, MINB)
     const XStage hs{reinterpret_cast<int8_t *>(smem + p.off_hq),
                     reinterpret_cast<float *>(smem + p.off_hd)};
     int *inv = reinterpret_cast<int *>(smem + p.off_inv);
-    float *ybuf = reinterpret_cast<float *>(smem + p.off_y);
-    stage_f32_l2(hs, p.h, p.n_ff, n_valid, [&](int j) { return tab[p.lay_pairs + j]; });
-    for (int i = threadIdx.x; i < P; i += kCT) inv[i] = -1;
-    named_bar_sync(kBarConsumers, kCT);
-    for (int j = threadIdx.x; j < n_valid; j += kCT) inv[tab[p.lay_pairs + j]] = j;
-    named_bar_sync(kBarConsumers, kCT);
+    float *ybuf = reinterpret_cast<float *>(smem + p.off_y) + (size_t)grp * P * nrb;
+    stage_f32_l2(hs, p.h, p.n_ff, n_valid, [&](int j) { return tab[p.lay_pairs + j]; },
+                 threadIdx.x, kAll);
+    for (int i = threadIdx.x; i < P; i += kAll) inv[i] = -1;
+    sync_all();
+    for (int j = threadIdx.x; j < n_valid; j += kAll) inv[tab[p.lay_pairs + j]] = j;
+    sync_all();
     Q8_TRACE(7);
 
     // ---------------- phase B: y = down . hq, out = sum_s p y
     const Geo gb{nrb * kCW, 1, nrb};
-    for (int64_t u = ub0; u < ub1; ++u) {
+    const int itb = (int)(ta1 - ta0);  // ring position of the first phase-B stage
+    const int gtid = threadIdx.x - grp * kCT;
+    for (int64_t u = ub0 + grp; u < ub1; u += G) {
         const int r0 = (int)u * nrb;
         const int nrv = min(nrb, p.k - r0);
-        for (int sg = 0; sg < sg_per_unit; ++sg, ++it) {
+        for (int sg = 0; sg < sg_per_unit; ++sg) {
+            const int it = itb + (int)(u - ub0) * sg_per_unit + sg;
             const int s = it % R.stages;
             mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_layer);
             Q8_TRACE(6);
-            const int mi = sg * kCW + warp;
+            const int mi = sg * kCW + w8;
             if (mi < n_exp) {
                 const int e = expert(mi);
                 const int cnt = tab[p.lay_count + e];
@@ -325,15 +347,15 @@ __global__ void __launch_bounds__(kThreadsStream, MINB)
                     with_nt<NB>(n, [&](auto ntc) {
                         constexpr int NTC = decltype(ntc)::value;
                         auto emit = [&](int row, int tt, float v) {
-                            const int rr = row - warp * nrb;
+                            const int rr = row - w8 * nrb;
                             if (tt < n && rr < nrv) ybuf[(off + tg + tt) * nrb + rr] = v;
                         };
                         if (nrb == 8)
                             warp_rows<NTC, 8>(R.qs(s), R.d(s), p.n_ff, (int)p.dn_ld_d, gb, hs,
-                                              off + tg, n, emit);
+                                              off + tg, n, emit, w8);
                         else
                             warp_rows<NTC, 4>(R.qs(s), R.d(s), p.n_ff, (int)p.dn_ld_d, gb, hs,
-                                              off + tg, n, emit);
+                                              off + tg, n, emit, w8);
                     });
                 }
             }
@@ -341,8 +363,8 @@ __global__ void __launch_bounds__(kThreadsStream, MINB)
             if (lane == 0) mbar_arrive(&R.empty[s]);
             Q8_TRACE(8);
         }
-        named_bar_sync(kBarConsumers, kCT);
-        for (int i = threadIdx.x; i < p.n_tok * nrv; i += kCT) {
+        sync_grp();
+        for (int i = gtid; i < p.n_tok * nrv; i += kCT) {
             const int t = i / nrv;
             const int rr = i - t * nrv;
             float acc = 0.0f;
@@ -352,7 +374,7 @@ __global__ void __launch_bounds__(kThreadsStream, MINB)
             }
             p.out[(int64_t)t * p.k + r0 + rr] = acc;
         }
-        named_bar_sync(kBarConsumers, kCT);
+        sync_grp();
         Q8_TRACE(10);
     }
 }
@@ -372,7 +394,7 @@ bool layer_eligible(const q8_tensor *up_gate, const q8_tensor *down, int64_t n_t
 // and the phase-B areas (all pairs' hq and scales, y, the pair inverse)
 // afterwards.
 static bool layer_plan(LayerParams &p, int64_t P, int n_ff, int tq, int td, int xrows, int ctas,
-                       int nrb, bool raw, int group_words) {
+                       int nrb, bool raw, int group_words, int groups) {
     const int budget = smem_budget(ctas);
     const int nb_ff = n_ff / QK;
     const int xmax = xrows;
@@ -387,7 +409,7 @@ static bool layer_plan(LayerParams &p, int64_t P, int n_ff, int tq, int td, int 
     const int hd = o;
     o += (int)(P * nb_ff * 4);
     const int y = o;
-    o += (int)(P * nrb * 4);
+    o += (int)(P * nrb * 4) * groups;  // one y buffer per consumer group
     const int inv = o;
     o += (int)(P * 4);
     const int union_bytes = (std::max(o, raw_bytes) + 127) / 128 * 128;
@@ -477,13 +499,15 @@ q8_status launch_layer(const q8_tensor *up_gate, const q8_tensor *down, const fl
     // ring each, measured slower: the ring then holds too little of the
     // stream); one token runs the variant without multi-row passes
     const int xrows = (int)std::min<int64_t>(n_tok, kMaxXRows);
-    if (!layer_plan(p, P, (int)n_ff, tq, td, xrows, 1, 8, aligned16(x), (int)L.words))
+    // one token: two consumer groups (the x row is staged once and shared)
+    const int groups = n_tok == 1 && aligned16(x) ? 2 : 1;
+    if (!layer_plan(p, P, (int)n_ff, tq, td, xrows, 1, 8, aligned16(x), (int)L.words, groups))
         Q8_FAIL(Q8_E_UNSUPPORTED, "moe layer: does not fit the shared-memory plan");
-    void (*kern)(LayerParams) = n_tok == 1 ? moe_layer_kernel<1, 1> : moe_layer_kernel<kLayerNT, 1>;
+    void (*kern)(LayerParams) = groups == 2 ? moe_layer_kernel<1, 2> : moe_layer_kernel<kLayerNT, 1>;
     if (!opt_in(kern)) Q8_FAIL(Q8_E_CUDA, "moe layer: shared-memory attribute refused");
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)(num_sms() * p.plan.ctas));
-    cfg.blockDim = dim3(kThreadsStream);
+    cfg.blockDim = dim3((unsigned)((groups * kCW + 1) * 32));
     cfg.dynamicSmemBytes = (size_t)p.plan.bytes;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];

@@ -569,9 +569,13 @@ __device__ __forceinline__ void stage_f32(const XStage &xs, const float *__restr
 // Quantize the n fp32 rows of the raw slot (row j at raw + j * k) into the
 // stage: stage_f32's rule, from shared memory, one consumer thread per block
 // (no cross-lane steps, so a thread's blocks are independent chains).
-__device__ __forceinline__ void stage_f32_raw(const XStage &xs, const float *raw, int k, int n) {
+// tid/nthr: this thread's index among the nthr threads that share the work
+// (default: the consumer threads).
+__device__ __forceinline__ void stage_f32_raw(const XStage &xs, const float *raw, int k, int n,
+                                              int tid = -1, int nthr = kCT) {
     const int nb = k / QK;
-    for (int blk = threadIdx.x; blk < n * nb; blk += kCT) {
+    if (tid < 0) tid = threadIdx.x;
+    for (int blk = tid; blk < n * nb; blk += nthr) {
         const int j = blk / nb;
         const int b = blk - j * nb;
         const float4 *src = reinterpret_cast<const float4 *>(raw + (size_t)j * k + b * QK);
@@ -741,11 +745,13 @@ __device__ __forceinline__ int reduce_scatter_lane(int idx) {
 // and hands each warp sum to emit(row, t, v) (row within the tile, t < NT;
 // called by the one lane that holds the sum).
 // RPW_ONLY != 0 compiles only that rows-per-warp case (g.rpw must equal it).
+// warp_id: the warp's index among the tile's consumer warps (default: its
+// index in the CTA).
 template <int NT, int RPW_ONLY = 0, class EmitFn>
 __device__ __forceinline__ void warp_rows(const int8_t *sq, const uint16_t *sd, int k, int ld_d,
                                           const Geo &g, const XStage &xs, int xrow0, int n,
-                                          EmitFn emit) {
-    const int warp = threadIdx.x >> 5;
+                                          EmitFn emit, int warp_id = -1) {
+    const int warp = warp_id >= 0 ? warp_id : (int)(threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     const int seg = warp % g.wpr;
     const int row0 = (warp / g.wpr) * g.rpw;
@@ -793,8 +799,8 @@ __device__ __forceinline__ void warp_rows(const int8_t *sq, const uint16_t *sd, 
 template <int NT, class EmitFn>
 __device__ __forceinline__ void warp_pairs(const int8_t *sq, const uint16_t *sd, int k, int ld_d,
                                            const Geo &g, int half, const XStage &xs, int xrow0,
-                                           int n, EmitFn emit) {
-    const int warp = threadIdx.x >> 5;
+                                           int n, EmitFn emit, int warp_id = -1) {
+    const int warp = warp_id >= 0 ? warp_id : (int)(threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
 #define Q8_PAIRS_CASE(RPW_)                                                                   \
     {                                                                                         \
