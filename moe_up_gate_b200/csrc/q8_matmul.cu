@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     Q8_TRACE(0);
     const Ring R = ring_init(smem, p.plan);
     Q8_TRACE(1);
-    const Geo g = geo_for_k(p.k);
+    const Geo g = geo_for_k(p.k, NT);
     const int tpm = (p.rows + g.nr - 1) / g.nr;
     griddep_launch_dependents();
     const int32_t *tab = p.ws;
@@ -243,7 +243,7 @@ q8_status launch_matmul(const MatmulParams &base, RowPlan rp, int64_t max_tiles,
     const int tab_words =
         p.ids ? (int)group_layout((int64_t)p.n_tok * p.n_used, p.n_mat).words : 0;
     int tq, td;
-    tile_bytes(geo_for_k(p.k), p.k, p.ld_d, &tq, &td);
+    tile_bytes(geo_for_k(p.k, nt), p.k, p.ld_d, &tq, &td);
     if (!make_plan(tq, td, p.k, (int)std::min<int64_t>(rp.x_rows, kMaxXRows), nt, &p.plan,
                    tab_words, p.af != nullptr && aligned16(p.af)))
         Q8_FAIL(Q8_E_UNSUPPORTED, "matmul: k=%d does not fit the shared-memory plan", p.k);
@@ -287,7 +287,7 @@ q8_status launch_matmul_routed(const q8_tensor *W, const int8_t *aq, const uint1
     // shape allows it; otherwise the dp4a kernel takes them too
     const bool tc = tc_eligible(W, false) && P >= kTcMinPairs;
     p.include_big = tc ? 0 : 1;
-    const Geo g = geo_for_k(p.k);
+    const Geo g = geo_for_k(p.k, 8);
     const int64_t tiles = std::min<int64_t>(W->n_mat, P) * ((p.rows + g.nr - 1) / g.nr);
     q8_status st = launch_matmul(p, routed_rows(n_tok, n_used, W->n_mat), tiles, s);
     if (st != Q8_OK || !tc) return st;
@@ -326,7 +326,7 @@ q8_status launch_matmul_routed_ids(const q8_tensor *W, const int8_t *aq, const u
     p.n_tok = (int)n_tok;
     p.n_mat = (int)W->n_mat;
     p.err_out = err_out;
-    const Geo g = geo_for_k(p.k);
+    const Geo g = geo_for_k(p.k, 8);
     const int64_t tiles = std::min<int64_t>(W->n_mat, P) * ((p.rows + g.nr - 1) / g.nr);
     return launch_matmul(p, routed_rows(n_tok, n_used, W->n_mat), tiles, s);
 }
@@ -334,7 +334,7 @@ q8_status launch_matmul_routed_ids(const q8_tensor *W, const int8_t *aq, const u
 // Dense matmul of fp32 (af) or Q8_0 (aq/ad) activation rows: y = W a.
 q8_status launch_matmul_dense(const q8_tensor *W, const int8_t *aq, const uint16_t *ad,
                               const float *af, int64_t n_tok, float *y, cudaStream_t s) {
-    const Geo g = geo_for_k((int)W->k);
+    const Geo g = geo_for_k((int)W->k, 8);
     const int64_t tiles = (W->rows + g.nr - 1) / g.nr;
     for (int64_t t0 = 0; t0 < n_tok; t0 += kMaxXRows) {
         const int64_t nt = std::min<int64_t>(kMaxXRows, n_tok - t0);
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
             auto src = [&](int64_t t) {
                 while (cur + 1 < p.n_desc && p.pr[cur + 1].tile_begin <= t) ++cur;
                 const GemvProblem &q = p.pr[cur];
-                const Geo g = geo_for_k(q.k);
+                const Geo g = geo_for_k(q.k, NT);
                 const int r0 = (int)(t - q.tile_begin) * g.nr;
                 TileSrc ts{};
                 ts.q0 = q.wq + (int64_t)r0 * q.k;
@@ -445,7 +445,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     for (int64_t t = tb; t < te; ++t, ++it) {
         while (cur + 1 < p.n_desc && p.pr[cur + 1].tile_begin <= t) ++cur;
         const GemvProblem &q = p.pr[cur];
-        const Geo g = geo_for_k(q.k);
+        const Geo g = geo_for_k(q.k, NT);
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_matmul);
         Q8_TRACE(6);
@@ -614,6 +614,7 @@ q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_t
     p.n_tok = (int)n_tok;
     int64_t tiles = 0;
     int max_k = 32, max_tq = 0, max_td = 0;
+    const int nt = pick_nt(n_tok);
     for (int i = 0; i < n_desc; ++i) {
         const q8_gemv_desc &d = descs[i];
         q8_status st = check_tensor(&d.W, "q8_gemv_batched: W", true);
@@ -631,7 +632,7 @@ q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_t
         q.k = (int)d.W.k;
         q.rows = (int)d.W.rows;
         q.tile_begin = (int)tiles;
-        const Geo g = geo_for_k(q.k);
+        const Geo g = geo_for_k(q.k, nt);
         tiles += (d.W.rows + g.nr - 1) / g.nr;
         max_k = std::max(max_k, q.k);
         int tq, td;
@@ -641,7 +642,6 @@ q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_t
     }
     Q8_REQUIRE(tiles < (1LL << 31), Q8_E_SHAPE, "q8_gemv_batched: too many tiles");
     p.total_tiles = (int)tiles;
-    const int nt = pick_nt(n_tok);
     if (!make_plan(max_tq, max_td, max_k, (int)std::min<int64_t>(n_tok, kMaxXRows), nt, &p.plan,
                    0, true))
         Q8_FAIL(Q8_E_UNSUPPORTED, "q8_gemv_batched: k=%d does not fit the plan", max_k);
@@ -658,7 +658,7 @@ q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_t
         double total = 0.0;
         for (int i = 0; i < n_desc; ++i) {
             const GemvProblem &q = p.pr[i];
-            const Geo g = geo_for_k(q.k);
+            const Geo g = geo_for_k(q.k, nt);
             const int64_t nt = (q.rows + g.nr - 1) / g.nr;
             const double tb_bytes = (double)g.nr * q.k * 1.0625;
             for (int64_t t = 0; t < nt; ++t) {

@@ -54,9 +54,11 @@ struct Geo {
     int nr, wpr, rpw;
 };
 __host__ __device__ inline int wpr_for_k(int k) { return k <= 4096 ? 1 : 8; }
-// Plain row tiles (at most 32 KB of quants).
-__host__ __device__ inline Geo geo_for_k(int k) {
-    if (k <= 768) return {40, 1, 5};
+// Plain row tiles (at most 32 KB of quants).  nt: activation rows per pass
+// of the kernel; at 8 a warp takes 4 rows (k <= 768) so that its rpw * nt
+// sums stay within one reduce-scatter (the sum order of a row is the same).
+__host__ __device__ inline Geo geo_for_k(int k, int nt = 1) {
+    if (k <= 768) return nt >= 8 ? Geo{32, 1, 4} : Geo{40, 1, 5};
     if (k <= 1024) return {32, 1, 4};
     if (k <= 2048) return {16, 1, 2};
     if (k <= 4096) return {8, 1, 1};

@@ -4,21 +4,18 @@
 // activation rows per expert the step is a real (small) dense contraction,
 // so it goes to the tensor cores; below that the dp4a streaming kernels serve.
 //
-// One CTA computes one 128-row weight tile of one expert (up/gate: 64 gate
-// rows and the 64 matching up rows) for up to 32 of the expert's routed rows
-// at a time:
-//  * warp 0 (one lane) streams the tile in 128-byte K chunks (4 Q8_0 blocks)
-//    with 2-D tensor (TMA) loads into a ring of 128-byte-swizzled stages;
-//  * the activation rows are staged once, as Q8_0, in the canonical no-swizzle
-//    K-major layout (8-row x 16-byte core matrices), padded with zero rows to
-//    a multiple of 16;
-//  * warp 1 (one lane) issues one tcgen05.mma.kind::i8 per Q8_0 block
-//    (M=128, N=16..32, K=32): every block's exact int32 dot products land in
-//    a tensor-memory slot of their own, because each block has its own pair
-//    of scales and the int32 sum cannot run across blocks;
-//  * warps 2-9 read each slot back (thread = weight row, 16 activation rows
-//    per warp), scale by d_w * d_x in fp32 and accumulate, in block order.
-// Every wait is bounded (q8_ptx.cuh); tensor memory is freed before exit.
+// A persistent grid (one CTA per SM) walks work items (expert, pass of up to
+// 32 of its rows, 128-row weight tile; up/gate tiles are 64 gate rows and the
+// 64 matching up rows) through one ring whose stages hold, per 128-byte K
+// chunk (4 Q8_0 blocks): the weight tile's chunk (2-D TMA, 128-byte swizzle),
+// the activation rows' chunk as Q8_0 in the canonical no-swizzle K-major
+// core-matrix layout (built by two warps from the rows the pair list names),
+// and those rows' block scales.  One tcgen05.mma.kind::i8 per Q8_0 block
+// (M=128, N=16/32, K=32) lands in its own tensor-memory slot, because each
+// block has its own pair of scales and the int32 sum cannot run across
+// blocks; eight epilogue warps read the slots back, scale by d_w * d_x in
+// fp32 and accumulate in block order.  Every wait is bounded (q8_ptx.cuh);
+// tensor memory is freed before exit.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -34,10 +31,15 @@ namespace q8 {
 constexpr int kTcN = 32;            // activation rows per pass
 constexpr int kTcSlots = 8;         // tensor-memory slots of kTcN columns
 constexpr int kTcCols = 256;        // columns allocated
-constexpr int kTcStage = 16384;     // 128 rows x 128 bytes
-constexpr int kTcThreads = 320;     // producer, MMA, 8 epilogue warps
+constexpr int kTcA = 16384;         // A part of a stage: 128 rows x 128 bytes (128B swizzle)
+constexpr int kTcB = kTcN * 128;    // B part: kTcN rows x 128 bytes (core matrices)
+constexpr int kTcDx = kTcN * 4 * 4; // activation scales of the stage's 4 blocks
+constexpr int kTcStage = 21504;     // kTcA + kTcB + kTcDx rounded to 1024
 constexpr int kTcEpiWarps = 8;
+constexpr int kTcBuildWarps = 2;
+constexpr int kTcThreads = (2 + kTcEpiWarps + kTcBuildWarps) * 32;  // 384
 constexpr int kTcMaxK = 4096;
+static_assert(kTcA + kTcB + kTcDx <= kTcStage && kTcStage % 1024 == 0, "stage layout");
 
 static __device__ int g_err_tc;
 
@@ -63,7 +65,8 @@ struct TcParams {
     const int32_t *ws;
     int64_t lay_count, lay_offset, lay_big, lay_pairs;
     int stages;
-    int off_x, off_dx, off_xchg, off_dw, off_bar;
+    int off_dws, off_xchg, off_bar;
+    int dws_bytes;  // one of the two tile-scale buffers
 };
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -72,43 +75,115 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ float tc_silu(float z) { return z / (1.0f + expf(-z)); }
 
+// The CTA's work items, in order: (expert of the tensor-core list, pass of
+// kTcN of its rows, weight tile).  Every role walks the same sequence.
+struct TcItem {
+    int mi, pass, tile;     // position
+    int e, cnt, c0, n, npad;
+    const int32_t *plist;
+};
+
+struct TcWalk {
+    const TcParams *p;
+    int n_big, n_tiles;
+    __device__ __forceinline__ int passes(int mi) const {
+        const int e = p->ws[p->lay_big + mi];
+        return (p->ws[p->lay_count + e] + kTcN - 1) / kTcN;
+    }
+    __device__ __forceinline__ void fill(TcItem &it) const {
+        it.e = p->ws[p->lay_big + it.mi];
+        it.cnt = p->ws[p->lay_count + it.e];
+        it.plist = p->ws + p->lay_pairs + p->ws[p->lay_offset + it.e];
+        it.c0 = it.pass * kTcN;
+        it.n = min(kTcN, it.cnt - it.c0);
+        it.npad = (it.n + 15) / 16 * 16;
+    }
+    // the item with index i (sequential scan of the expert list)
+    __device__ __forceinline__ TcItem seek(int64_t i) const {
+        TcItem it{};
+        int64_t before = 0;
+        for (it.mi = 0; it.mi < n_big; ++it.mi) {
+            const int64_t cnt = (int64_t)passes(it.mi) * n_tiles;
+            if (i < before + cnt) break;
+            before += cnt;
+        }
+        const int64_t r = i - before;
+        it.pass = (int)(r / n_tiles);
+        it.tile = (int)(r % n_tiles);
+        if (it.mi < n_big) fill(it);
+        return it;
+    }
+    __device__ __forceinline__ void next(TcItem &it) const {
+        if (++it.tile == n_tiles) {
+            it.tile = 0;
+            if (++it.pass == passes(it.mi)) {
+                it.pass = 0;
+                ++it.mi;
+            }
+        }
+        if (it.mi < n_big) fill(it);
+    }
+    __device__ __forceinline__ int64_t total() const {
+        int64_t t = 0;
+        for (int mi = 0; mi < n_big; ++mi) t += (int64_t)passes(mi) * n_tiles;
+        return t;
+    }
+};
+
+// Persistent: each CTA takes a contiguous run of the work items and streams
+// them through one ring, keeping its tensor memory.  Roles:
+//  warp 0        A producer: the tile's K chunks by 2-D TMA (128B swizzle),
+//                and the tile's weight scales by bulk copy (two buffers);
+//  warp 1        tensor-memory owner and MMA issuer: one kind::i8 MMA per
+//                Q8_0 block into its own tensor-memory slot;
+//  warps 2-9     epilogue: thread = weight row, 16 activation rows per warp;
+//  warps 10-11   B builders: the chunk's activation rows (gathered through
+//                the pair list) as Q8_0 core matrices and their scales, into
+//                the same stage.
+// A stage is freed by the epilogue (it reads the stage's activation scales).
 __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant__ TcParams p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // the 128-byte-swizzled stages need 1024-byte alignment
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     griddep_launch_dependents();
     griddep_wait();  // the grouping tables and the activations come from earlier kernels
-    if ((int)blockIdx.y >= p.ws[WS_N_BIG]) return;  // uniform: before any barrier
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool upgate = p.n_ff > 0;
-    const int e = p.ws[p.lay_big + blockIdx.y];
-    const int cnt = p.ws[p.lay_count + e];
-    const int32_t *plist = p.ws + p.lay_pairs + p.ws[p.lay_offset + e];
-    const int row0 = blockIdx.x * (upgate ? 64 : 128);
     const int k = p.k, nb = k / QK, nkc = (k + 127) / 128;
+    TcWalk W{&p, p.ws[WS_N_BIG], upgate ? p.n_ff / 64 : (p.rows + 127) / 128};
+    // the item count, by one lane per warp (a scan of the expert list)
+    int64_t total = 0;
+    if (lane == 0) total = W.total();
+    total = __shfl_sync(0xffffffffu, total, 0);
+    const int64_t i0 = total * blockIdx.x / gridDim.x, i1 = total * (blockIdx.x + 1) / gridDim.x;
+    if (i0 >= i1) return;  // uniform: before any barrier
 
     unsigned char *ring = smem;
-    int8_t *xs = reinterpret_cast<int8_t *>(smem + p.off_x);
-    float *dxs = reinterpret_cast<float *>(smem + p.off_dx);
     float *xchg = reinterpret_cast<float *>(smem + p.off_xchg);
-    uint16_t *dws = reinterpret_cast<uint16_t *>(smem + p.off_dw);  // the tile's weight scales
-    uint64_t *wfull = reinterpret_cast<uint64_t *>(smem + p.off_bar);
-    uint64_t *wempty = wfull + p.stages;
-    uint64_t *sfull = wempty + p.stages;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.off_bar);
+    uint64_t *empty = full + p.stages;
+    uint64_t *sfull = empty + p.stages;
     uint64_t *sempty = sfull + kTcSlots;
     uint64_t *dfull = sempty + kTcSlots;
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(dfull + 1);
+    uint64_t *dempty = dfull + 2;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(dempty + 2);
+    auto dws = [&](int d) {
+        return reinterpret_cast<uint16_t *>(smem + p.off_dws + (size_t)d * p.dws_bytes);
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
-            mbar_init(&wfull[s], 1);
-            mbar_init(&wempty[s], 1);
+            mbar_init(&full[s], 1 + kTcBuildWarps);
+            mbar_init(&empty[s], kTcEpiWarps);
         }
         for (int s = 0; s < kTcSlots; ++s) {
             mbar_init(&sfull[s], 1);
             mbar_init(&sempty[s], kTcEpiWarps);
         }
-        mbar_init(dfull, 1);
+        for (int d = 0; d < 2; ++d) {
+            mbar_init(&dfull[d], 1);
+            mbar_init(&dempty[d], kTcEpiWarps);
+        }
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -120,115 +195,127 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
 
-    int kcg = 0;  // k chunks streamed so far (ring position)
-    int bg = 0;   // blocks issued / consumed so far (slot position)
-    for (int c0 = 0; c0 < cnt; c0 += kTcN) {
-        const int n = min(kTcN, cnt - c0);
-        const int npad = (n + 15) / 16 * 16;
-        const int ngrp = npad / 8;  // 8-row groups
-        __syncthreads();  // the previous pass's MMAs and epilogue are done with xs
-        // ---- stage the activation rows as Q8_0, no-swizzle K-major core matrices
-        auto arow = [&](int j) {
-            const int pr = plist[c0 + j];
-            return p.a_per_slot ? pr : pr / p.n_used;
-        };
-        if (p.af) {
-            for (int blk = warp; blk < npad * nb; blk += kTcThreads / 32) {
-                const int j = blk / nb, b = blk - j * nb;
-                const float v = j < n ? p.af[(int64_t)arow(j) * k + b * QK + lane] : 0.0f;
-                const float amax = warp_max_all(fabsf(v));
-                const float d32 = block_scale(amax);
-                const float id = block_inv_scale(d32);
-                const int kbyte = b * QK + lane;
-                const int c = kbyte >> 4;
-                xs[(c * ngrp + (j >> 3)) * 128 + (j & 7) * 16 + (kbyte & 15)] =
-                    (int8_t)quantize_one(v, id);
-                if (lane == 0) dxs[j * nb + b] = j < n ? scale_value(scale_bits(d32)) : 0.0f;
-            }
-        } else {
-            const int chunks = k / 16;
-            for (int i = threadIdx.x; i < npad * chunks; i += kTcThreads) {
-                const int j = i / chunks, c = i - j * chunks;
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (j < n) v = *reinterpret_cast<const uint4 *>(p.aq + (int64_t)arow(j) * k + c * 16);
-                *reinterpret_cast<uint4 *>(xs + (c * ngrp + (j >> 3)) * 128 + (j & 7) * 16) = v;
-            }
-            for (int i = threadIdx.x; i < npad * nb; i += kTcThreads) {
-                const int j = i / nb, b = i - j * nb;
-                dxs[i] = j < n ? scale_value(p.ad[(int64_t)arow(j) * nb + b]) : 0.0f;
-            }
-        }
-        fence_proxy_async_smem();  // generic-proxy writes, read by the tensor cores
-        __syncthreads();
-
+    TcItem it = W.seek(i0);
+    int g = 0;   // K chunks so far (ring position)
+    int bg = 0;  // blocks so far (slot position)
+    for (int64_t ii = 0; ii < i1 - i0; ++ii, W.next(it)) {
+        const int d = (int)(ii & 1);
+        const int row0 = it.tile * (upgate ? 64 : 128);
+        const int64_t mrow = (int64_t)it.e * p.mat_stride;
         if (warp == 0) {
-            // ---- producer: the tile's K chunks through the ring
+            // ---- A producer
             if (lane == 0) {
-                if (c0 == 0) {  // the tile's scales, once: contiguous rows of ld_d halves
-                    const int64_t mrow = (int64_t)e * p.mat_stride;
-                    if (upgate) {
-                        const uint32_t bytes = (uint32_t)(64 * p.ld_d * 2);
-                        mbar_arrive_expect_tx(dfull, 2 * bytes);
-                        bulk_g2s(dws, p.wd + (mrow + row0) * p.ld_d, bytes, dfull);
-                        bulk_g2s(dws + 64 * p.ld_d, p.wd + (mrow + p.n_ff + row0) * p.ld_d, bytes, dfull);
-                    } else {
-                        const int valid = min(128, p.rows - row0);
-                        const uint32_t bytes = (uint32_t)(valid * p.ld_d * 2);
-                        mbar_arrive_expect_tx(dfull, bytes);
-                        bulk_g2s(dws, p.wd + (mrow + row0) * p.ld_d, bytes, dfull);
-                    }
+                if (ii >= 2) mbar_wait(&dempty[d], (int)((ii / 2 - 1) & 1), &g_err_tc);
+                if (upgate) {
+                    const uint32_t bytes = (uint32_t)(64 * p.ld_d * 2);
+                    mbar_arrive_expect_tx(&dfull[d], 2 * bytes);
+                    bulk_g2s(dws(d), p.wd + (mrow + row0) * p.ld_d, bytes, &dfull[d]);
+                    bulk_g2s(dws(d) + 64 * p.ld_d, p.wd + (mrow + p.n_ff + row0) * p.ld_d, bytes,
+                             &dfull[d]);
+                } else {
+                    const int valid = min(128, p.rows - row0);
+                    const uint32_t bytes = (uint32_t)(valid * p.ld_d * 2);
+                    mbar_arrive_expect_tx(&dfull[d], bytes);
+                    bulk_g2s(dws(d), p.wd + (mrow + row0) * p.ld_d, bytes, &dfull[d]);
                 }
-                for (int kc = 0; kc < nkc; ++kc, ++kcg) {
-                    const int s = kcg % p.stages, round = kcg / p.stages;
-                    if (round > 0) mbar_wait(&wempty[s], (round - 1) & 1, &g_err_tc);
-                    mbar_arrive_expect_tx(&wfull[s], kTcStage);
+                for (int kc = 0; kc < nkc; ++kc) {
+                    const int gg = g + kc, s = gg % p.stages;
+                    if (gg >= p.stages) mbar_wait(&empty[s], (gg / p.stages - 1) & 1, &g_err_tc);
+                    mbar_arrive_expect_tx(&full[s], kTcA);
                     unsigned char *dst = ring + (size_t)s * kTcStage;
-                    const int64_t mrow = (int64_t)e * p.mat_stride;
                     if (upgate) {
-                        tma_load_2d(dst, &p.tmap, kc * 128, (int)(mrow + row0), &wfull[s]);
-                        tma_load_2d(dst + kTcStage / 2, &p.tmap, kc * 128,
-                                    (int)(mrow + p.n_ff + row0), &wfull[s]);
+                        tma_load_2d(dst, &p.tmap, kc * 128, (int)(mrow + row0), &full[s]);
+                        tma_load_2d(dst + kTcA / 2, &p.tmap, kc * 128, (int)(mrow + p.n_ff + row0),
+                                    &full[s]);
                     } else {
-                        tma_load_2d(dst, &p.tmap, kc * 128, (int)(mrow + row0), &wfull[s]);
+                        tma_load_2d(dst, &p.tmap, kc * 128, (int)(mrow + row0), &full[s]);
                     }
                 }
-            } else {
-                kcg += nkc;
+            }
+        } else if (warp >= 2 + kTcEpiWarps) {
+            // ---- B builders: thread per (row, block of the chunk)
+            const int tid = threadIdx.x - (2 + kTcEpiWarps) * 32;
+            const int ngrp = it.npad / 8;
+            for (int kc = 0; kc < nkc; ++kc) {
+                const int gg = g + kc, s = gg % p.stages;
+                if (gg >= p.stages) mbar_wait(&empty[s], (gg / p.stages - 1) & 1, &g_err_tc);
+                unsigned char *bst = ring + (size_t)s * kTcStage + kTcA;
+                float *dxs = reinterpret_cast<float *>(bst + kTcB);
+                for (int idx = tid; idx < it.npad * 4; idx += kTcBuildWarps * 32) {
+                    const int j = idx >> 2, b4 = idx & 3;
+                    const int kb = kc * 4 + b4;
+                    uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+                    float dx = 0.0f;
+                    if (j < it.n && kb < nb) {
+                        const int pr = it.plist[it.c0 + j];
+                        const int64_t r = p.a_per_slot ? pr : pr / p.n_used;
+                        if (p.af) {
+                            const float4 *src =
+                                reinterpret_cast<const float4 *>(p.af + r * k + kb * QK);
+                            float v[32];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float4 f = src[i];
+                                v[4 * i] = f.x;
+                                v[4 * i + 1] = f.y;
+                                v[4 * i + 2] = f.z;
+                                v[4 * i + 3] = f.w;
+                            }
+                            uint32_t q[8];
+                            const float d32 = quantize_block_thread(v, q);
+                            lo = make_uint4(q[0], q[1], q[2], q[3]);
+                            hi = make_uint4(q[4], q[5], q[6], q[7]);
+                            dx = scale_value(scale_bits(d32));
+                        } else {
+                            const uint4 *src = reinterpret_cast<const uint4 *>(p.aq + r * k + kb * QK);
+                            lo = src[0];
+                            hi = src[1];
+                            dx = scale_value(p.ad[r * nb + kb]);
+                        }
+                    }
+                    // core matrix (16-byte column c, 8-row group j/8)
+                    const int c = 2 * b4;
+                    *reinterpret_cast<uint4 *>(bst + (c * ngrp + (j >> 3)) * 128 + (j & 7) * 16) = lo;
+                    *reinterpret_cast<uint4 *>(bst + ((c + 1) * ngrp + (j >> 3)) * 128 + (j & 7) * 16) = hi;
+                    dxs[j * 4 + b4] = dx;
+                }
+                fence_proxy_async_smem();  // generic-proxy writes, read by the tensor cores
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[s]);
             }
         } else if (warp == 1) {
-            // ---- MMA issuer: one MMA per Q8_0 block into its own slot
-            const uint32_t idesc = idesc_i8(npad);
-            const uint32_t xs_addr = smem_u32(xs);
-            const uint32_t lbo = (uint32_t)ngrp * 128;
-            for (int b = 0; b < nb; ++b, ++bg) {
-                const int kq = kcg + b / 4;
-                const int s = kq % p.stages;
-                if (lane == 0) {
-                    if ((b & 3) == 0) {
-                        mbar_wait(&wfull[s], (kq / p.stages) & 1, &g_err_tc);
-                        tc_fence_after();
+            // ---- MMA issuer
+            if (lane == 0) {
+                const uint32_t idesc = idesc_i8(it.npad);
+                const uint32_t lbo = (uint32_t)(it.npad / 8) * 128;
+                int bb = bg;
+                for (int kc = 0; kc < nkc; ++kc) {
+                    const int gg = g + kc, s = gg % p.stages;
+                    mbar_wait(&full[s], (gg / p.stages) & 1, &g_err_tc);
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(ring + (size_t)s * kTcStage);
+                    const uint32_t b_base = a_base + kTcA;
+                    const int gn = min(4, nb - kc * 4);
+                    for (int b4 = 0; b4 < gn; ++b4, ++bb) {
+                        const int slot = bb % kTcSlots;
+                        if (bb >= kTcSlots) {
+                            mbar_wait(&sempty[slot], (bb / kTcSlots - 1) & 1, &g_err_tc);
+                            tc_fence_after();
+                        }
+                        const uint64_t adesc = smem_desc(a_base + b4 * 32, 16, 1024, 2);
+                        const uint64_t bdesc = smem_desc(b_base + (uint32_t)(2 * b4) * lbo, lbo, 128, 0);
+                        mma_i8(tmem + (uint32_t)(slot * kTcN), adesc, bdesc, idesc, 0);
+                        tc_commit(&sfull[slot]);
                     }
-                    const int slot = bg % kTcSlots, sround = bg / kTcSlots;
-                    if (sround > 0) {
-                        mbar_wait(&sempty[slot], (sround - 1) & 1, &g_err_tc);
-                        tc_fence_after();
-                    }
-                    const uint32_t a_addr = smem_u32(ring + (size_t)s * kTcStage) + (b & 3) * 32;
-                    const uint64_t adesc = smem_desc(a_addr, 16, 1024, 2);
-                    const uint64_t bdesc = smem_desc(xs_addr + (uint32_t)(2 * b) * lbo, lbo, 128, 0);
-                    mma_i8(tmem + (uint32_t)(slot * kTcN), adesc, bdesc, idesc, 0);
-                    tc_commit(&sfull[slot]);
-                    if ((b & 3) == 3 || b == nb - 1) tc_commit(&wempty[s]);
                 }
-                __syncwarp();
             }
-            kcg += nkc;
+            __syncwarp();
         } else {
-            // ---- epilogue: thread = weight row, 16 activation rows per warp
+            // ---- epilogue
             const int q = warp & 3;            // tensor-memory lane quarter
             const int half = (warp - 2) >> 2;  // activation rows half*16 .. +16
             const int row = q * 32 + lane;     // tile row (lane of tensor memory)
-            int64_t grow;                      // weight row in the matrix
+            int64_t grow;
             bool row_ok;
             if (upgate) {
                 grow = row < 64 ? row0 + row : p.n_ff + row0 + (row - 64);
@@ -237,20 +324,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 grow = row0 + row;
                 row_ok = grow < p.rows;
             }
-            const uint16_t *drow = dws + (size_t)row * p.ld_d;
-            const bool active = half * 16 < npad;
-            if (c0 == 0) mbar_wait(dfull, 0, &g_err_tc);
+            const bool active = half * 16 < it.npad;
+            mbar_wait(&dfull[d], (int)((ii / 2) & 1), &g_err_tc);
+            const uint16_t *drow = dws(d) + (size_t)row * p.ld_d;
             float acc[16];
 #pragma unroll
             for (int t = 0; t < 16; ++t) acc[t] = 0.0f;
-            // blocks in groups of up to 4 (one K chunk): the MMA thread's
-            // commit on the group's last slot covers the group's earlier
-            // MMAs too, so one wait and one tensor-memory load round trip
-            // serve four blocks
-            for (int b = 0; b < nb; b += 4) {
-                const int gn = min(4, nb - b);
-                const int slot_last = (bg + gn - 1) % kTcSlots;
-                mbar_wait(&sfull[slot_last], ((bg + gn - 1) / kTcSlots) & 1, &g_err_tc);
+            int bb = bg;
+            for (int kc = 0; kc < nkc; ++kc) {
+                const int gg = g + kc, s = gg % p.stages;
+                const int gn = min(4, nb - kc * 4);
+                // the builders' scales of this stage (that phase is complete)
+                mbar_wait(&full[s], (gg / p.stages) & 1, &g_err_tc);
+                const float *dxs = reinterpret_cast<const float *>(ring + (size_t)s * kTcStage + kTcA + kTcB);
+                const int slot_last = (bb + gn - 1) % kTcSlots;
+                mbar_wait(&sfull[slot_last], ((bb + gn - 1) / kTcSlots) & 1, &g_err_tc);
                 tc_fence_after();
                 uint32_t v[4][16];
                 if (active) {
@@ -258,29 +346,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     for (int i = 0; i < 4; ++i)
                         if (i < gn)
                             tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) +
-                                          (uint32_t)(((bg + i) % kTcSlots) * kTcN + half * 16),
+                                          (uint32_t)(((bb + i) % kTcSlots) * kTcN + half * 16),
                                       v[i]);
                     tmem_ld_wait();
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
-                    for (int i = 0; i < gn; ++i) mbar_arrive(&sempty[(bg + i) % kTcSlots]);
+                    for (int i = 0; i < gn; ++i) mbar_arrive(&sempty[(bb + i) % kTcSlots]);
                 if (active) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         if (i < gn) {
-                            const float dw = row_ok ? scale_value(drow[b + i]) : 0.0f;
-                            const float *dxb = dxs + (half * 16) * nb + b + i;
+                            const float dw = row_ok ? scale_value(drow[kc * 4 + i]) : 0.0f;
 #pragma unroll
                             for (int t = 0; t < 16; ++t)
-                                acc[t] = fmaf(dw * dxb[t * nb], small_int_to_float((int)v[i][t]),
-                                              acc[t]);
+                                acc[t] = fmaf(dw * dxs[(half * 16 + t) * 4 + i],
+                                              small_int_to_float((int)v[i][t]), acc[t]);
                         }
                     }
                 }
-                bg += gn;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                bb += gn;
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&dempty[d]);
             // ---- outputs
             if (upgate) {
                 if (row >= 64 && active) {
@@ -292,20 +383,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
 #pragma unroll
                     for (int t = 0; t < 16; ++t) {
                         const int tl = half * 16 + t;
-                        if (tl < n) {
+                        if (tl < it.n) {
                             const float u = xchg[row * kTcN + tl];
-                            p.out[(int64_t)plist[c0 + tl] * p.n_ff + row0 + row] = tc_silu(acc[t]) * u;
+                            p.out[(int64_t)it.plist[it.c0 + tl] * p.n_ff + row0 + row] =
+                                tc_silu(acc[t]) * u;
                         }
                     }
                 }
+                named_bar_sync(2, kTcEpiWarps * 32);  // xchg is free for the next item
             } else if (row_ok && active) {
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     const int tl = half * 16 + t;
-                    if (tl < n) p.out[(int64_t)plist[c0 + tl] * p.rows + grow] = acc[t];
+                    if (tl < it.n) p.out[(int64_t)it.plist[it.c0 + tl] * p.rows + grow] = acc[t];
                 }
             }
         }
+        g += nkc;
+        bg += nb;
     }
     tc_fence_before();
     __syncthreads();
@@ -350,6 +445,8 @@ q8_status launch_tc(const q8_tensor *W, bool upgate, const int8_t *aq, const uin
     const int64_t P = n_tok * n_used;
     const int64_t max_big = std::min<int64_t>(W->n_mat, P / kTcMinPairs);
     if (max_big <= 0) return Q8_OK;  // no expert can reach the threshold
+    if (af && !aligned16(af))
+        Q8_FAIL(Q8_E_ALIGN, "tensor-core path: fp32 activations must be 16-byte aligned");
     PFN_cuTensorMapEncodeTiled_v12000 enc;
     q8_status st = encode_fn(&enc);
     if (st != Q8_OK) return st;
@@ -381,23 +478,20 @@ q8_status launch_tc(const q8_tensor *W, bool upgate, const int8_t *aq, const uin
     p.lay_offset = L.offset;
     p.lay_big = L.list_big;
     p.lay_pairs = L.pairs;
-    // shared memory: ring, activations, their scales, the gate/up exchange, barriers
-    const int nb = (int)(W->k / QK);
-    const int x_bytes = kTcN * (int)W->k;
-    const int dx_bytes = ((kTcN * nb * 4 + 127) / 128) * 128;
+    // shared memory: the ring (A, B and the activation scales per stage),
+    // two tile-scale buffers, the gate/up exchange, the barriers
     const int xchg_bytes = 64 * kTcN * 4;
-    const int dw_bytes = ((int)(128 * W->ld_d * 2) + 127) / 128 * 128;
-    const int bar_bytes = 2 * (8 + kTcSlots) * 8 + 32;
-    const int fixed = x_bytes + dx_bytes + xchg_bytes + dw_bytes + bar_bytes + 1024;
+    const int dws_bytes = ((int)(128 * W->ld_d * 2) + 127) / 128 * 128;
+    const int bar_bytes = ((2 * 8 + 2 * kTcSlots + 4) * 8 + 16 + 127) / 128 * 128;
+    const int fixed = 2 * dws_bytes + xchg_bytes + bar_bytes + 1024;
     int stages = (kSmemLimit - fixed) / kTcStage;
     if (stages > 8) stages = 8;
-    if (stages < 2) Q8_FAIL(Q8_E_UNSUPPORTED, "tensor-core path: k=%lld too large", (long long)W->k);
+    if (stages < 3) Q8_FAIL(Q8_E_UNSUPPORTED, "tensor-core path: k=%lld too large", (long long)W->k);
     p.stages = stages;
-    p.off_x = stages * kTcStage;
-    p.off_dx = p.off_x + x_bytes;
-    p.off_xchg = p.off_dx + dx_bytes;
-    p.off_dw = p.off_xchg + xchg_bytes;
-    p.off_bar = p.off_dw + dw_bytes;
+    p.dws_bytes = dws_bytes;
+    p.off_dws = stages * kTcStage;
+    p.off_xchg = p.off_dws + 2 * dws_bytes;
+    p.off_bar = p.off_xchg + xchg_bytes;
     const int smem = p.off_bar + bar_bytes + 1024;  // + alignment slack
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) Q8_FAIL(Q8_E_CUDA, "tensor-core path: no device");
@@ -408,9 +502,13 @@ q8_status launch_tc(const q8_tensor *W, bool upgate, const int8_t *aq, const uin
             Q8_FAIL(Q8_E_CUDA, "tensor-core path: shared-memory attribute: %s", cudaGetErrorString(e));
         set_smem_opted_in((const void *)tc_kernel, dev);
     }
-    const int tiles = upgate ? (int)(W->rows / 2 / 64) : (int)((W->rows + 127) / 128);
-    return launch_pdl("tc_kernel", tc_kernel, dim3((unsigned)tiles, (unsigned)max_big),
-                      dim3(kTcThreads), (size_t)smem, s, p);
+    // persistent: one CTA per SM (at most one per work item); each CTA finds
+    // its run of items from the grouping tables
+    const int64_t tiles = upgate ? W->rows / 2 / 64 : (W->rows + 127) / 128;
+    const int64_t max_items = tiles * max_big * ((P + kTcN - 1) / kTcN);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), max_items));
+    return launch_pdl("tc_kernel", tc_kernel, dim3((unsigned)grid), dim3(kTcThreads), (size_t)smem,
+                      s, p);
 }
 
 }  // namespace q8
