@@ -160,6 +160,11 @@ q8_status read_wait_errors_tc(int *flags);
 // rows: whether a weight view can take it, and the launch over the
 // tensor-core list of a grouping workspace.
 constexpr int kTcMinPairs = 16;
+// Dense calls (one matrix) with kTcMinDense..kTcMaxDense activation rows go
+// to the tensor cores too (one pass over the weights): launch_tc with
+// ws == nullptr.
+constexpr int kTcMinDense = 16;
+constexpr int kTcMaxDense = 32;
 bool tc_eligible(const q8_tensor *W, bool upgate);
 q8_status launch_tc(const q8_tensor *W, bool upgate, const int8_t *aq, const uint16_t *ad,
                     const float *af, int a_per_slot, int64_t n_tok, int32_t n_used, float *out,

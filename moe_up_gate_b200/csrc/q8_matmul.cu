@@ -334,6 +334,10 @@ q8_status launch_matmul_routed_ids(const q8_tensor *W, const int8_t *aq, const u
 // Dense matmul of fp32 (af) or Q8_0 (aq/ad) activation rows: y = W a.
 q8_status launch_matmul_dense(const q8_tensor *W, const int8_t *aq, const uint16_t *ad,
                               const float *af, int64_t n_tok, float *y, cudaStream_t s) {
+    // a real (small) dense contraction: the tensor cores, one pass over W
+    if (n_tok >= kTcMinDense && n_tok <= kTcMaxDense && tc_eligible(W, false) &&
+        (af == nullptr || aligned16(af)))
+        return launch_tc(W, false, aq, ad, af, 1, n_tok, 1, y, nullptr, s);
     const Geo g = geo_for_k((int)W->k, 8);
     const int64_t tiles = (W->rows + g.nr - 1) / g.nr;
     for (int64_t t0 = 0; t0 < n_tok; t0 += kMaxXRows) {

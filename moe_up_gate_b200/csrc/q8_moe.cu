@@ -453,7 +453,11 @@ static q8_status up_gate_entry(const char *fn, const q8_tensor *up_gate, const i
                    "%s: dense call (ids NULL) needs n_mat == 1, n_used == 1", fn);
         p.ws = nullptr;
         p.n_dense = (int)n_tok;
-        st = launch_up_gate(p, dense_rows(n_tok), 1, s);
+        if (n_tok >= kTcMinDense && n_tok <= kTcMaxDense && tc_eligible(up_gate, true) && !g_out &&
+            !u_out)
+            st = launch_tc(up_gate, true, xq, xd, nullptr, 1, n_tok, 1, h, nullptr, s);
+        else
+            st = launch_up_gate(p, dense_rows(n_tok), 1, s);
         if (st != Q8_OK || hq == nullptr) return st;
         // h -> Q8_0 with the activation quantizer (a 32-block of h spans
         // several weight tiles, so it is not formed inside one tile)
@@ -618,6 +622,9 @@ q8_status q8_moe_up_gate_swiglu_fp32(const q8_tensor *up_gate, const float *x, i
         Q8_REQUIRE(up_gate->n_mat == 1 && n_used == 1, Q8_E_SHAPE,
                    "%s: dense call (ids NULL) needs n_mat == 1, n_used == 1", fn);
         p.n_dense = (int)n_tok;
+        if (n_tok >= kTcMinDense && n_tok <= kTcMaxDense && tc_eligible(up_gate, true) &&
+            aligned16(x))
+            return launch_tc(up_gate, true, nullptr, nullptr, x, 1, n_tok, 1, h, nullptr, s);
         return launch_up_gate(p, dense_rows(n_tok), 1, s);
     }
     const GroupLayout L = group_layout(n_tok * n_used, up_gate->n_mat);

@@ -103,6 +103,27 @@ __device__ __forceinline__ void bulk_g2s_keep(void *dst, const void *src, uint32
         : "memory");
 }
 
+// Per-thread asynchronous copies global -> shared (the non-bulk form): the
+// thread continues at once; cp_async_commit closes a group of its copies and
+// cp_async_wait<N> returns when at most N of its groups are still in flight.
+// 16-byte copies: both addresses 16-byte aligned, L2 only; 4-byte copies:
+// both addresses 4-byte aligned.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
+                 "l"(__cvta_generic_to_global(src))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)),
+                 "l"(__cvta_generic_to_global(src))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Programmatic dependent launch: wait until the grids this one depends on
 // have completed and their memory is visible; allow dependents to launch.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

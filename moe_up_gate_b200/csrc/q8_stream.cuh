@@ -349,59 +349,66 @@ __device__ __forceinline__ void produce(const Ring &R, int64_t tb, int64_t te, S
 // recorded in tab[WS_ERR] and, by CTA 0, in *err_out (if given).  The
 // tensor-core list is not used here; its words serve as the scatter cursors.
 // ---------------------------------------------------------------------------
+// The grouping of at most 32 pairs by one warp (all its lanes), with no CTA
+// barrier: each lane is a pair, ranks come from shuffles.  Same tables as
+// cta_group.
+__device__ __forceinline__ void group_small_warp(const int32_t *__restrict__ ids, int n_tok,
+                                                 int n_used, int n_mat, const GroupLayout &L,
+                                                 int32_t *tab, int32_t *err_out) {
+    const int P = n_tok * n_used;
+    const int lane = threadIdx.x & 31;
+    const bool live = lane < P;
+    const int e = live ? ids[lane] : -1;
+    const bool valid = live && e >= 0 && e < n_mat;
+    int err = (live && !valid) ? ERR_ID_RANGE : 0;
+    const int tok0 = live ? (lane / n_used) * n_used : 0;
+    int rank = 0, cnt_e = 0, dpos = 0;
+    bool first = true;
+#pragma unroll
+    for (int s2 = 0; s2 < 32; ++s2) {
+        const int e2 = __shfl_sync(0xffffffffu, e, s2);
+        const bool v2 = __shfl_sync(0xffffffffu, valid ? 1 : 0, s2) != 0;
+        if (!valid || !v2) continue;
+        if (e2 < e || (e2 == e && s2 < lane)) ++rank;
+        if (e2 == e) {
+            ++cnt_e;
+            if (s2 < lane) {
+                first = false;
+                if (s2 >= tok0) err |= ERR_ID_REPEAT;
+            }
+        }
+    }
+    const unsigned firsts = __ballot_sync(0xffffffffu, valid && first);
+#pragma unroll
+    for (int s2 = 0; s2 < 32; ++s2) {
+        const int e2 = __shfl_sync(0xffffffffu, e, s2);
+        if (((firsts >> s2) & 1u) && e2 < e) ++dpos;
+    }
+    if (valid) tab[L.pairs + rank] = lane;
+    if (valid && first) {
+        tab[L.list_small + dpos] = e;
+        tab[L.count + e] = cnt_e;
+        tab[L.offset + e] = rank;
+    }
+    const unsigned vb = __ballot_sync(0xffffffffu, valid);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) err |= __shfl_xor_sync(0xffffffffu, err, o);
+    if (lane == 0) {
+        tab[WS_ERR] = err;
+        tab[WS_N_SMALL] = __popc(firsts);
+        tab[WS_N_BIG] = 0;
+        tab[WS_N_PAIRS] = P;
+        tab[L.offset + n_mat] = __popc(vb);
+        if (err_out && blockIdx.x == 0) *err_out = err;
+    }
+}
+
 __device__ __forceinline__ void cta_group(const int32_t *__restrict__ ids, int n_tok, int n_used,
                                           int n_mat, const GroupLayout &L, int32_t *tab,
                                           int32_t *err_out) {
     const int P = n_tok * n_used;
     if (P <= 32) {
-        // one warp, one load: each lane is a pair; ranks by shuffles
-        if (threadIdx.x < 32) {
-            const int lane = threadIdx.x;
-            const bool live = lane < P;
-            const int e = live ? ids[lane] : -1;
-            const bool valid = live && e >= 0 && e < n_mat;
-            int err = (live && !valid) ? ERR_ID_RANGE : 0;
-            const int tok0 = live ? (lane / n_used) * n_used : 0;
-            int rank = 0, cnt_e = 0, dpos = 0;
-            bool first = true;
-#pragma unroll
-            for (int s2 = 0; s2 < 32; ++s2) {
-                const int e2 = __shfl_sync(0xffffffffu, e, s2);
-                const bool v2 = __shfl_sync(0xffffffffu, valid ? 1 : 0, s2) != 0;
-                if (!valid || !v2) continue;
-                if (e2 < e || (e2 == e && s2 < lane)) ++rank;
-                if (e2 == e) {
-                    ++cnt_e;
-                    if (s2 < lane) {
-                        first = false;
-                        if (s2 >= tok0) err |= ERR_ID_REPEAT;
-                    }
-                }
-            }
-            const unsigned firsts = __ballot_sync(0xffffffffu, valid && first);
-#pragma unroll
-            for (int s2 = 0; s2 < 32; ++s2) {
-                const int e2 = __shfl_sync(0xffffffffu, e, s2);
-                if (((firsts >> s2) & 1u) && e2 < e) ++dpos;
-            }
-            if (valid) tab[L.pairs + rank] = lane;
-            if (valid && first) {
-                tab[L.list_small + dpos] = e;
-                tab[L.count + e] = cnt_e;
-                tab[L.offset + e] = rank;
-            }
-            const unsigned vb = __ballot_sync(0xffffffffu, valid);
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) err |= __shfl_xor_sync(0xffffffffu, err, o);
-            if (lane == 0) {
-                tab[WS_ERR] = err;
-                tab[WS_N_SMALL] = __popc(firsts);
-                tab[WS_N_BIG] = 0;
-                tab[WS_N_PAIRS] = P;
-                tab[L.offset + n_mat] = __popc(vb);
-                if (err_out && blockIdx.x == 0) *err_out = err;
-            }
-        }
+        if (threadIdx.x < 32) group_small_warp(ids, n_tok, n_used, n_mat, L, tab, err_out);
         __syncthreads();
         return;
     }

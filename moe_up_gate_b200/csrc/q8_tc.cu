@@ -7,12 +7,14 @@
 // A persistent grid (one CTA per SM) walks work items (expert, pass of up to
 // 32 of its rows, 128-row weight tile; up/gate tiles are 64 gate rows and the
 // 64 matching up rows) through one ring whose stages hold, per 128-byte K
-// chunk (4 Q8_0 blocks): the weight tile's chunk (2-D TMA, 128-byte swizzle),
-// the activation rows' chunk as Q8_0 in the canonical no-swizzle K-major
-// core-matrix layout (built by two warps from the rows the pair list names),
-// and those rows' block scales.  One tcgen05.mma.kind::i8 per Q8_0 block
-// (M=128, N=16/32, K=32) lands in its own tensor-memory slot, because each
-// block has its own pair of scales and the int32 sum cannot run across
+// chunk (4 Q8_0 blocks): the weight tile's chunk (2-D TMA, 128-byte swizzle)
+// and the activation rows' chunk as Q8_0 in the canonical no-swizzle K-major
+// core-matrix layout (gathered by two warps from the rows the pair list
+// names).  The MMAs' commit frees a stage; the rows' block scales go to a
+// ring of their own, freed by the epilogue.  One tcgen05.mma.kind::i8 per
+// Q8_0 block (M=128, N=16/32, K=32) lands in its own tensor-memory slot
+// (16 slots: the MMAs run up to four chunks ahead of the epilogue), because
+// each block has its own pair of scales and the int32 sum cannot run across
 // blocks; eight epilogue warps read the slots back, scale by d_w * d_x in
 // fp32 and accumulate in block order.  Every wait is bounded (q8_ptx.cuh);
 // tensor memory is freed before exit.
@@ -29,17 +31,21 @@
 namespace q8 {
 
 constexpr int kTcN = 32;            // activation rows per pass
-constexpr int kTcSlots = 8;         // tensor-memory slots of kTcN columns
-constexpr int kTcCols = 256;        // columns allocated
+constexpr int kTcSlots = 16;        // tensor-memory slots of kTcN columns
+constexpr int kTcCols = 512;        // columns allocated (all of them: one CTA per SM)
 constexpr int kTcA = 16384;         // A part of a stage: 128 rows x 128 bytes (128B swizzle)
 constexpr int kTcB = kTcN * 128;    // B part: kTcN rows x 128 bytes (core matrices)
-constexpr int kTcDx = kTcN * 4 * 4; // activation scales of the stage's 4 blocks
-constexpr int kTcStage = 21504;     // kTcA + kTcB + kTcDx rounded to 1024
+constexpr int kTcStage = 20480;     // kTcA + kTcB
+constexpr int kTcDxRing = 16;       // entries of the activation-scale ring, one per K chunk
+constexpr int kTcDx = kTcN * 4 * 4; // an entry: the chunk's 4 blocks' scales, fp32 [block][row]
+constexpr int kTcDh = kTcN * 4 * 2; // and the same as copied, fp16 [row][block]
+constexpr int kTcDxEntry = kTcDx + kTcDh;
+constexpr int kTcLag = 3;           // chunks a builder keeps in flight before it reports one
 constexpr int kTcEpiWarps = 8;
 constexpr int kTcBuildWarps = 2;
 constexpr int kTcThreads = (2 + kTcEpiWarps + kTcBuildWarps) * 32;  // 384
 constexpr int kTcMaxK = 4096;
-static_assert(kTcA + kTcB + kTcDx <= kTcStage && kTcStage % 1024 == 0, "stage layout");
+static_assert(kTcA + kTcB == kTcStage && kTcStage % 1024 == 0, "stage layout");
 
 static __device__ int g_err_tc;
 
@@ -64,8 +70,10 @@ struct TcParams {
     float *out;
     const int32_t *ws;
     int64_t lay_count, lay_offset, lay_big, lay_pairs;
+    int n_dense;  // > 0: one matrix, its rows the n_dense activation rows (ws unused)
+    int x_async;  // Q8_0 activations gathered by cp.async (aq 16-byte, ad 4-byte aligned, nb even)
     int stages;
-    int off_dws, off_xchg, off_bar;
+    int off_dx, off_dws, off_xchg, off_bar;
     int dws_bytes;  // one of the two tile-scale buffers
 };
 
@@ -80,20 +88,27 @@ __device__ __forceinline__ float tc_silu(float z) { return z / (1.0f + expf(-z))
 struct TcItem {
     int mi, pass, tile;     // position
     int e, cnt, c0, n, npad;
-    const int32_t *plist;
+    const int32_t *plist;   // nullptr: dense, row j is activation row j
+    __device__ __forceinline__ int pair(int j) const { return plist ? plist[j] : j; }
 };
 
 struct TcWalk {
     const TcParams *p;
     int n_big, n_tiles;
-    __device__ __forceinline__ int passes(int mi) const {
-        const int e = p->ws[p->lay_big + mi];
-        return (p->ws[p->lay_count + e] + kTcN - 1) / kTcN;
+    __device__ __forceinline__ int count(int mi) const {
+        return p->n_dense > 0 ? p->n_dense : p->ws[p->lay_count + p->ws[p->lay_big + mi]];
     }
+    __device__ __forceinline__ int passes(int mi) const { return (count(mi) + kTcN - 1) / kTcN; }
     __device__ __forceinline__ void fill(TcItem &it) const {
-        it.e = p->ws[p->lay_big + it.mi];
-        it.cnt = p->ws[p->lay_count + it.e];
-        it.plist = p->ws + p->lay_pairs + p->ws[p->lay_offset + it.e];
+        if (p->n_dense > 0) {
+            it.e = 0;
+            it.cnt = p->n_dense;
+            it.plist = nullptr;
+        } else {
+            it.e = p->ws[p->lay_big + it.mi];
+            it.cnt = p->ws[p->lay_count + it.e];
+            it.plist = p->ws + p->lay_pairs + p->ws[p->lay_offset + it.e];
+        }
         it.c0 = it.pass * kTcN;
         it.n = min(kTcN, it.cnt - it.c0);
         it.npad = (it.n + 15) / 16 * 16;
@@ -138,9 +153,9 @@ struct TcWalk {
 //                Q8_0 block into its own tensor-memory slot;
 //  warps 2-9     epilogue: thread = weight row, 16 activation rows per warp;
 //  warps 10-11   B builders: the chunk's activation rows (gathered through
-//                the pair list) as Q8_0 core matrices and their scales, into
-//                the same stage.
-// A stage is freed by the epilogue (it reads the stage's activation scales).
+//                the pair list) as Q8_0 core matrices into the same stage,
+//                their scales into the scale ring.
+// A stage is freed by the MMA issuer's commit, a scale entry by the epilogue.
 __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant__ TcParams p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // the 128-byte-swizzled stages need 1024-byte alignment
@@ -150,7 +165,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool upgate = p.n_ff > 0;
     const int k = p.k, nb = k / QK, nkc = (k + 127) / 128;
-    TcWalk W{&p, p.ws[WS_N_BIG], upgate ? p.n_ff / 64 : (p.rows + 127) / 128};
+    TcWalk W{&p, p.n_dense > 0 ? 1 : p.ws[WS_N_BIG], upgate ? p.n_ff / 64 : (p.rows + 127) / 128};
     // the item count, by one lane per warp (a scan of the expert list)
     int64_t total = 0;
     if (lane == 0) total = W.total();
@@ -166,7 +181,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
     uint64_t *sempty = sfull + kTcSlots;
     uint64_t *dfull = sempty + kTcSlots;
     uint64_t *dempty = dfull + 2;
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(dempty + 2);
+    uint64_t *xfull = dempty + 2;
+    uint64_t *xempty = xfull + kTcDxRing;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(xempty + kTcDxRing);
+    auto dx_entry = [&](int e) { return smem + p.off_dx + (size_t)e * kTcDxEntry; };
     auto dws = [&](int d) {
         return reinterpret_cast<uint16_t *>(smem + p.off_dws + (size_t)d * p.dws_bytes);
     };
@@ -174,7 +192,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full[s], 1 + kTcBuildWarps);
-            mbar_init(&empty[s], kTcEpiWarps);
+            mbar_init(&empty[s], 1);  // the MMA issuer's commit once the chunk's MMAs are done
+        }
+        for (int e = 0; e < kTcDxRing; ++e) {
+            mbar_init(&xfull[e], kTcBuildWarps);
+            mbar_init(&xempty[e], kTcEpiWarps);
         }
         for (int s = 0; s < kTcSlots; ++s) {
             mbar_init(&sfull[s], 1);
@@ -198,6 +220,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
     TcItem it = W.seek(i0);
     int g = 0;   // K chunks so far (ring position)
     int bg = 0;  // blocks so far (slot position)
+    // asynchronous builders: the chunks whose copies have been reported
+    int reported = 0;
+    // a builder thread's part of chunk pc has landed: convert its two fp16
+    // scales into the scale entry's fp32 [block][row] table, make the stage's
+    // shared-memory writes visible to the tensor cores, report the warp's part
+    auto report = [&](int pc) {
+        const int s = pc % p.stages, e = pc % kTcDxRing;
+        unsigned char *dxe = dx_entry(e);
+        const int j = (threadIdx.x - (2 + kTcEpiWarps) * 32) >> 1, h = threadIdx.x & 1;
+        const uint32_t two = *reinterpret_cast<const uint32_t *>(dxe + kTcDx + j * 8 + h * 4);
+        float *dxs = reinterpret_cast<float *>(dxe);
+        dxs[(2 * h) * kTcN + j] = scale_value((uint16_t)(two & 0xffffu));
+        dxs[(2 * h + 1) * kTcN + j] = scale_value((uint16_t)(two >> 16));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&full[s]);
+            mbar_arrive(&xfull[e]);
+        }
+    };
+    // a builder may write chunk gg once the MMAs of the stage's previous
+    // chunk are done and the epilogue has read the scale entry's previous chunk
+    auto builder_wait = [&](int gg) {
+        if (gg >= p.stages) mbar_wait(&empty[gg % p.stages], (gg / p.stages - 1) & 1, &g_err_tc);
+        if (gg >= kTcDxRing)
+            mbar_wait(&xempty[gg % kTcDxRing], (gg / kTcDxRing - 1) & 1, &g_err_tc);
+    };
     for (int64_t ii = 0; ii < i1 - i0; ++ii, W.next(it)) {
         const int d = (int)(ii & 1);
         const int row0 = it.tile * (upgate ? 64 : 128);
@@ -232,22 +281,58 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     }
                 }
             }
+        } else if (warp >= 2 + kTcEpiWarps && p.x_async) {
+            // ---- B builders, asynchronous (Q8_0 activations): thread (row j,
+            // blocks 2h and 2h+1 of every chunk) copies its two blocks as four
+            // 16-byte pieces straight into their core-matrix places and the
+            // two fp16 scales into the stage's staging; a chunk is reported
+            // kTcLag chunks later, once its copies have landed, so the gathers
+            // of several chunks are in flight at once
+            const int j = (threadIdx.x - (2 + kTcEpiWarps) * 32) >> 1, h = threadIdx.x & 1;
+            const int ngrp = it.npad / 8;
+            const int8_t *xrow = nullptr;
+            const uint16_t *dxrow = nullptr;
+            if (j < it.n) {
+                const int pr = it.pair(it.c0 + j);
+                const int64_t r = p.a_per_slot ? pr : pr / p.n_used;
+                xrow = p.aq + r * k;
+                dxrow = p.ad + r * nb;
+            }
+            for (int kc = 0; kc < nkc; ++kc) {
+                const int gg = g + kc, s = gg % p.stages;
+                builder_wait(gg);
+                unsigned char *bst = ring + (size_t)s * kTcStage + kTcA;
+                // nb is even, so both blocks of the pair are present or neither
+                if (xrow && 2 * h < nb - kc * 4) {
+#pragma unroll
+                    for (int c = 4 * h; c < 4 * h + 4; ++c)
+                        cp_async16(bst + (c * ngrp + (j >> 3)) * 128 + (j & 7) * 16,
+                                   xrow + kc * 128 + c * 16);
+                    cp_async4(dx_entry(gg % kTcDxRing) + kTcDx + j * 8 + h * 4, dxrow + kc * 4 + 2 * h);
+                }
+                cp_async_commit();
+                if (gg - reported >= kTcLag) {
+                    cp_async_wait<kTcLag>();
+                    report(reported++);
+                }
+            }
         } else if (warp >= 2 + kTcEpiWarps) {
-            // ---- B builders: thread per (row, block of the chunk)
+            // ---- B builders: thread per (row, block of the chunk); a
+            // thread owns items tid and tid + 64 of every chunk (npad * 4 <= 128)
             const int tid = threadIdx.x - (2 + kTcEpiWarps) * 32;
             const int ngrp = it.npad / 8;
             for (int kc = 0; kc < nkc; ++kc) {
                 const int gg = g + kc, s = gg % p.stages;
-                if (gg >= p.stages) mbar_wait(&empty[s], (gg / p.stages - 1) & 1, &g_err_tc);
+                builder_wait(gg);
                 unsigned char *bst = ring + (size_t)s * kTcStage + kTcA;
-                float *dxs = reinterpret_cast<float *>(bst + kTcB);
+                float *dxs = reinterpret_cast<float *>(dx_entry(gg % kTcDxRing));
                 for (int idx = tid; idx < it.npad * 4; idx += kTcBuildWarps * 32) {
                     const int j = idx >> 2, b4 = idx & 3;
                     const int kb = kc * 4 + b4;
                     uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
                     float dx = 0.0f;
                     if (j < it.n && kb < nb) {
-                        const int pr = it.plist[it.c0 + j];
+                        const int pr = it.pair(it.c0 + j);
                         const int64_t r = p.a_per_slot ? pr : pr / p.n_used;
                         if (p.af) {
                             const float4 *src =
@@ -277,11 +362,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     const int c = 2 * b4;
                     *reinterpret_cast<uint4 *>(bst + (c * ngrp + (j >> 3)) * 128 + (j & 7) * 16) = lo;
                     *reinterpret_cast<uint4 *>(bst + ((c + 1) * ngrp + (j >> 3)) * 128 + (j & 7) * 16) = hi;
-                    dxs[j * 4 + b4] = dx;
+                    dxs[b4 * kTcN + j] = dx;  // [block][row]: a row's 16 scales are contiguous
                 }
                 fence_proxy_async_smem();  // generic-proxy writes, read by the tensor cores
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&full[s]);
+                if (lane == 0) {
+                    mbar_arrive(&full[s]);
+                    mbar_arrive(&xfull[gg % kTcDxRing]);
+                }
             }
         } else if (warp == 1) {
             // ---- MMA issuer
@@ -307,6 +395,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                         mma_i8(tmem + (uint32_t)(slot * kTcN), adesc, bdesc, idesc, 0);
                         tc_commit(&sfull[slot]);
                     }
+                    tc_commit(&empty[s]);  // the stage is free once these MMAs are done
                 }
             }
             __syncwarp();
@@ -332,11 +421,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             for (int t = 0; t < 16; ++t) acc[t] = 0.0f;
             int bb = bg;
             for (int kc = 0; kc < nkc; ++kc) {
-                const int gg = g + kc, s = gg % p.stages;
+                const int gg = g + kc;
                 const int gn = min(4, nb - kc * 4);
-                // the builders' scales of this stage (that phase is complete)
-                mbar_wait(&full[s], (gg / p.stages) & 1, &g_err_tc);
-                const float *dxs = reinterpret_cast<const float *>(ring + (size_t)s * kTcStage + kTcA + kTcB);
+                const int e = gg % kTcDxRing;
+                mbar_wait(&xfull[e], (gg / kTcDxRing) & 1, &g_err_tc);
+                const float *dxs = reinterpret_cast<const float *>(dx_entry(e));
                 const int slot_last = (bb + gn - 1) % kTcSlots;
                 mbar_wait(&sfull[slot_last], ((bb + gn - 1) / kTcSlots) & 1, &g_err_tc);
                 tc_fence_after();
@@ -359,15 +448,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     for (int i = 0; i < 4; ++i) {
                         if (i < gn) {
                             const float dw = row_ok ? scale_value(drow[kc * 4 + i]) : 0.0f;
+                            // the block's 16 activation scales: four 16-byte loads
+                            const float4 *dx4 =
+                                reinterpret_cast<const float4 *>(dxs + i * kTcN + half * 16);
+                            float dx[16];
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4) {
+                                const float4 f = dx4[q4];
+                                dx[4 * q4] = f.x;
+                                dx[4 * q4 + 1] = f.y;
+                                dx[4 * q4 + 2] = f.z;
+                                dx[4 * q4 + 3] = f.w;
+                            }
 #pragma unroll
                             for (int t = 0; t < 16; ++t)
-                                acc[t] = fmaf(dw * dxs[(half * 16 + t) * 4 + i],
-                                              small_int_to_float((int)v[i][t]), acc[t]);
+                                acc[t] = fmaf(dw * dx[t], small_int_to_float((int)v[i][t]), acc[t]);
                         }
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
+                if (lane == 0) mbar_arrive(&xempty[e]);
                 bb += gn;
             }
             __syncwarp();
@@ -385,7 +485,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                         const int tl = half * 16 + t;
                         if (tl < it.n) {
                             const float u = xchg[row * kTcN + tl];
-                            p.out[(int64_t)it.plist[it.c0 + tl] * p.n_ff + row0 + row] =
+                            p.out[(int64_t)it.pair(it.c0 + tl) * p.n_ff + row0 + row] =
                                 tc_silu(acc[t]) * u;
                         }
                     }
@@ -395,13 +495,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     const int tl = half * 16 + t;
-                    if (tl < it.n) p.out[(int64_t)it.plist[it.c0 + tl] * p.rows + grow] = acc[t];
+                    if (tl < it.n) p.out[(int64_t)it.pair(it.c0 + tl) * p.rows + grow] = acc[t];
                 }
             }
         }
         g += nkc;
         bg += nb;
     }
+    if (warp >= 2 + kTcEpiWarps && p.x_async) {
+        cp_async_wait<0>();
+        while (reported < g) report(reported++);
+    }
+    // the last stage commit lands before the CTA's shared memory is released
+    if (warp == 1 && lane == 0)
+        mbar_wait(&empty[(g - 1) % p.stages], ((g - 1) / p.stages) & 1, &g_err_tc);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -443,7 +550,8 @@ q8_status launch_tc(const q8_tensor *W, bool upgate, const int8_t *aq, const uin
                     const float *af, int a_per_slot, int64_t n_tok, int32_t n_used, float *out,
                     const int32_t *ws, cudaStream_t s) {
     const int64_t P = n_tok * n_used;
-    const int64_t max_big = std::min<int64_t>(W->n_mat, P / kTcMinPairs);
+    const bool dense = ws == nullptr;  // one matrix; its rows are the n_tok activation rows
+    const int64_t max_big = dense ? 1 : std::min<int64_t>(W->n_mat, P / kTcMinPairs);
     if (max_big <= 0) return Q8_OK;  // no expert can reach the threshold
     if (af && !aligned16(af))
         Q8_FAIL(Q8_E_ALIGN, "tensor-core path: fp32 activations must be 16-byte aligned");
@@ -478,18 +586,25 @@ q8_status launch_tc(const q8_tensor *W, bool upgate, const int8_t *aq, const uin
     p.lay_offset = L.offset;
     p.lay_big = L.list_big;
     p.lay_pairs = L.pairs;
+    p.n_dense = dense ? (int)n_tok : 0;
+    // the gathers go by cp.async when their 16- and 4-byte pieces are aligned
+    p.x_async = !af && aq && ad && W->k % 64 == 0 && aligned16(aq) &&
+                (reinterpret_cast<uintptr_t>(ad) & 3u) == 0;
     // shared memory: the ring (A, B and the activation scales per stage),
     // two tile-scale buffers, the gate/up exchange, the barriers
     const int xchg_bytes = 64 * kTcN * 4;
     const int dws_bytes = ((int)(128 * W->ld_d * 2) + 127) / 128 * 128;
-    const int bar_bytes = ((2 * 8 + 2 * kTcSlots + 4) * 8 + 16 + 127) / 128 * 128;
-    const int fixed = 2 * dws_bytes + xchg_bytes + bar_bytes + 1024;
+    const int bar_bytes = ((2 * 8 + 2 * kTcSlots + 4 + 2 * kTcDxRing) * 8 + 16 + 127) / 128 * 128;
+    const int dx_bytes = kTcDxRing * kTcDxEntry;
+    const int fixed = dx_bytes + 2 * dws_bytes + xchg_bytes + bar_bytes + 1024;
     int stages = (kSmemLimit - fixed) / kTcStage;
     if (stages > 8) stages = 8;
     if (stages < 3) Q8_FAIL(Q8_E_UNSUPPORTED, "tensor-core path: k=%lld too large", (long long)W->k);
+    if (stages <= kTcLag) p.x_async = 0;  // a builder's lag must stay below the ring depth
     p.stages = stages;
     p.dws_bytes = dws_bytes;
-    p.off_dws = stages * kTcStage;
+    p.off_dx = stages * kTcStage;
+    p.off_dws = p.off_dx + dx_bytes;
     p.off_xchg = p.off_dws + 2 * dws_bytes;
     p.off_bar = p.off_xchg + xchg_bytes;
     const int smem = p.off_bar + bar_bytes + 1024;  // + alignment slack

@@ -84,6 +84,7 @@ def test_tc_up_gate(n_exp, n_ff, n_embd, n_tok, n_used, hot):
     (4, 200, 704, 40, 2, 4),      # a ragged last row tile, k with a half K chunk
     (3, 256, 2816, 50, 1, 3),
     (8, 128, 128, 72, 2, 2),
+    (4, 128, 224, 40, 2, 4),      # an odd block count: the gather by plain loads
 ])
 def test_tc_mul_mat_id(n_mat, rows, k, n_tok, n_used, hot):
     w = synth.normal((n_mat, rows, k), seed=801 + k, std=0.02)
@@ -177,3 +178,54 @@ def test_large_batch_ffn_step_sampled():
             e = sub_ids[0, s]
             S = S_norm(dnq[e], dnd[e], hq_t[s][None], hd_t[s][None])[0]
             assert_p3(host(y)[tok, s], yr[0, s], S, "down")
+
+
+@pytest.mark.parametrize("rows,k,n_tok", [(300, 704, 16), (128, 2816, 16), (77, 256, 32),
+                                          (256, 4096, 21), (130, 160, 19)])
+def test_tc_dense_gemv(rows, k, n_tok):
+    """Dense matmuls with 16..32 activation rows run on the tensor cores (one
+    pass over W): P3 against the oracle, every output written."""
+    w = synth.normal((rows, k), seed=811 + k + n_tok, std=0.02)
+    W = q8.pack(w.to(DEV))
+    a = synth.normal((n_tok, k), seed=812 + k)
+    aq, ad = q8.quantize_row(a.to(DEV))
+    y = torch.full((n_tok, rows), float("nan"), device=DEV)
+    q8.gemv(W, aq, ad, y=y)
+    wq, wd = host(W.qs), canon_d(W.d, k)
+    ref = oracle.gemv(wq, wd, host(aq), bits(ad))
+    assert not torch.isnan(y).any()
+    assert_p3(host(y), ref, S_norm(wq, wd, host(aq), bits(ad)), "tc dense gemv")
+
+
+@pytest.mark.parametrize("n_ff,n_embd,n_tok", [(128, 512, 16), (64, 2816, 24), (192, 1024, 32)])
+def test_tc_dense_up_gate(n_ff, n_embd, n_tok):
+    """Dense up/gate + SwiGLU with 16..32 rows on the tensor cores: h against
+    the oracle (the bound P3 on g and u implies), hq by the oracle's quantizer
+    (P5), and the fp32 entry point gives the same bits."""
+    shape = synth.MoeShape(n_embd=n_embd, n_ff=n_ff, n_exp=1, n_used=1)
+    t = synth.moe_layer_tensors(820 + n_tok, 0, shape, n_tok, 1.0)
+    UG = q8.pack(t["up_gate"].to(DEV))
+    x = t["x"].to(DEV)
+    xq, xd = q8.quantize_row(x)
+    r = q8.moe_up_gate_swiglu(UG, xq, xd, None, want_hq=True)
+    ids0 = torch.zeros((n_tok, 1), dtype=torch.int32)
+    _check_h(UG, xq, xd, ids0, r["h"])
+    rq, _ = oracle.quantize_rows(host(r["h"]).reshape(-1, n_ff))
+    assert np.array_equal(host(r["hq"]).reshape(-1, n_ff), rq)
+    h32 = q8.moe_up_gate_swiglu_fp32(UG, x, None)
+    assert torch.equal(h32, r["h"])
+
+
+def test_tc_dense_ffn_equals_chain():
+    """The dense feed-forward step at 16 tokens (both matmuls on the tensor
+    cores) equals quantize -> up/gate -> GEMV bitwise."""
+    shape = synth.MoeShape(n_embd=512, n_ff=256, n_exp=1, n_used=1)
+    t = synth.moe_layer_tensors(840, 0, shape, 16, 1.0)
+    UG = q8.pack(t["up_gate"].to(DEV))
+    DN = q8.pack(t["down"].to(DEV))
+    x = t["x"].to(DEV)
+    out = q8.moe_ffn(UG, DN, x)
+    xq, xd = q8.quantize_row(x)
+    r = q8.moe_up_gate_swiglu(UG, xq, xd, None, want_hq=True)
+    y = q8.gemv(DN, r["hq"].reshape(16, 256), r["hd"].reshape(16, 8))
+    assert torch.equal(out, y)
