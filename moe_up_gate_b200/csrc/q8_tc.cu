@@ -32,6 +32,7 @@ namespace q8 {
 
 constexpr int kTcN = 32;            // activation rows per pass
 constexpr int kTcSlots = 16;        // tensor-memory slots of kTcN columns
+constexpr int kTcGroups = kTcSlots / 4;  // slot groups: one K chunk's 4 blocks each
 constexpr int kTcCols = 512;        // columns allocated (all of them: one CTA per SM)
 constexpr int kTcA = 16384;         // A part of a stage: 128 rows x 128 bytes (128B swizzle)
 constexpr int kTcB = kTcN * 128;    // B part: kTcN rows x 128 bytes (core matrices)
@@ -178,8 +179,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.off_bar);
     uint64_t *empty = full + p.stages;
     uint64_t *sfull = empty + p.stages;
-    uint64_t *sempty = sfull + kTcSlots;
-    uint64_t *dfull = sempty + kTcSlots;
+    uint64_t *sempty = sfull + kTcGroups;
+    uint64_t *dfull = sempty + kTcGroups;
     uint64_t *dempty = dfull + 2;
     uint64_t *xfull = dempty + 2;
     uint64_t *xempty = xfull + kTcDxRing;
@@ -198,9 +199,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             mbar_init(&xfull[e], kTcBuildWarps);
             mbar_init(&xempty[e], kTcEpiWarps);
         }
-        for (int s = 0; s < kTcSlots; ++s) {
-            mbar_init(&sfull[s], 1);
-            mbar_init(&sempty[s], kTcEpiWarps);
+        for (int q4 = 0; q4 < kTcGroups; ++q4) {
+            mbar_init(&sfull[q4], 1);
+            mbar_init(&sempty[q4], kTcEpiWarps);
         }
         for (int d = 0; d < 2; ++d) {
             mbar_init(&dfull[d], 1);
@@ -219,7 +220,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
 
     TcItem it = W.seek(i0);
     int g = 0;   // K chunks so far (ring position)
-    int bg = 0;  // blocks so far (slot position)
     // asynchronous builders: the chunks whose copies have been reported
     int reported = 0;
     // a builder thread's part of chunk pc has landed: convert its two fp16
@@ -374,28 +374,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
         } else if (warp == 1) {
             // ---- MMA issuer
             if (lane == 0) {
+                // one thread issues everything, so the per-chunk work is kept
+                // small: one wait for the stage, one for the chunk's slot group,
+                // descriptors advanced by adds, two commits
                 const uint32_t idesc = idesc_i8(it.npad);
                 const uint32_t lbo = (uint32_t)(it.npad / 8) * 128;
-                int bb = bg;
+                const uint64_t bstep = (uint64_t)((2 * lbo) >> 4);  // next block: 2 core-matrix columns
                 for (int kc = 0; kc < nkc; ++kc) {
-                    const int gg = g + kc, s = gg % p.stages;
+                    const int gg = g + kc, s = gg % p.stages, grp = gg % kTcGroups;
                     mbar_wait(&full[s], (gg / p.stages) & 1, &g_err_tc);
+                    if (gg >= kTcGroups) mbar_wait(&sempty[grp], (gg / kTcGroups - 1) & 1, &g_err_tc);
                     tc_fence_after();
                     const uint32_t a_base = smem_u32(ring + (size_t)s * kTcStage);
-                    const uint32_t b_base = a_base + kTcA;
+                    uint64_t adesc = smem_desc(a_base, 16, 1024, 2);
+                    uint64_t bdesc = smem_desc(a_base + kTcA, lbo, 128, 0);
+                    uint32_t dt = tmem + (uint32_t)(grp * 4 * kTcN);
                     const int gn = min(4, nb - kc * 4);
-                    for (int b4 = 0; b4 < gn; ++b4, ++bb) {
-                        const int slot = bb % kTcSlots;
-                        if (bb >= kTcSlots) {
-                            mbar_wait(&sempty[slot], (bb / kTcSlots - 1) & 1, &g_err_tc);
-                            tc_fence_after();
-                        }
-                        const uint64_t adesc = smem_desc(a_base + b4 * 32, 16, 1024, 2);
-                        const uint64_t bdesc = smem_desc(b_base + (uint32_t)(2 * b4) * lbo, lbo, 128, 0);
-                        mma_i8(tmem + (uint32_t)(slot * kTcN), adesc, bdesc, idesc, 0);
-                        tc_commit(&sfull[slot]);
+                    for (int b4 = 0; b4 < gn; ++b4) {
+                        mma_i8(dt, adesc, bdesc, idesc, 0);
+                        adesc += 2;  // 32 bytes along K within the swizzled rows
+                        bdesc += bstep;
+                        dt += kTcN;
                     }
-                    tc_commit(&empty[s]);  // the stage is free once these MMAs are done
+                    tc_commit(&sfull[grp]);   // the chunk's slots hold its block sums
+                    tc_commit(&empty[s]);     // the stage is free once these MMAs are done
                 }
             }
             __syncwarp();
@@ -419,30 +421,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             float acc[16];
 #pragma unroll
             for (int t = 0; t < 16; ++t) acc[t] = 0.0f;
-            int bb = bg;
             for (int kc = 0; kc < nkc; ++kc) {
-                const int gg = g + kc;
+                const int gg = g + kc, grp = gg % kTcGroups;
                 const int gn = min(4, nb - kc * 4);
                 const int e = gg % kTcDxRing;
                 mbar_wait(&xfull[e], (gg / kTcDxRing) & 1, &g_err_tc);
                 const float *dxs = reinterpret_cast<const float *>(dx_entry(e));
-                const int slot_last = (bb + gn - 1) % kTcSlots;
-                mbar_wait(&sfull[slot_last], ((bb + gn - 1) / kTcSlots) & 1, &g_err_tc);
+                mbar_wait(&sfull[grp], (gg / kTcGroups) & 1, &g_err_tc);
                 tc_fence_after();
                 uint32_t v[4][16];
                 if (active) {
+                    const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) +
+                                        (uint32_t)(grp * 4 * kTcN + half * 16);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        if (i < gn)
-                            tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) +
-                                          (uint32_t)(((bb + i) % kTcSlots) * kTcN + half * 16),
-                                      v[i]);
+                        if (i < gn) tmem_ld16(ta + (uint32_t)(i * kTcN), v[i]);
                     tmem_ld_wait();
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0)
-                    for (int i = 0; i < gn; ++i) mbar_arrive(&sempty[(bb + i) % kTcSlots]);
+                if (lane == 0) mbar_arrive(&sempty[grp]);
                 if (active) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
@@ -468,7 +466,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&xempty[e]);
-                bb += gn;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&dempty[d]);
@@ -500,7 +497,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             }
         }
         g += nkc;
-        bg += nb;
     }
     if (warp >= 2 + kTcEpiWarps && p.x_async) {
         cp_async_wait<0>();
@@ -594,7 +590,7 @@ q8_status launch_tc(const q8_tensor *W, bool upgate, const int8_t *aq, const uin
     // two tile-scale buffers, the gate/up exchange, the barriers
     const int xchg_bytes = 64 * kTcN * 4;
     const int dws_bytes = ((int)(128 * W->ld_d * 2) + 127) / 128 * 128;
-    const int bar_bytes = ((2 * 8 + 2 * kTcSlots + 4 + 2 * kTcDxRing) * 8 + 16 + 127) / 128 * 128;
+    const int bar_bytes = ((2 * 8 + 2 * kTcGroups + 4 + 2 * kTcDxRing) * 8 + 16 + 127) / 128 * 128;
     const int dx_bytes = kTcDxRing * kTcDxEntry;
     const int fixed = dx_bytes + 2 * dws_bytes + xchg_bytes + bar_bytes + 1024;
     int stages = (kSmemLimit - fixed) / kTcStage;
