@@ -409,7 +409,10 @@ class MoeWorkload:
             self.launches_per_step = layers * (3 if self.routed else 2)
         elif self.routed:
             # quantize x, group, up/gate (dp4a + tensor cores), quantize h,
-            # down (dp4a + tensor cores), combine
+            # down (dp4a + tensor cores), combine; the timed unit is the
+            # up/gate step: tc_kernel for the experts with >= 16 rows and
+            # up_gate_kernel for the rest
+            self.kernel = "up_gate_step"
             self.launches_per_step = layers * 8
         else:
             self.launches_per_step = layers * 4
@@ -541,6 +544,7 @@ KERNEL_SOURCES = {
     "up_gate_kernel": ["q8_moe.cu"],
     "moe_layer_kernel": ["q8_layer.cu"],
     "tc_kernel": ["q8_tc.cu", "q8_tc.cuh"],
+    "up_gate_step": ["q8_moe.cu", "q8_tc.cu", "q8_tc.cuh"],
 }
 SHARED_SOURCES = ["q8_stream.cuh", "q8_device.cuh", "q8_ptx.cuh", "q8_internal.h"]
 

@@ -42,10 +42,13 @@ constexpr int kTcDx = kTcN * 4 * 4; // an entry: the chunk's 4 blocks' scales, f
 constexpr int kTcDh = kTcN * 4 * 2; // and the same as copied, fp16 [row][block]
 constexpr int kTcDxEntry = kTcDx + kTcDh;
 constexpr int kTcLag = 3;           // chunks a builder keeps in flight before it reports one
-constexpr int kTcEpiWarps = 8;
+constexpr int kTcEpiWarps = 16;
+constexpr int kTcCw = kTcN * 4 / kTcEpiWarps;  // activation rows (columns) per epilogue warp
 constexpr int kTcBuildWarps = 2;
-constexpr int kTcThreads = (2 + kTcEpiWarps + kTcBuildWarps) * 32;  // 384
+constexpr int kTcThreads = (2 + kTcEpiWarps + kTcBuildWarps) * 32;  // 640
+static_assert(kTcCw == 8 || kTcCw == 16, "epilogue split");
 constexpr int kTcMaxK = 4096;
+constexpr int kTcXs = kTcN + 1;     // gate/up exchange row stride (floats): rows land in distinct banks
 static_assert(kTcA + kTcB == kTcStage && kTcStage % 1024 == 0, "stage layout");
 
 static __device__ int g_err_tc;
@@ -83,6 +86,44 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 __device__ __forceinline__ float tc_silu(float z) { return z / (1.0f + expf(-z)); }
+
+// A warp's kTcCw columns of one slot (this thread's lane).
+__device__ __forceinline__ void tmem_ld_cols(uint32_t addr, uint32_t (&v)[16]) { tmem_ld16(addr, v); }
+__device__ __forceinline__ void tmem_ld_cols(uint32_t addr, uint32_t (&v)[8]) { tmem_ld8(addr, v); }
+
+// Pairs of fp32 in one 64-bit register pair, for the packed sm_100 forms of
+// add, mul and fma: each lane of the pair is rounded exactly as the scalar
+// instruction rounds it, at half the instruction count.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+// Two block sums |v| < 2^22 as fp32 (exact): the bits of 1.5 * 2^23 + v,
+// less 1.5 * 2^23.
+__device__ __forceinline__ uint64_t f2_from_ints(uint32_t a, uint32_t b) {
+    const float c = 12582912.0f;
+    return f2_add(f2_pack(__int_as_float((int)a + 0x4B400000), __int_as_float((int)b + 0x4B400000)),
+                  f2_pack(-c, -c));
+}
 
 // The CTA's work items, in order: (expert of the tensor-core list, pass of
 // kTcN of its rows, weight tile).  Every role walks the same sequence.
@@ -152,8 +193,8 @@ struct TcWalk {
 //                and the tile's weight scales by bulk copy (two buffers);
 //  warp 1        tensor-memory owner and MMA issuer: one kind::i8 MMA per
 //                Q8_0 block into its own tensor-memory slot;
-//  warps 2-9     epilogue: thread = weight row, 16 activation rows per warp;
-//  warps 10-11   B builders: the chunk's activation rows (gathered through
+//  warps 2-17    epilogue: thread = weight row, kTcCw activation rows per warp;
+//  warps 18-19   B builders: the chunk's activation rows (gathered through
 //                the pair list) as Q8_0 core matrices into the same stage,
 //                their scales into the scale ring.
 // A stage is freed by the MMA issuer's commit, a scale entry by the epilogue.
@@ -404,7 +445,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
         } else {
             // ---- epilogue
             const int q = warp & 3;            // tensor-memory lane quarter
-            const int half = (warp - 2) >> 2;  // activation rows half*16 .. +16
+            const int part = (warp - 2) >> 2;  // activation rows part*kTcCw .. +kTcCw
             const int row = q * 32 + lane;     // tile row (lane of tensor memory)
             int64_t grow;
             bool row_ok;
@@ -415,12 +456,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 grow = row0 + row;
                 row_ok = grow < p.rows;
             }
-            const bool active = half * 16 < it.npad;
+            const bool active = part * kTcCw < it.npad;
             mbar_wait(&dfull[d], (int)((ii / 2) & 1), &g_err_tc);
             const uint16_t *drow = dws(d) + (size_t)row * p.ld_d;
-            float acc[16];
+            uint64_t acc2[kTcCw / 2];  // activation rows (2t2, 2t2 + 1) of the warp's kTcCw
 #pragma unroll
-            for (int t = 0; t < 16; ++t) acc[t] = 0.0f;
+            for (int t2 = 0; t2 < kTcCw / 2; ++t2) acc2[t2] = 0ull;  // +0.0f in both lanes
             for (int kc = 0; kc < nkc; ++kc) {
                 const int gg = g + kc, grp = gg % kTcGroups;
                 const int gn = min(4, nb - kc * 4);
@@ -429,38 +470,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 const float *dxs = reinterpret_cast<const float *>(dx_entry(e));
                 mbar_wait(&sfull[grp], (gg / kTcGroups) & 1, &g_err_tc);
                 tc_fence_after();
-                uint32_t v[4][16];
+                uint32_t v[4][kTcCw];
                 if (active) {
                     const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) +
-                                        (uint32_t)(grp * 4 * kTcN + half * 16);
+                                        (uint32_t)(grp * 4 * kTcN + part * kTcCw);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        if (i < gn) tmem_ld16(ta + (uint32_t)(i * kTcN), v[i]);
+                    for (int i = 0; i < 4; ++i) {
+                        if (i < gn) tmem_ld_cols(ta + (uint32_t)(i * kTcN), v[i]);
+                    }
                     tmem_ld_wait();
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sempty[grp]);
                 if (active) {
+                    // the row's 4 weight scales of the chunk in one 8-byte load (ld_d is a
+                    // multiple of 8, so the 4 stay inside the row's padded scales)
+                    const uint2 dw4 = *reinterpret_cast<const uint2 *>(drow + kc * 4);
+                    const uint16_t dwh[4] = {(uint16_t)(dw4.x & 0xffffu), (uint16_t)(dw4.x >> 16),
+                                             (uint16_t)(dw4.y & 0xffffu), (uint16_t)(dw4.y >> 16)};
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         if (i < gn) {
-                            const float dw = row_ok ? scale_value(drow[kc * 4 + i]) : 0.0f;
-                            // the block's 16 activation scales: four 16-byte loads
+                            const float dw = row_ok ? scale_value(dwh[i]) : 0.0f;
+                            // the block's kTcCw activation scales: 16-byte loads
                             const float4 *dx4 =
-                                reinterpret_cast<const float4 *>(dxs + i * kTcN + half * 16);
-                            float dx[16];
+                                reinterpret_cast<const float4 *>(dxs + i * kTcN + part * kTcCw);
+                            const uint64_t dw2 = f2_pack(dw, dw);
+                            // acc[t] = fma(dw * dx[t], float(v[t]), acc[t]), two rows at a time
 #pragma unroll
-                            for (int q4 = 0; q4 < 4; ++q4) {
+                            for (int q4 = 0; q4 < kTcCw / 4; ++q4) {
                                 const float4 f = dx4[q4];
-                                dx[4 * q4] = f.x;
-                                dx[4 * q4 + 1] = f.y;
-                                dx[4 * q4 + 2] = f.z;
-                                dx[4 * q4 + 3] = f.w;
+                                const int t = 4 * q4;
+                                acc2[2 * q4] = f2_fma(f2_mul(dw2, f2_pack(f.x, f.y)),
+                                                      f2_from_ints(v[i][t], v[i][t + 1]), acc2[2 * q4]);
+                                acc2[2 * q4 + 1] =
+                                    f2_fma(f2_mul(dw2, f2_pack(f.z, f.w)),
+                                           f2_from_ints(v[i][t + 2], v[i][t + 3]), acc2[2 * q4 + 1]);
                             }
-#pragma unroll
-                            for (int t = 0; t < 16; ++t)
-                                acc[t] = fmaf(dw * dx[t], small_int_to_float((int)v[i][t]), acc[t]);
                         }
                     }
                 }
@@ -469,19 +516,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&dempty[d]);
+            float acc[kTcCw];
+#pragma unroll
+            for (int t2 = 0; t2 < kTcCw / 2; ++t2) f2_unpack(acc2[t2], acc[2 * t2], acc[2 * t2 + 1]);
             // ---- outputs
             if (upgate) {
                 if (row >= 64 && active) {
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) xchg[(row - 64) * kTcN + half * 16 + t] = acc[t];
+                    for (int t = 0; t < kTcCw; ++t) xchg[(row - 64) * kTcXs + part * kTcCw + t] = acc[t];
                 }
                 named_bar_sync(2, kTcEpiWarps * 32);
                 if (row < 64 && active) {
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) {
-                        const int tl = half * 16 + t;
+                    for (int t = 0; t < kTcCw; ++t) {
+                        const int tl = part * kTcCw + t;
                         if (tl < it.n) {
-                            const float u = xchg[row * kTcN + tl];
+                            const float u = xchg[row * kTcXs + tl];
                             p.out[(int64_t)it.pair(it.c0 + tl) * p.n_ff + row0 + row] =
                                 tc_silu(acc[t]) * u;
                         }
@@ -490,8 +540,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 named_bar_sync(2, kTcEpiWarps * 32);  // xchg is free for the next item
             } else if (row_ok && active) {
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const int tl = half * 16 + t;
+                for (int t = 0; t < kTcCw; ++t) {
+                    const int tl = part * kTcCw + t;
                     if (tl < it.n) p.out[(int64_t)it.pair(it.c0 + tl) * p.rows + grow] = acc[t];
                 }
             }
@@ -588,7 +638,7 @@ q8_status launch_tc(const q8_tensor *W, bool upgate, const int8_t *aq, const uin
                 (reinterpret_cast<uintptr_t>(ad) & 3u) == 0;
     // shared memory: the ring (A, B and the activation scales per stage),
     // two tile-scale buffers, the gate/up exchange, the barriers
-    const int xchg_bytes = 64 * kTcN * 4;
+    const int xchg_bytes = (64 * kTcXs * 4 + 127) / 128 * 128;
     const int dws_bytes = ((int)(128 * W->ld_d * 2) + 127) / 128 * 128;
     const int bar_bytes = ((2 * 8 + 2 * kTcGroups + 4 + 2 * kTcDxRing) * 8 + 16 + 127) / 128 * 128;
     const int dx_bytes = kTcDxRing * kTcDxEntry;
