@@ -37,10 +37,17 @@ constexpr int kTcCols = 512;        // columns allocated (all of them: one CTA p
 constexpr int kTcA = 16384;         // A part of a stage: 128 rows x 128 bytes (128B swizzle)
 constexpr int kTcB = kTcN * 128;    // B part: kTcN rows x 128 bytes (core matrices)
 constexpr int kTcStage = 20480;     // kTcA + kTcB
-constexpr int kTcDxRing = 16;       // entries of the activation-scale ring, one per K chunk
-constexpr int kTcDx = kTcN * 4 * 4; // an entry: the chunk's 4 blocks' scales, fp32 [block][row]
-constexpr int kTcDh = kTcN * 4 * 2; // and the same as copied, fp16 [row][block]
-constexpr int kTcDxEntry = kTcDx + kTcDh;
+constexpr int kTcDxRing = 8;        // entries of the activation-scale ring, one per K chunk
+constexpr int kTcDx = kTcN * 4 * 4; // an entry: the chunk's 4 blocks' scales d_x, fp32 [block][row]
+constexpr int kTcDm = kTcN * 4 * 4; // then -kTcMagic * d_x, fp32 [block][row]
+constexpr int kTcDh = kTcN * 4 * 2; // then d_x as copied, fp16 [row][block]
+constexpr int kTcDxEntry = kTcDx + kTcDm + kTcDh;
+// A block sum |v| < 2^22 becomes the fp32 kTcMagic + v by adding v to the
+// bits of kTcMagic.  kTcMagic * d_x is exact in fp32 (d_x is an fp16 value,
+// 11 significant bits), so fma(kTcMagic + v, d_x, -kTcMagic * d_x) is v * d_x
+// rounded once.
+constexpr float kTcMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr int kTcMagicBits = 0x4B400000;
 constexpr int kTcLag = 3;           // chunks a builder keeps in flight before it reports one
 constexpr int kTcEpiWarps = 16;
 constexpr int kTcCw = kTcN * 4 / kTcEpiWarps;  // activation rows (columns) per epilogue warp
@@ -91,9 +98,9 @@ __device__ __forceinline__ float tc_silu(float z) { return z / (1.0f + expf(-z))
 __device__ __forceinline__ void tmem_ld_cols(uint32_t addr, uint32_t (&v)[16]) { tmem_ld16(addr, v); }
 __device__ __forceinline__ void tmem_ld_cols(uint32_t addr, uint32_t (&v)[8]) { tmem_ld8(addr, v); }
 
-// Pairs of fp32 in one 64-bit register pair, for the packed sm_100 forms of
-// add, mul and fma: each lane of the pair is rounded exactly as the scalar
-// instruction rounds it, at half the instruction count.
+// Pairs of fp32 in one 64-bit register pair, for the packed sm_100 form of
+// fma: each lane of the pair is rounded exactly as the scalar instruction
+// rounds it, at half the instruction count.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
     uint64_t r;
     asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
@@ -102,27 +109,14 @@ __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
 __device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
 __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
     uint64_t r;
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
     return r;
 }
-// Two block sums |v| < 2^22 as fp32 (exact): the bits of 1.5 * 2^23 + v,
-// less 1.5 * 2^23.
-__device__ __forceinline__ uint64_t f2_from_ints(uint32_t a, uint32_t b) {
-    const float c = 12582912.0f;
-    return f2_add(f2_pack(__int_as_float((int)a + 0x4B400000), __int_as_float((int)b + 0x4B400000)),
-                  f2_pack(-c, -c));
+// Two block sums |v| < 2^22 as the fp32 values 1.5 * 2^23 + v (exact).
+__device__ __forceinline__ uint64_t f2_biased(uint32_t a, uint32_t b) {
+    return f2_pack(__int_as_float((int)a + kTcMagicBits), __int_as_float((int)b + kTcMagicBits));
 }
 
 // The CTA's work items, in order: (expert of the tensor-core list, pass of
@@ -270,10 +264,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
         const int s = pc % p.stages, e = pc % kTcDxRing;
         unsigned char *dxe = dx_entry(e);
         const int j = (threadIdx.x - (2 + kTcEpiWarps) * 32) >> 1, h = threadIdx.x & 1;
-        const uint32_t two = *reinterpret_cast<const uint32_t *>(dxe + kTcDx + j * 8 + h * 4);
+        const uint32_t two =
+            *reinterpret_cast<const uint32_t *>(dxe + kTcDx + kTcDm + j * 8 + h * 4);
         float *dxs = reinterpret_cast<float *>(dxe);
-        dxs[(2 * h) * kTcN + j] = scale_value((uint16_t)(two & 0xffffu));
-        dxs[(2 * h + 1) * kTcN + j] = scale_value((uint16_t)(two >> 16));
+        float *dms = reinterpret_cast<float *>(dxe + kTcDx);
+        const float d0 = scale_value((uint16_t)(two & 0xffffu)), d1 = scale_value((uint16_t)(two >> 16));
+        dxs[(2 * h) * kTcN + j] = d0;
+        dxs[(2 * h + 1) * kTcN + j] = d1;
+        dms[(2 * h) * kTcN + j] = -kTcMagic * d0;
+        dms[(2 * h + 1) * kTcN + j] = -kTcMagic * d1;
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -349,7 +348,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     for (int c = 4 * h; c < 4 * h + 4; ++c)
                         cp_async16(bst + (c * ngrp + (j >> 3)) * 128 + (j & 7) * 16,
                                    xrow + kc * 128 + c * 16);
-                    cp_async4(dx_entry(gg % kTcDxRing) + kTcDx + j * 8 + h * 4, dxrow + kc * 4 + 2 * h);
+                    cp_async4(dx_entry(gg % kTcDxRing) + kTcDx + kTcDm + j * 8 + h * 4,
+                              dxrow + kc * 4 + 2 * h);
                 }
                 cp_async_commit();
                 if (gg - reported >= kTcLag) {
@@ -403,7 +403,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     const int c = 2 * b4;
                     *reinterpret_cast<uint4 *>(bst + (c * ngrp + (j >> 3)) * 128 + (j & 7) * 16) = lo;
                     *reinterpret_cast<uint4 *>(bst + ((c + 1) * ngrp + (j >> 3)) * 128 + (j & 7) * 16) = hi;
-                    dxs[b4 * kTcN + j] = dx;  // [block][row]: a row's 16 scales are contiguous
+                    dxs[b4 * kTcN + j] = dx;  // [block][row]: a warp's rows are contiguous
+                    dxs[kTcN * 4 + b4 * kTcN + j] = -kTcMagic * dx;
                 }
                 fence_proxy_async_smem();  // generic-proxy writes, read by the tensor cores
                 __syncwarp();
@@ -493,20 +494,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     for (int i = 0; i < 4; ++i) {
                         if (i < gn) {
                             const float dw = row_ok ? scale_value(dwh[i]) : 0.0f;
-                            // the block's kTcCw activation scales: 16-byte loads
+                            // the block's kTcCw activation scales and their
+                            // -kTcMagic multiples: 16-byte loads
                             const float4 *dx4 =
                                 reinterpret_cast<const float4 *>(dxs + i * kTcN + part * kTcCw);
+                            const float4 *dm4 = reinterpret_cast<const float4 *>(
+                                dxs + kTcN * 4 + i * kTcN + part * kTcCw);
                             const uint64_t dw2 = f2_pack(dw, dw);
-                            // acc[t] = fma(dw * dx[t], float(v[t]), acc[t]), two rows at a time
+                            // acc[t] = fma(dw, round(v[t] * dx[t]), acc[t]), two rows at a time
 #pragma unroll
                             for (int q4 = 0; q4 < kTcCw / 4; ++q4) {
-                                const float4 f = dx4[q4];
+                                const float4 f = dx4[q4], m = dm4[q4];
                                 const int t = 4 * q4;
-                                acc2[2 * q4] = f2_fma(f2_mul(dw2, f2_pack(f.x, f.y)),
-                                                      f2_from_ints(v[i][t], v[i][t + 1]), acc2[2 * q4]);
-                                acc2[2 * q4 + 1] =
-                                    f2_fma(f2_mul(dw2, f2_pack(f.z, f.w)),
-                                           f2_from_ints(v[i][t + 2], v[i][t + 3]), acc2[2 * q4 + 1]);
+                                const uint64_t vd01 = f2_fma(f2_biased(v[i][t], v[i][t + 1]),
+                                                             f2_pack(f.x, f.y), f2_pack(m.x, m.y));
+                                const uint64_t vd23 = f2_fma(f2_biased(v[i][t + 2], v[i][t + 3]),
+                                                             f2_pack(f.z, f.w), f2_pack(m.z, m.w));
+                                acc2[2 * q4] = f2_fma(dw2, vd01, acc2[2 * q4]);
+                                acc2[2 * q4 + 1] = f2_fma(dw2, vd23, acc2[2 * q4 + 1]);
                             }
                         }
                     }
