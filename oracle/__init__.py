@@ -85,6 +85,9 @@ def lib():
                                             ctypes.c_void_p, i64, ctypes.c_void_p,
                                             ctypes.c_void_p, P(ctypes.c_double)]
         L.oracle_up_gate_swiglu.restype = ctypes.c_int
+        L.oracle_swiglu.argtypes = [P(ctypes.c_double), P(ctypes.c_double), i64,
+                                    P(ctypes.c_double)]
+        L.oracle_swiglu.restype = None
         L.oracle_mul_mat_id.argtypes = [P(ctypes.c_int8), P(ctypes.c_uint16), i64, i64, i64,
                                         P(ctypes.c_int8), P(ctypes.c_uint16), ctypes.c_int, i64,
                                         P(i32), i64, P(ctypes.c_double)]
@@ -263,6 +266,42 @@ def mul_mat_id(wq, wd, aq, ad, ids, a_per_slot: bool):
     if rc:
         raise ValueError("expert id out of range")
     return y
+
+
+def swiglu(g, u) -> np.ndarray:
+    """h = silu(g) * u elementwise in fp64 (the C oracle's silu)."""
+    g = _c(g, np.float64)
+    u = _c(u, np.float64)
+    assert g.shape == u.shape
+    h = np.empty_like(g)
+    lib().oracle_swiglu(_p(g, ctypes.c_double), _p(u, ctypes.c_double), g.size,
+                        _p(h, ctypes.c_double))
+    return h
+
+
+def up_gate_swiglu_split(gq, gd, uq, ud, xq, xd, ids=None, want_gu=False):
+    """The path with separate gate and up weights (page "GPUなしで13年前のXeon上で
+    Gemma 4 26Bを毎秒5トークンで実行する", section 「3段階で構成された修正」):
+    g = mul_mat_id(W_gate, x), u = mul_mat_id(W_up, x), h = silu(g) * u.
+
+    gate, up: [n_exp, n_ff, n_embd] Q8_0 each ([n_ff, n_embd] for a dense
+    layer); x [n_tok, n_embd] Q8_0; ids [n_tok, n_used] or None (dense: every
+    token uses matrix 0).  Returns h fp64 [n_tok, n_used, n_ff] (and g, u
+    when want_gu)."""
+    gq, gd, uq, ud = (_c(gq, np.int8), _c(gd, np.uint16), _c(uq, np.int8), _c(ud, np.uint16))
+    if gq.ndim == 2:
+        gq, gd, uq, ud = gq[None], gd[None], uq[None], ud[None]
+    assert gq.shape == uq.shape and gd.shape == ud.shape
+    n_embd = gq.shape[2]
+    xq = _c(xq, np.int8).reshape(-1, n_embd)
+    xd = _c(xd, np.uint16).reshape(xq.shape[0], -1)
+    n_tok = xq.shape[0]
+    ids = (np.zeros((n_tok, 1), np.int32) if ids is None
+           else _c(ids, np.int32).reshape(n_tok, -1))
+    g = mul_mat_id(gq, gd, xq, xd, ids, a_per_slot=False)
+    u = mul_mat_id(uq, ud, xq, xd, ids, a_per_slot=False)
+    h = swiglu(g, u)
+    return (h, g, u) if want_gu else h
 
 
 def combine(y, p) -> np.ndarray:

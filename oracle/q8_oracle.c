@@ -255,6 +255,17 @@ int oracle_up_gate_swiglu(const int8_t *wq, const uint16_t *wd, int64_t n_exp, i
     return bad ? -1 : 0;
 }
 
+/* The fused multiply-unary of the path with separate gate and up weights
+ * (page "GPUなしで13年前のXeon上でGemma 4 26Bを毎秒5トークンで実行する",
+ * section 「3段階で構成された修正」, runtime graph fallback): when the gate
+ * and up weights are already separate tensors, two mul_mat_id products g and
+ * u are joined by one SILU-and-multiply op.  h[i] = silu(g[i]) * u[i], fp64. */
+void oracle_swiglu(const double *g, const double *u, int64_t n, double *h)
+{
+    for (int64_t i = 0; i < n; ++i)
+        h[i] = oracle_silu(g[i]) * u[i];
+}
+
 /* ------------------------------------------------------------------------ */
 /* mul_mat_id: y[t][k] = W[ids[t][k]] . a(t, k)                              */
 /* ------------------------------------------------------------------------ */

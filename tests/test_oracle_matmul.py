@@ -15,6 +15,8 @@ What pins what:
   * mul_mat_id: routing selects exactly the named experts (marker expert test,
     perturbation of an unnamed expert leaves the output bitwise unchanged);
     per-pair numpy.
+  * split gate/up weights: bitwise the combined op on the concatenated rows,
+    g and u against numpy, gate/up not interchangeable, silu closed forms.
   * combine: numpy einsum.
   * invariants: dense op == one expert with every id 0; permuting tokens
     permutes outputs bitwise.
@@ -143,6 +145,48 @@ def test_up_gate_halves_split_exactly(orc):
     for t in range(n_tok):
         assert np.allclose(uc[t], xs[t], rtol=1e-12, atol=1e-12)
         assert np.allclose(hc[t], gc[t] / (1 + np.exp(-gc[t])) * xs[t], rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("n_exp,n_ff,n_embd,n_tok,n_used", [(4, 64, 96, 3, 2), (1, 32, 64, 5, 1)])
+def test_split_weights_path(orc, n_exp, n_ff, n_embd, n_tok, n_used):
+    """Separate gate and up tensors (two mul_mat_id, then silu(g) * u): bitwise
+    the combined-tensor op on their row concatenation; g and u against numpy;
+    gate and up not interchangeable; the dense form is expert 0 for every token."""
+    rng = np.random.default_rng(40 + n_exp)
+    gq, gd = _qrand(orc, rng, (n_exp, n_ff, n_embd), 0.02)
+    uq, ud = _qrand(orc, rng, (n_exp, n_ff, n_embd), 0.02)
+    xq, xd = _qrand(orc, rng, (n_tok, n_embd), 1.0)
+    ids = np.stack([rng.permutation(n_exp)[:n_used] for _ in range(n_tok)]).astype(np.int32)
+    h, g, u = orc.up_gate_swiglu_split(gq, gd, uq, ud, xq, xd, ids, want_gu=True)
+    ugq = np.concatenate([gq, uq], axis=1)
+    ugd = np.concatenate([gd, ud], axis=1)
+    hc, gc, uc = orc.up_gate_swiglu(ugq, ugd, xq, xd, ids, want_gu=True)
+    assert np.array_equal(h, hc) and np.array_equal(g, gc) and np.array_equal(u, uc)
+    xdq = _deq(xq, xd)
+    for t in range(n_tok):
+        for s in range(n_used):
+            e = ids[t, s]
+            Wg, Wu = _deq(gq[e], gd[e]), _deq(uq[e], ud[e])
+            gr, ur = Wg @ xdq[t], Wu @ xdq[t]
+            assert np.all(np.abs(g[t, s] - gr) <= 1e-12 * (np.abs(Wg) @ np.abs(xdq[t])))
+            assert np.all(np.abs(u[t, s] - ur) <= 1e-12 * (np.abs(Wu) @ np.abs(xdq[t])))
+            assert np.allclose(h[t, s], gr / (1.0 + np.exp(-gr)) * ur, rtol=1e-10, atol=1e-15)
+    assert not np.allclose(orc.up_gate_swiglu_split(uq, ud, gq, gd, xq, xd, ids), h)
+    if n_exp == 1:
+        assert np.array_equal(orc.up_gate_swiglu_split(gq[0], gd[0], uq[0], ud[0], xq, xd), h)
+
+
+def test_swiglu_elementwise(orc):
+    g = np.array([0.0, 1.0, -1.0, 30.0, -30.0, 2.5], np.float64)
+    u = np.array([3.0, 2.0, 2.0, 0.5, 4.0, -1.0], np.float64)
+    h = orc.swiglu(g, u)
+    assert h[0] == 0.0
+    assert abs(h[1] - 2.0 * 0.7310585786300049) < 1e-15      # silu(1) = 1 / (1 + e^-1)
+    assert abs(h[2] - 2.0 * -0.2689414213699951) < 1e-15     # silu(-1) = -1 / (1 + e)
+    # far tails: silu(30) = 30 / (1 + e^-30) ~ 30, silu(-30) = -30 / (1 + e^30) ~ -2.8e-12
+    assert abs(h[3] / (0.5 * 30.0 / (1.0 + np.exp(-30.0))) - 1.0) < 1e-15
+    assert abs(h[4] / (4.0 * -30.0 / (1.0 + np.exp(30.0))) - 1.0) < 1e-14
+    assert np.allclose(h, g / (1.0 + np.exp(-g)) * u, rtol=1e-15, atol=0)
 
 
 def test_dense_equals_single_expert(orc):
