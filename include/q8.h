@@ -35,6 +35,15 @@
  *    to another device or to the CPU, and no partial dispatch.
  *  - Results are deterministic: the same inputs give bitwise-equal outputs
  *    (no floating-point atomics; every sum has a fixed order).
+ *  - Accuracy: block dots are exact int32; every fp32 output of a matmul lies
+ *    within 1e-5 * sum|w * x| (the sum of the dequantized products' magnitudes)
+ *    of the exact value of its definition.  Which kernel runs depends on the
+ *    shape: experts with >= 16 routed rows in a call, and dense calls with
+ *    16..32 activation rows (k a multiple of 32 up to 4096), run on the int8
+ *    tensor cores (tcgen05.mma.kind::i8); the rest run on the dp4a streaming
+ *    kernels.  The two round their fp32 sums differently, so the same row can
+ *    differ in its last bits between a call where its expert crosses the
+ *    16-row line and one where it does not; both are within the bound.
  *  - Thread safety: calls may come from several host threads on different
  *    streams; the library holds no mutable global state except a per-thread
  *    detail string for the last error.
