@@ -41,7 +41,8 @@
  *    shape: experts with >= 16 routed rows in a call, and dense calls with
  *    16..32 activation rows, run on the int8 tensor cores
  *    (tcgen05.mma.kind::i8) when 128 <= k <= 4096 (and, for up/gate, n_ff is
- *    a multiple of 64); the rest run on the dp4a streaming kernels.  The two round their fp32 sums differently, so the same row can
+ *    a multiple of 64, and no g_out/u_out is asked for); the rest run on
+ *    the dp4a streaming kernels.  The two round their fp32 sums differently, so the same row can
  *    differ in its last bits between a call where its expert crosses the
  *    16-row line and one where it does not; both are within the bound.
  *  - Thread safety: calls may come from several host threads on different
