@@ -121,6 +121,24 @@ q8_status q8_pack(const float *w, int64_t n_rows, int64_t k, int8_t *qs, uint16_
                   int64_t ld_d, void *stream);
 
 /*
+ * q8_pack_up_gate -- pack separate gate and up weights into the combined
+ * up/gate layout (setup step).  [HADA] 「3段階で構成された修正」: when the gate
+ * and up weights are already separate tensors, the step is silu(W_gate x) *
+ * (W_up x); here they are packed once into the combined tensor, and the one
+ * fused up/gate kernel serves both forms.
+ *  w_gate, w_up: fp32 [n_mat][n_ff][k] each (n_mat == 1 for a dense layer);
+ *       16-byte aligned.
+ *  qs:  out int8 [n_mat][2*n_ff][k]: in each matrix, rows 0..n_ff-1 are the
+ *       gate rows and rows n_ff..2*n_ff-1 the up rows.
+ *  d:   out fp16 bits [n_mat][2*n_ff][ld_d], entries b >= k/32 written as 0.
+ *  ld_d: >= k/32, multiple of 8 (use q8_scale_stride(k)).
+ * The result equals q8_pack of the row concatenation [gate; up] of every
+ * matrix, bit for bit.  qs and d 16-byte aligned; n_ff % 32 == 0.
+ */
+q8_status q8_pack_up_gate(const float *w_gate, const float *w_up, int64_t n_mat, int64_t n_ff,
+                          int64_t k, int8_t *qs, uint16_t *d, int64_t ld_d, void *stream);
+
+/*
  * q8_quantize_row -- Q8_0 activation quantizer ([HADA] 「3段階で構成された修正」:
  * quantize_row_q8_0_x4; the plain one-row form).
  *  x:  fp32 [n_rows][k], 16-byte aligned.  k a multiple of 32, <= Q8_MAX_K.

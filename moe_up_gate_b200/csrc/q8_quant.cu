@@ -159,6 +159,40 @@ q8_status q8_pack(const float *w, int64_t n_rows, int64_t k, int8_t *qs, uint16_
     return launch_quantize(w, n_rows, k, qs, d, ld_d, s, true);
 }
 
+q8_status q8_pack_up_gate(const float *w_gate, const float *w_up, int64_t n_mat, int64_t n_ff,
+                          int64_t k, int8_t *qs, uint16_t *d, int64_t ld_d, void *stream) {
+    Q8_REQUIRE(w_gate && w_up && qs && d, Q8_E_NULL, "q8_pack_up_gate: NULL pointer");
+    Q8_REQUIRE(n_mat >= 1 && n_mat <= 65535, Q8_E_SHAPE, "q8_pack_up_gate: n_mat=%lld",
+               (long long)n_mat);
+    Q8_REQUIRE(n_ff >= QK && n_ff % QK == 0 && n_ff <= ((int64_t)1 << 29), Q8_E_SHAPE,
+               "q8_pack_up_gate: n_ff=%lld must be a positive multiple of 32", (long long)n_ff);
+    Q8_REQUIRE(k > 0 && k % QK == 0 && k <= Q8_MAX_K, Q8_E_SHAPE,
+               "q8_pack_up_gate: k=%lld must be a positive multiple of 32 <= %d", (long long)k,
+               Q8_MAX_K);
+    Q8_REQUIRE(ld_d >= k / QK && ld_d % 8 == 0, Q8_E_ALIGN,
+               "q8_pack_up_gate: ld_d=%lld must be >= k/32 and a multiple of 8", (long long)ld_d);
+    Q8_REQUIRE(aligned16(w_gate) && aligned16(w_up) && aligned16(qs) && aligned16(d), Q8_E_ALIGN,
+               "q8_pack_up_gate: w_gate, w_up, qs and d must be 16-byte aligned");
+    cudaStream_t s = (cudaStream_t)stream;
+    if (ld_d > k / QK) {
+        cudaError_t e =
+            cudaMemsetAsync(d, 0, (size_t)n_mat * 2 * n_ff * ld_d * sizeof(uint16_t), s);
+        if (e != cudaSuccess) Q8_FAIL(Q8_E_CUDA, "q8_pack_up_gate: memset: %s", cudaGetErrorString(e));
+    }
+    // each matrix: its gate rows to rows 0..n_ff-1, its up rows to n_ff..2*n_ff-1
+    // (offsets are multiples of k floats / k bytes / ld_d scales: 16-byte aligned)
+    for (int64_t m = 0; m < n_mat; ++m) {
+        const int64_t r0 = m * 2 * n_ff;
+        q8_status st = launch_quantize(w_gate + m * n_ff * k, n_ff, k, qs + r0 * k, d + r0 * ld_d,
+                                       ld_d, s, true);
+        if (st != Q8_OK) return st;
+        st = launch_quantize(w_up + m * n_ff * k, n_ff, k, qs + (r0 + n_ff) * k,
+                             d + (r0 + n_ff) * ld_d, ld_d, s, true);
+        if (st != Q8_OK) return st;
+    }
+    return Q8_OK;
+}
+
 const char *q8_status_string(q8_status st) {
     switch (st) {
         case Q8_OK: return "ok";

@@ -42,8 +42,8 @@ class _GemvDesc(ctypes.Structure):
     _fields_ = [("W", _Tensor), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p)]
 
 
-EXPORTS = ["q8_scale_stride", "q8_pack", "q8_quantize_row", "q8_gemv", "q8_gemv_batched",
-           "q8_moe_workspace_size", "q8_moe_up_gate_swiglu", "q8_mul_mat_id", "q8_moe_combine",
+EXPORTS = ["q8_scale_stride", "q8_pack", "q8_pack_up_gate", "q8_quantize_row", "q8_gemv",
+           "q8_gemv_batched", "q8_moe_workspace_size", "q8_moe_up_gate_swiglu", "q8_mul_mat_id", "q8_moe_combine",
            "q8_moe_ffn_workspace_size", "q8_moe_ffn", "q8_check", "q8_debug_block_dots",
            "q8_status_string", "q8_last_error", "q8_moe_group",
            "q8_moe_up_gate_swiglu_pregrouped", "q8_mul_mat_id_pregrouped",
@@ -72,6 +72,7 @@ def load(auto_build: bool = True):
         sig = {
             "q8_scale_stride": (i64, [i64]),
             "q8_pack": (st, [vp, i64, i64, vp, vp, i64, vp]),
+            "q8_pack_up_gate": (st, [vp, vp, i64, i64, i64, vp, vp, i64, vp]),
             "q8_quantize_row": (st, [vp, i64, i64, vp, vp, vp]),
             "q8_gemv": (st, [P(_Tensor), vp, vp, i64, vp, vp]),
             "q8_gemv_batched": (st, [P(_GemvDesc), i32, i64, vp]),
@@ -184,6 +185,26 @@ def pack(w: torch.Tensor, stream=None) -> Q8Tensor:
     d = torch.empty((n_mat * rows, ld), dtype=torch.float16, device=w.device)
     _call("q8_pack", _ptr(w), n_mat * rows, k, _ptr(qs), _ptr(d), ld, _stream(stream))
     return Q8Tensor(qs, d, k, rows, n_mat, ld, rows)
+
+
+def pack_up_gate(w_gate: torch.Tensor, w_up: torch.Tensor, stream=None) -> Q8Tensor:
+    """Separate fp32 gate and up weights, [n_ff, k] or [n_mat, n_ff, k] each (CUDA)
+    -> the combined packed up/gate tensor (gate rows first in every matrix)."""
+    assert w_gate.is_cuda and w_gate.dtype == torch.float32 and w_up.shape == w_gate.shape
+    assert w_up.is_cuda and w_up.dtype == torch.float32
+    w_gate, w_up = w_gate.contiguous(), w_up.contiguous()
+    if w_gate.dim() == 2:
+        n_mat, n_ff, k = 1, w_gate.shape[0], w_gate.shape[1]
+    else:
+        n_mat, n_ff, k = w_gate.shape
+    ld = scale_stride(k)
+    if ld == 0:
+        raise Q8Error(2, "pack_up_gate", f"k={k} must be a positive multiple of 32")
+    qs = torch.empty((n_mat * 2 * n_ff, k), dtype=torch.int8, device=w_gate.device)
+    d = torch.empty((n_mat * 2 * n_ff, ld), dtype=torch.float16, device=w_gate.device)
+    _call("q8_pack_up_gate", _ptr(w_gate), _ptr(w_up), n_mat, n_ff, k, _ptr(qs), _ptr(d), ld,
+          _stream(stream))
+    return Q8Tensor(qs, d, k, 2 * n_ff, n_mat, ld, 2 * n_ff)
 
 
 def quantize_row(x: torch.Tensor, stream=None):

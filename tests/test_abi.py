@@ -81,6 +81,17 @@ def test_pack_validation(q8):
     assert lib.q8_pack(FAKE, 4, 63, FAKE, FAKE, 8, None) == 2
 
 
+def test_pack_up_gate_validation(q8):
+    lib = q8.load()
+    assert lib.q8_pack_up_gate(FAKE, None, 2, 64, 64, FAKE, FAKE, 8, None) == 1       # NULL
+    assert lib.q8_pack_up_gate(FAKE, FAKE, 0, 64, 64, FAKE, FAKE, 8, None) == 2       # n_mat
+    assert lib.q8_pack_up_gate(FAKE, FAKE, 2, 48, 64, FAKE, FAKE, 8, None) == 2       # n_ff % 32
+    assert lib.q8_pack_up_gate(FAKE, FAKE, 2, 64, 63, FAKE, FAKE, 8, None) == 2       # k % 32
+    assert lib.q8_pack_up_gate(FAKE, FAKE, 2, 64, 64, FAKE, FAKE, 4, None) == 3       # ld_d % 8
+    assert lib.q8_pack_up_gate(FAKE_ODD, FAKE, 2, 64, 64, FAKE, FAKE, 8, None) == 3   # alignment
+    assert b"16-byte" in lib.q8_last_error()
+
+
 def test_gemv_validation(q8):
     lib = q8.load()
     W = _tensor(q8)

@@ -65,6 +65,35 @@ def test_up_gate_routed(n_exp, n_ff, n_embd, n_tok, n_used):
     _check_up_gate(UG, xq, xd, ids, r)
 
 
+@pytest.mark.parametrize("n_exp,n_ff,n_embd,n_tok,n_used", [(6, 64, 128, 5, 3), (1, 96, 256, 4, 1)])
+def test_separate_gate_up_weights(n_exp, n_ff, n_embd, n_tok, n_used):
+    """Separate gate and up weights packed by q8_pack_up_gate: bitwise the pack
+    of their row concatenation; the fused step on it passes P3-P5, and its
+    oracle value is the oracle's separate-weights path (two mul_mat_id, then
+    silu(g) * u) on the separately quantized halves."""
+    wg = synth.normal((n_exp, n_ff, n_embd), seed=500 + n_exp, std=0.02)
+    wu = synth.normal((n_exp, n_ff, n_embd), seed=600 + n_exp, std=0.02)
+    P = q8.pack_up_gate(wg.to(DEV), wu.to(DEV))
+    C = q8.pack(torch.cat([wg, wu], dim=1).to(DEV))
+    assert torch.equal(P.qs, C.qs)
+    assert torch.equal(P.d.view(torch.int16), C.d.view(torch.int16))
+    xq, xd = q8.quantize_row(synth.normal((n_tok, n_embd), seed=700 + n_tok).to(DEV))
+    if n_exp == 1:
+        ids = None
+    else:
+        ids = torch.stack([torch.randperm(n_exp, generator=torch.Generator().manual_seed(800 + t))
+                           [:n_used] for t in range(n_tok)]).to(torch.int32).to(DEV)
+    r = q8.moe_up_gate_swiglu(P, xq, xd, ids, want_hq=True, want_gu=True)
+    h_ref = _check_up_gate(P, xq, xd, ids, r)
+    gq, gd = oracle.quantize_rows(wg.numpy().reshape(-1, n_embd))
+    uq, ud = oracle.quantize_rows(wu.numpy().reshape(-1, n_embd))
+    sh_q, sh_d = (n_exp, n_ff, n_embd), (n_exp, n_ff, n_embd // 32)
+    h_split = oracle.up_gate_swiglu_split(gq.reshape(sh_q), gd.reshape(sh_d), uq.reshape(sh_q),
+                                          ud.reshape(sh_d), host(xq), bits(xd),
+                                          None if ids is None else host(ids))
+    assert np.array_equal(h_split, h_ref)
+
+
 @pytest.mark.parametrize("n_ff,n_embd,n_tok", [(64, 128, 1), (96, 256, 8), (32, 64, 11)])
 def test_up_gate_dense(n_ff, n_embd, n_tok):
     t, UG, DN, ids, p = _layer(1, n_ff, n_embd, n_tok, 1, seed=40 + n_tok)
