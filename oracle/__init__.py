@@ -5,9 +5,10 @@ TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
 product library (``moe_up_gate_b200``) never imports it, and this package never
 imports the product library: the two share no code.
 
-The arithmetic lives in ``q8_oracle.c`` (plain scalar C, fp64 sums, exact int32
-block dots).  This module only builds it with gcc, marshals numpy arrays into
-it through ctypes and returns numpy arrays.  Layouts are the canonical dense
+The Q8_0 arithmetic lives in ``q8_oracle.c`` (plain scalar C, fp64 sums, exact
+int32 block dots); this module builds it with gcc, marshals numpy arrays into
+it through ctypes and returns numpy arrays.  The router (``router_logits``,
+``route``), the step before the path, is plain numpy and Python here.  Layouts are the canonical dense
 ones: a Q8_0 tensor is ``qs`` int8 ``[..., rows, k]`` plus ``d`` uint16 (fp16
 bits) ``[..., rows, k // 32]``.
 
@@ -368,3 +369,39 @@ def moe_ffn(ugq, ugd, dnq, dnd, x, ids=None, p=None):
     if rc:
         raise ValueError("oracle_moe_ffn: bad id or quantization range")
     return dict(out=out, xq=xq, xd=xd, h=h, hf=hf, hq=hq, hd=hd, y=y)
+
+
+# --------------------------------------------------------------------------
+# Router (the step before the path: ids and routing weights from logits).
+# The pages name MoE routing only as a run-time option ("CPU-aware MoE
+# routing"); the reading here is the plain top-k router: fp32 router weights
+# (not quantized), logits in fp64, the n_used largest logits per token in
+# descending order with equal logits taken by ascending expert index, and the
+# routing weights a softmax over the selected logits only.  Plain numpy and
+# Python loops: test infrastructure for small cases.
+# --------------------------------------------------------------------------
+def router_logits(w_router, x) -> np.ndarray:
+    """w_router fp32 [n_exp, n_embd], x fp32 [n_tok, n_embd] -> logits fp64 [n_tok, n_exp]."""
+    w = np.asarray(w_router, dtype=np.float64)
+    xx = np.asarray(x, dtype=np.float64).reshape(-1, w.shape[1])
+    return xx @ w.T
+
+
+def route(logits, n_used: int):
+    """logits [n_tok, n_exp] -> (ids int32 [n_tok, n_used], p fp64 [n_tok, n_used]).
+
+    ids[t] lists the n_used experts with the largest logits, largest first;
+    equal logits go by ascending expert index.  p[t] = softmax of the selected
+    logits (the largest subtracted before exp)."""
+    lg = np.asarray(logits, dtype=np.float64)
+    n_tok, n_exp = lg.shape
+    assert 1 <= n_used <= n_exp
+    ids = np.empty((n_tok, n_used), np.int32)
+    p = np.empty((n_tok, n_used), np.float64)
+    for t in range(n_tok):
+        order = sorted(range(n_exp), key=lambda e: (-lg[t, e], e))[:n_used]
+        sel = lg[t, order]
+        ex = np.exp(sel - sel[0])
+        ids[t] = order
+        p[t] = ex / ex.sum()
+    return ids, p
