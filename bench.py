@@ -47,6 +47,8 @@ def parse():
                              "moe_30layer"])
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-subs", action="store_true",
+                    help="skip the MoE sub-records of the default run")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="bound on the CPU baseline sample")
     ap.add_argument("--min-seconds", type=float, default=1.0,
@@ -220,12 +222,12 @@ class LlamaDecode:
     name = "llama2_110m_q8_decode"
     kernel = "gemv_batched_kernel"
 
-    def __init__(self, dev, tokens=None, gemv768=False):
+    def __init__(self, dev, tokens=None, gemv768=False, host_only=False):
         import torch
 
-        from moe_up_gate_b200 import q8, synth
-        self.q8 = q8
+        from moe_up_gate_b200 import synth
         self.dev = dev
+        self.host_only = host_only
         if gemv768:
             self.name = "gemv_768"
             mats = [("w", 768, 768)]
@@ -243,16 +245,30 @@ class LlamaDecode:
         for _, rows, k in mats:
             offs.append(o)
             o += k
-        self.x_host = torch.empty(o, dtype=torch.float32).pin_memory()
+        self.x_host = torch.empty(o, dtype=torch.float32)
         for (_, rows, k), off, (ws, xs) in zip(mats, offs, seeds):
             self.x_host[off:off + k] = synth.normal((1, k), xs)[0]
-        self.x = self.x_host.to(dev)
-        self.y = [torch.empty((1, rows), dtype=torch.float32, device=dev) for _, rows, _ in mats]
-        self.out_host = torch.empty(mats[-1][1], dtype=torch.float32).pin_memory()
         self.w_fp32_seeds = seeds
+        self.offs = offs
+        self.weight_bytes = sum(q8_bytes(r, k) for _, r, k in mats)
         # L2 defeat: rotate through enough byte-identical weight copies
         self.copies = max(1, -(-3 * L2_BYTES // self.weight_bytes)) if self.weight_bytes > 4e6 else 1
         self.flush = self.weight_bytes < 4e6
+        self.config = {"workload": self.name, "matvecs": len(mats), "batch": 1,
+                       "weight_bytes_per_step": self.weight_bytes,
+                       "l2": ("flush 256 MiB between steps" if self.flush else
+                              f"{self.copies} rotating weight copies "
+                              f"({self.copies * self.weight_bytes / 2**20:.0f} MiB)")}
+        self.e2e_copies = ("every step: all matvec inputs host->device; the last matvec's "
+                           "output (the classifier logits) device->host")
+        if host_only:
+            return
+        from moe_up_gate_b200 import q8
+        self.q8 = q8
+        self.x_host = self.x_host.pin_memory()
+        self.x = self.x_host.to(dev)
+        self.y = [torch.empty((1, rows), dtype=torch.float32, device=dev) for _, rows, _ in mats]
+        self.out_host = torch.empty(mats[-1][1], dtype=torch.float32).pin_memory()
         packed = []
         for (_, rows, k), (ws, _) in zip(mats, seeds):
             w = synth.normal((rows, k), ws, std=synth.W_STD, device=dev)
@@ -262,7 +278,6 @@ class LlamaDecode:
         for c in range(1, self.copies):
             self.W.append([q8.Q8Tensor(P.qs.clone(), P.d.clone(), P.k, P.rows, P.n_mat, P.ld_d,
                                        P.mat_stride) for P in packed])
-        self.offs = offs
         self.sets = 1
         self.dominant_launches = 1
         self.tokens_per_step = 1
@@ -270,11 +285,6 @@ class LlamaDecode:
         self.dominant_bytes = self.weight_bytes
         self.h2d_bytes = self.x_host.numel() * 4
         self.d2h_bytes = self.out_host.numel() * 4
-        self.config = {"workload": self.name, "matvecs": len(mats), "batch": 1,
-                       "weight_bytes_per_step": self.weight_bytes,
-                       "l2": ("flush 256 MiB between steps" if self.flush else
-                              f"{self.copies} rotating weight copies "
-                              f"({self.copies * self.weight_bytes / 2**20:.0f} MiB)")}
 
     def issue(self, i, marks, input_set=None):
         W = self.W[i % self.copies]
@@ -286,13 +296,16 @@ class LlamaDecode:
     def unique_bytes(self, i):
         return self.weight_bytes
 
-    def e2e_pre(self):
+    def e2e_pre(self, i):
         self.x.copy_(self.x_host, non_blocking=True)
 
-    def e2e_post(self):
+    def e2e_post(self, i):
         self.out_host.copy_(self.y[-1][0], non_blocking=True)
 
-    # CPU oracle: one token of the same matvec set
+    # CPU oracle: one token of the same matvec set.  The weights are drawn
+    # with the same seeds on self.dev (on "cpu" for the host-only reference
+    # arm, where the values differ from a device draw but the recipe, shapes
+    # and sizes are the same).
     def oracle_setup(self):
         import oracle
         from moe_up_gate_b200 import synth
@@ -311,69 +324,116 @@ class LlamaDecode:
         return 1  # tokens
 
 
+ORACLE_TOKENS = 16
+
+
 class MoeWorkload:
     """MoE (or dense) feed-forward layers through the public calls:
     quantize x -> group -> fused up/gate + SwiGLU (+ h quantization) -> down
-    mul_mat_id -> combine (dense: quantize -> up/gate -> down GEMV)."""
+    mul_mat_id -> combine (dense: quantize -> up/gate -> down GEMV).
+
+    layer_ids: the layers to build (default all; a parity test builds a few
+    of them, with the same seeds and the same calls).  packed: the packed
+    layers of another workload of the same kind and layers (their weights
+    depend only on the layer's seed), reused instead of packing again.
+    host_only: only the shapes, inputs and oracle side (the reference arm)."""
     kernel = "up_gate_kernel"
 
-    def __init__(self, dev, kind, tokens):
+    def __init__(self, dev, kind, tokens, layer_ids=None, packed=None, host_only=False):
         import torch
 
-        from moe_up_gate_b200 import q8, synth
-        self.q8 = q8
+        from moe_up_gate_b200 import synth
         self.dev = dev
         if kind == "dense_ffn":
             shape, layers, c, x_std = synth.DENSE_FFN, 1, 3, 1.0
-            tokens = tokens or 1
         elif kind == "moe_layer":
             shape, layers, c, x_std = synth.MOE_LAYER, 1, 4, 1.0
-            tokens = tokens or 1
         else:
             shape, layers, c, x_std = synth.MOE_LAYER, synth.MOE_LAYERS, 5, synth.W_STD
-            tokens = tokens or 1
+        tokens = tokens or 1
+        self.layer_ids = list(range(layers)) if layer_ids is None else list(layer_ids)
         self.name = kind
-        self.shape, self.layers, self.T = shape, layers, tokens
+        self.c, self.x_std = c, x_std
+        self.shape, self.layers, self.T = shape, len(self.layer_ids), tokens
         self.routed = shape.n_exp > 1
         U = shape.n_used
         D, F, E = shape.n_embd, shape.n_ff, shape.n_exp
         self.expert_bytes = q8_bytes(2 * F, D) + q8_bytes(D, F)
         layer_bytes = E * self.expert_bytes
         # L2 defeat: enough layer copies that a step never re-reads from L2
-        per_step_max = layers * layer_bytes
+        per_step_max = self.layers * layer_bytes
         self.copies = 1 if per_step_max >= 3 * L2_BYTES else -(-3 * L2_BYTES // per_step_max)
-        self.sets = max(self.copies, 4 if self.routed else 1)  # rotating input sets
-        self.L = []
-        for l in range(layers):
-            t = synth.moe_layer_tensors(c, l, shape, tokens, x_std, device=dev)
-            UG = q8.pack(t["up_gate"])
-            DN = q8.pack(t["down"])
-            del t["up_gate"], t["down"]
-            self.L.append((UG, DN))
-        torch.cuda.synchronize()
-        self.Lc = [self.L]
-        for cc in range(1, self.copies):
-            self.Lc.append([tuple(q8.Q8Tensor(P.qs.clone(), P.d.clone(), P.k, P.rows, P.n_mat,
-                                              P.ld_d, P.mat_stride) for P in pair)
-                            for pair in self.L])
+        # rotating input sets: enough that the experts a set names were last
+        # read more than 3x L2 of other weights ago (expected unique experts
+        # of a step: E (1 - (1 - U/E)^T))
+        uniq = E * (1 - (1 - U / E) ** tokens) if self.routed else 1
+        self.sets = max(self.copies, 4 if self.routed else 1,
+                        min(32, math.ceil(3 * L2_BYTES / (self.layers * uniq * self.expert_bytes)))
+                        if self.routed else 1)
         # inputs per (set, layer)
         self.x_host, self.ids_host, self.p_host = [], [], []
         for s in range(self.sets):
             xs, ids, ps = [], [], []
-            for l in range(layers):
+            for l in self.layer_ids:
                 xs.append(synth.normal((tokens, D), synth.seed_of(c, l, 2) + 7919 * s, x_std))
                 if self.routed:
                     ids.append(synth.routing_ids(tokens, E, U, synth.seed_of(c, l, 3) + 7919 * s))
                     ps.append(synth.routing_weights(tokens, U, synth.seed_of(c, l, 4) + 7919 * s))
-            self.x_host.append(torch.stack(xs).pin_memory())
+            self.x_host.append(torch.stack(xs))
             if self.routed:
-                self.ids_host.append(torch.stack(ids).pin_memory())
-                self.p_host.append(torch.stack(ps).pin_memory())
+                self.ids_host.append(torch.stack(ids))
+                self.p_host.append(torch.stack(ps))
+        Uu = U if self.routed else 1
+        P = tokens * Uu
+        # algorithmic bytes: the experts each layer's ids actually name
+        self.step_bytes, self.up_gate_bytes = [], []
+        self.fused = self.routed and P <= 32 and D <= 4096 and F <= 2048
+        for s in range(self.sets):
+            tot, ug = 0, 0
+            for li in range(self.layers):
+                ne = len(set(self.ids_host[s][li].flatten().tolist())) if self.routed else 1
+                tot += ne * self.expert_bytes
+                ug += ne * q8_bytes(2 * F, D)
+            self.step_bytes.append(tot)
+            # bytes of one launch of the dominant kernel (a layer's up/gate, or
+            # the whole layer when it is fused)
+            self.up_gate_bytes.append((tot if self.fused else ug) / self.layers)
+        self.tokens_per_step = tokens
+        self.small = P <= 1024 and E <= 512
+        self.config = {"workload": kind, "tokens": tokens, "layers": self.layers, "n_embd": D,
+                       "n_ff": F, "n_experts": E, "n_used": Uu,
+                       "mean_weight_bytes_per_step": statistics.mean(self.step_bytes),
+                       "l2": (f"{self.copies} rotating weight copies, {self.sets} input sets"
+                              if self.copies > 1 else
+                              f"weights per step > 3x L2; {self.sets} input sets")}
+        self.e2e_copies = ("every step: x (and ids, routing weights) host->device; every "
+                           "layer's output device->host")
+        if host_only:
+            return
+        from moe_up_gate_b200 import q8
+        self.q8 = q8
+        if packed is not None:
+            self.L = packed
+        else:
+            self.L = []
+            for l in self.layer_ids:
+                t = synth.moe_layer_tensors(c, l, shape, 1, x_std, device=dev)
+                UG = q8.pack(t["up_gate"])
+                DN = q8.pack(t["down"])
+                del t
+                self.L.append((UG, DN))
+        torch.cuda.synchronize()
+        self.Lc = [self.L]
+        for cc in range(1, self.copies):
+            self.Lc.append([tuple(q8.Q8Tensor(P_.qs.clone(), P_.d.clone(), P_.k, P_.rows,
+                                              P_.n_mat, P_.ld_d, P_.mat_stride) for P_ in pair)
+                            for pair in self.L])
+        self.x_host = [xh.pin_memory() for xh in self.x_host]
+        self.ids_host = [ih.pin_memory() for ih in self.ids_host]
+        self.p_host = [ph.pin_memory() for ph in self.p_host]
         self.x = [xh.to(dev) for xh in self.x_host]
         self.ids = [ih.to(dev) for ih in self.ids_host]
         self.p = [ph.to(dev) for ph in self.p_host]
-        Uu = U if self.routed else 1
-        P = tokens * Uu
         self.ws = q8.moe_workspace(tokens, Uu, E, dev) if self.routed else None
         self.xq = torch.empty((tokens, D), dtype=torch.int8, device=dev)
         self.xd = torch.empty((tokens, D // 32), dtype=torch.float16, device=dev)
@@ -381,51 +441,29 @@ class MoeWorkload:
         self.hq = torch.empty((P, F), dtype=torch.int8, device=dev)
         self.hd = torch.empty((P, F // 32), dtype=torch.float16, device=dev)
         self.y = torch.empty((tokens, Uu, D), dtype=torch.float32, device=dev)
-        self.out = torch.empty((layers, tokens, D), dtype=torch.float32, device=dev)
-        self.out_host = torch.empty((layers, tokens, D), dtype=torch.float32).pin_memory()
-        # algorithmic bytes: the experts each layer's ids actually name
-        self.step_bytes, self.up_gate_bytes = [], []
-        for s in range(self.sets):
-            tot, ug = 0, 0
-            for l in range(layers):
-                ne = len(set(self.ids_host[s][l].flatten().tolist())) if self.routed else 1
-                tot += ne * self.expert_bytes
-                ug += ne * q8_bytes(2 * F, D)
-            self.step_bytes.append(tot)
-            # bytes of one launch of the dominant kernel (a layer's up/gate, or
-            # the whole layer when it is fused)
-            self.up_gate_bytes.append((tot if self.routed and P <= 32 and D <= 4096 and F <= 2048
-                                       else ug) / layers)
-        self.tokens_per_step = tokens
-        self.small = P <= 1024 and E <= 512
+        self.out = torch.empty((self.layers, tokens, D), dtype=torch.float32, device=dev)
+        self.out_host = torch.empty((self.layers, tokens, D), dtype=torch.float32).pin_memory()
         # routed batches of at most 32 pairs: q8_moe_ffn runs the whole layer
         # as one kernel (the dominant kernel is then the layer kernel)
-        self.fused = self.routed and P <= 32 and D <= 4096 and F <= 2048
         if self.fused:
             self.kernel = "moe_layer_kernel"
             self.ffn_ws = q8.moe_ffn_workspace(tokens, U, E, D, F, dev)
-            self.launches_per_step = layers
+            self.launches_per_step = self.layers
         elif self.small:
-            self.launches_per_step = layers * (3 if self.routed else 2)
+            self.launches_per_step = self.layers * (3 if self.routed else 2)
         elif self.routed:
             # quantize x, group, up/gate (dp4a + tensor cores), quantize h,
             # down (dp4a + tensor cores), combine; the timed unit is the
             # up/gate step: tc_kernel for the experts with >= 16 rows and
             # up_gate_kernel for the rest
             self.kernel = "up_gate_step"
-            self.launches_per_step = layers * 8
+            self.launches_per_step = self.layers * 8
         else:
-            self.launches_per_step = layers * 4
-        self.dominant_launches = layers
+            self.launches_per_step = self.layers * 4
+        self.dominant_launches = self.layers
         self.h2d_bytes = self.x_host[0].numel() * 4 + (
             (self.ids_host[0].numel() * 4 + self.p_host[0].numel() * 4) if self.routed else 0)
         self.d2h_bytes = self.out_host.numel() * 4
-        self.config = {"workload": kind, "tokens": tokens, "layers": layers, "n_embd": D,
-                       "n_ff": F, "n_experts": E, "n_used": Uu,
-                       "mean_weight_bytes_per_step": statistics.mean(self.step_bytes),
-                       "l2": (f"{self.copies} rotating weight copies, {self.sets} input sets"
-                              if self.copies > 1 else
-                              f"weights per step > 3x L2; {self.sets} input sets")}
 
     def issue(self, i, marks, input_set=None):
         q8 = self.q8
@@ -486,41 +524,45 @@ class MoeWorkload:
     def dominant_bytes_at(self, i):
         return self.up_gate_bytes[i % self.sets]
 
-    def e2e_pre(self):
-        self.x[0].copy_(self.x_host[0], non_blocking=True)
+    def e2e_pre(self, i):
+        s = i % self.sets
+        self.x[s].copy_(self.x_host[s], non_blocking=True)
         if self.routed:
-            self.ids[0].copy_(self.ids_host[0], non_blocking=True)
-            self.p[0].copy_(self.p_host[0], non_blocking=True)
+            self.ids[s].copy_(self.ids_host[s], non_blocking=True)
+            self.p[s].copy_(self.p_host[s], non_blocking=True)
 
-    def e2e_post(self):
+    def e2e_post(self, i):
         self.out_host.copy_(self.out, non_blocking=True)
 
     def oracle_setup(self):
         import oracle
         from moe_up_gate_b200 import synth
-        # one layer through the oracle (its own quantization of the fp32 weights)
-        c = {"dense_ffn": 3, "moe_layer": 4, "moe_30layer": 5}[self.name]
-        x_std = synth.W_STD if self.name == "moe_30layer" else 1.0
-        t = synth.moe_layer_tensors(c, 0, self.shape, self.T, x_std, device=self.dev)
+        # one layer through the oracle (its own quantization of the fp32
+        # weights, drawn with the layer's seeds on self.dev)
+        l0 = self.layer_ids[0]
+        t = synth.moe_layer_tensors(self.c, l0, self.shape, 1, self.x_std, device=self.dev)
         self.o_ug = oracle.quantize_rows(t["up_gate"].cpu().numpy())
         self.o_dn = oracle.quantize_rows(t["down"].cpu().numpy())
-        self.o_x = self.x_host[0][0].numpy()
-        self.o_ids = self.ids_host[0][0].numpy() if self.routed else None
-        self.o_p = self.p_host[0][0].numpy() if self.routed else None
+        # a bounded sample: at most ORACLE_TOKENS of the step's tokens per
+        # oracle step (the oracle's time grows with the tokens)
+        self.o_tok = min(self.T, ORACLE_TOKENS)
+        self.o_x = self.x_host[0][0][:self.o_tok].numpy()
+        self.o_ids = self.ids_host[0][0][:self.o_tok].numpy() if self.routed else None
+        self.o_p = self.p_host[0][0][:self.o_tok].numpy() if self.routed else None
 
     def oracle_step(self):
         import oracle
         oracle.moe_ffn(self.o_ug[0], self.o_ug[1], self.o_dn[0], self.o_dn[1], self.o_x,
                        self.o_ids, self.o_p)
-        return self.T / self.layers  # one layer of a layers-deep step
+        return self.o_tok / self.layers  # one layer of a layers-deep step
 
 
-def make_workload(args, dev):
-    if args.workload == "llama2_110m_q8_decode":
-        return LlamaDecode(dev)
-    if args.workload == "gemv_768":
-        return LlamaDecode(dev, gemv768=True)
-    return MoeWorkload(dev, args.workload, args.tokens)
+def make_workload(workload, tokens, dev, host_only=False, packed=None):
+    if workload == "llama2_110m_q8_decode":
+        return LlamaDecode(dev, host_only=host_only)
+    if workload == "gemv_768":
+        return LlamaDecode(dev, gemv768=True, host_only=host_only)
+    return MoeWorkload(dev, workload, tokens, packed=packed, host_only=host_only)
 
 
 # ---------------------------------------------------------------------------
@@ -606,17 +648,13 @@ def time_oracle(wl, seconds, steps=None):
 
 # ---------------------------------------------------------------------------
 def run_reference(args, dist):
-    """The reference arm: the CPU oracle, as it stands, on the host cores."""
+    """The reference arm: the CPU oracle, as it stands, on the host cores.
+    Host only: the inputs are drawn on the CPU with the workload's seeds, and
+    nothing of the CUDA library is loaded."""
     if dist.rank != 0:
         return
-    import torch
-    dev = "cuda:0" if torch.cuda.is_available() else "cpu"
-    wl = make_workload(args, dev) if dev != "cpu" else None
-    if wl is None:
-        print(json.dumps({"impl": "reference", "unavailable": "needs a CUDA device to draw the "
-                          "same synthetic inputs"}))
-        return
     import oracle
+    wl = make_workload(args.workload, args.tokens, "cpu", host_only=True)
     wl.oracle_setup()
     for _ in range(args.warmup):
         wl.oracle_step()
@@ -626,20 +664,182 @@ def run_reference(args, dist):
         toks += wl.oracle_step()
     el = time.perf_counter() - t0
     v = toks / el
-    sample = (f"{args.steps} steps of one {wl.name} token through the scalar C oracle"
+    sample = (f"{args.steps} steps of one {wl.name} token through the scalar C oracle "
+              f"(inputs drawn on the CPU with the workload's seeds)"
               if isinstance(wl, LlamaDecode) else
-              f"{args.steps} x one layer of {wl.name} (T={wl.T}) through the scalar C oracle, "
-              f"counted as 1/{wl.layers} of a step")
-    out = {"metric": "Q8_0 decode tokens/s", "value": v, "unit": "tokens/s", "impl": "reference",
+              f"{args.steps} x one layer of {wl.name} (T={wl.T}; the first {wl.o_tok} tokens) "
+              f"through the scalar C oracle, counted as 1/{wl.layers} of a step (inputs drawn "
+              f"on the CPU with the workload's seeds)")
+    out = {"metric": METRIC, "value": v, "unit": "tokens/s", "impl": "reference",
            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "int8 x int8 -> int32, fp64 sums", "data": "synthetic",
-           "config": wl.config,
+           "vs_baseline": None, "dtype": "int8 x int8 -> int32, fp64 sums",
+           "data": DATA, "config": dict(wl.config, parallelism=f"replicas x{dist.world}"),
            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.max_threads(),
                             "kind": "oracle", "sample": sample},
            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out))
+
+
+METRIC = "Q8_0 decode tokens/s"
+DATA = "synthetic (seeded N(0, 0.02) weights quantized to Q8_0, N(0,1) inputs)"
+
+# The default run reports, beside the headline decode step, the fused MoE
+# feed-forward step on these workloads (one sub-record each).
+SUB_WORKLOADS = [("moe_layer", 1), ("moe_30layer", 1), ("moe_30layer", 256)]
+
+
+def measure(wl, args, dist, stream, cpu_seconds):
+    """Time K steps of workload wl (device events), its dominant kernel
+    (in-graph event marks), the end-to-end rate through host buffers and the
+    oracle on the host cores.  Returns the record (without the shared keys)."""
+    import torch
+    K, W = args.steps, max(args.warmup, 3)
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=wl.dev) \
+        if getattr(wl, "flush", False) else None
+
+    # one CUDA graph per step index, without timing marks (the step rate), and
+    # one per timed step with event marks around the dominant launches (the
+    # kernel time); the marks are kept out of the step-rate graphs
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        wl.issue(0, NoMarks())  # eager warm-up (sets kernel attributes)
+    torch.cuda.synchronize()
+
+    def capture(i, m, input_set=None):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            wl.issue(i, m, input_set)
+        return g
+
+    graphs = [capture(i, NoMarks()) for i in range(W + K)]
+    marks = [Marks(wl.dominant_launches) for _ in range(K)]
+    mgraphs = [capture(W + i, marks[i]) for i in range(K)]
+    torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            if flush is not None:
+                flush.zero_()
+            graphs[i].replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_id(dist.local))
+    clocks.start()
+    time.sleep(0.5)  # let the sampler start before the timed work
+
+    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    st_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    en_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+
+    def timed_steps(step):
+        """K steps, bracketed by a barrier + synchronize on both sides; ms of
+        device time, max over ranks.  Timed by one pair of events around the K
+        steps, or, when an L2 flush runs between steps, by a pair around each
+        step (the flush stays outside the timed intervals)."""
+        torch.cuda.synchronize()
+        dist.barrier()
+        with torch.cuda.stream(stream):
+            if flush is None:
+                ev[0].record(stream)
+                for i in range(K):
+                    step(i)
+                ev[1].record(stream)
+            else:
+                for i in range(K):
+                    flush.zero_()
+                    st_ev[i].record(stream)
+                    step(i)
+                    en_ev[i].record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        ms = (ev[0].elapsed_time(ev[1]) if flush is None else
+              sum(a.elapsed_time(b) for a, b in zip(st_ev, en_ev)))
+        return dist.max(ms)
+
+    def one_round():
+        return timed_steps(lambda i: graphs[W + i].replay())
+
+    torch.cuda.nvtx.range_push("timed")
+    first_ms = one_round()
+    rounds = int(min(1000, max(3, math.ceil(args.min_seconds * 1e3 / max(first_ms, 1e-3)))))
+    round_ms = [first_ms] + [one_round() for _ in range(rounds - 1)]
+    torch.cuda.nvtx.range_pop()
+    # the dominant kernel: the same steps with the in-graph marks
+    dom_ms = []
+    for _ in range(max(3, min(rounds, 50))):
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for i in range(K):
+                if flush is not None:
+                    flush.zero_()
+                mgraphs[i].replay()
+        torch.cuda.synchronize()
+        for m in marks:
+            dom_ms.extend(m.ms())
+    clk = clocks.stop()
+    total_ms = statistics.median(round_ms)
+
+    # end to end through the public API with host buffers: every step copies
+    # its inputs from pinned host memory, runs the step (graphs of the same
+    # public calls, on the same rotation of weight copies and input sets, with
+    # the same L2 flush) and copies its result back
+    n_e2e = max(wl.copies, wl.sets)
+    e2e_graphs = [capture(c, NoMarks(), c % wl.sets) for c in range(n_e2e)]
+
+    def e2e_step(i):
+        wl.e2e_pre(i)
+        e2e_graphs[i % n_e2e].replay()
+        wl.e2e_post(i)
+
+    e2e_ms = timed_steps(e2e_step)
+    e2e_rate, _ = job_rate(dist, wl.tokens_per_step * K, e2e_ms)
+
+    n = dist.world
+    value, total_ms = job_rate(dist, wl.tokens_per_step * K, total_ms)
+    step_bytes = statistics.mean(wl.unique_bytes(W + i) for i in range(K))
+    peak, peak_kind = measured_peak()
+    if isinstance(wl, LlamaDecode):
+        dom_bytes = wl.dominant_bytes
+    else:
+        dom_bytes = statistics.mean(wl.dominant_bytes_at(W + i) for i in range(K))
+    dom_avg_ms = statistics.mean(dom_ms) if dom_ms else None
+    achieved = dom_bytes / (dom_avg_ms / 1e3) / 1e9 if dom_avg_ms else None
+    traffic = recorded_traffic(wl.name + (f"_t{wl.T}" if hasattr(wl, "T") else ""), wl.kernel)
+    out = {
+        "value": value, "unit": "tokens/s", "ms_per_step": total_ms / K,
+        "config": dict(wl.config, parallelism=f"replicas x{n}"),
+        "timing": {"rounds": len(round_ms),
+                   "round_ms_min_median_max": [min(round_ms), total_ms, max(round_ms)],
+                   "step_timer": ("one event pair around each round of K steps"
+                                  if flush is None else
+                                  "an event pair around each step (the L2 flush between "
+                                  "steps is not timed)")},
+        "effective_weight_GBps": step_bytes / (total_ms / K / 1e3) / 1e9,
+        "effective_weight_frac_of_hbm": step_bytes / (total_ms / K / 1e3) / 1e9 / peak,
+        "roofline": {"bound": "hbm", "kernel": wl.kernel, "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": (achieved / peak) if achieved else None,
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "bytes_per_launch": dom_bytes, "avg_launch_ms": dom_avg_ms,
+                     "launches_timed": len(dom_ms), "traffic": traffic},
+        "clocks": clk,
+        "e2e": {"value": e2e_rate, "unit": "tokens/s",
+                "h2d_bytes_per_step": wl.h2d_bytes, "d2h_bytes_per_step": wl.d2h_bytes,
+                "copies": wl.e2e_copies},
+        "gpu_launches": wl.launches_per_step * K,
+    }
+    if dist.rank == 0 and n == 1 and cpu_seconds > 0:
+        done, el, nsteps, cores, _ = time_oracle(wl, cpu_seconds)
+        out["cpu_baseline"] = {
+            "value": done / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": (f"{nsteps} tokens of {wl.name} through the scalar C oracle "
+                       f"(OpenMP over output rows), {el:.1f} s"
+                       if isinstance(wl, LlamaDecode) else
+                       f"{nsteps} x one layer of {wl.name} (T={wl.T}) through the scalar C "
+                       f"oracle (the first {wl.o_tok} of its tokens), counted as "
+                       f"1/{wl.layers} of a step, {el:.1f} s")}
+    del graphs, mgraphs, e2e_graphs
+    return out
 
 
 def main():
@@ -654,140 +854,31 @@ def main():
     dist.init("nccl")
     from moe_up_gate_b200 import q8
     q8.load()
-    wl = make_workload(args, dev)
     stream = torch.cuda.Stream(device=dev)
-    K, W = args.steps, max(args.warmup, 3)
-    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev) if getattr(wl, "flush", False) \
-        else None
-
-    # one CUDA graph per step index (each with its own timing marks)
-    graphs, marks = [], []
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        wl.issue(0, NoMarks())  # eager warm-up (sets kernel attributes)
-    torch.cuda.synchronize()
-    for i in range(W + K):
-        m = Marks(wl.dominant_launches) if i >= W else NoMarks()
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            wl.issue(i, m)
-        graphs.append(g)
-        marks.append(m)
-    torch.cuda.synchronize()
-
-    # device-timed region: rounds of exactly K steps, each bracketed by a
-    # barrier and a synchronize; enough rounds for about --min-seconds of
-    # timed work (the clock sampler needs that long); the median round is
-    # reported (after the 11-round, median protocol of the narray-llm README)
-    st_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    en_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    with torch.cuda.stream(stream):
-        for i in range(W):
-            if flush is not None:
-                flush.zero_()
-            graphs[i].replay()
-    torch.cuda.synchronize()
-    clocks = ClockSampler(gpu_id(dist.local))
-    clocks.start()
-    time.sleep(0.5)  # let the sampler start before the timed work
-
-    def one_round():
-        torch.cuda.synchronize()
-        dist.barrier()
-        with torch.cuda.stream(stream):
-            for i in range(K):
-                if flush is not None:
-                    flush.zero_()
-                st_ev[i].record(stream)
-                graphs[W + i].replay()
-                en_ev[i].record(stream)
-        torch.cuda.synchronize()
-        dist.barrier()
-        ms = dist.max(sum(a.elapsed_time(b) for a, b in zip(st_ev, en_ev)))
-        dom = []
-        for m in marks[W:]:
-            dom.extend(m.ms())
-        return ms, dom
-
-    torch.cuda.nvtx.range_push("timed")
-    first_ms, dom_ms = one_round()
-    rounds = int(min(1000, max(3, math.ceil(args.min_seconds * 1e3 / max(first_ms, 1e-3)))))
-    round_ms = [first_ms]
-    for _ in range(rounds - 1):
-        ms, dom = one_round()
-        round_ms.append(ms)
-        dom_ms.extend(dom)
-    torch.cuda.nvtx.range_pop()
-    clk = clocks.stop()
-    total_ms = statistics.median(round_ms)
-
-    # end to end through the public API with host buffers: every step copies
-    # its inputs from pinned host memory, runs the step (graphs of the same
-    # public calls, reading input set 0) and copies its result back
-    e2e_graphs = []
-    for c in range(wl.copies):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            wl.issue(c, NoMarks(), input_set=0)
-        e2e_graphs.append(g)
-    e2e_ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-    torch.cuda.synchronize()
-    dist.barrier()
-    with torch.cuda.stream(stream):
-        e2e_ev[0].record(stream)
-        for i in range(K):
-            wl.e2e_pre()
-            e2e_graphs[i % wl.copies].replay()
-            wl.e2e_post()
-        e2e_ev[1].record(stream)
-    torch.cuda.synchronize()
-    e2e_rate, e2e_ms = job_rate(dist, wl.tokens_per_step * K, e2e_ev[0].elapsed_time(e2e_ev[1]))
-    dist.barrier()
-
-    n = dist.world
-    # total_ms is already the max over ranks of each round (one_round)
-    value, total_ms = job_rate(dist, wl.tokens_per_step * K, total_ms)
-    step_bytes = statistics.mean(wl.unique_bytes(W + i) for i in range(K))
-    peak, peak_kind = measured_peak()
-    if isinstance(wl, LlamaDecode):
-        dom_bytes = wl.dominant_bytes
-    else:
-        dom_bytes = statistics.mean(wl.dominant_bytes_at(W + i) for i in range(K))
-    dom_avg_ms = statistics.mean(dom_ms) if dom_ms else None
-    achieved = dom_bytes / (dom_avg_ms / 1e3) / 1e9 if dom_avg_ms else None
-    traffic = recorded_traffic(wl.name + (f"_t{wl.T}" if hasattr(wl, "T") else ""), wl.kernel)
-    out = {
-        "metric": "Q8_0 decode tokens/s", "value": value, "unit": "tokens/s", "n_gpus": n,
-        "steps": K, "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8 x int8 -> int32, fp32 sums",
-        "data": "synthetic (seeded N(0, 0.02) weights quantized to Q8_0, N(0,1) inputs)",
-        "config": dict(wl.config, parallelism=f"replicas x{n}", rounds=len(round_ms),
-                       round_ms_min_median_max=[min(round_ms), total_ms, max(round_ms)]),
-        "effective_weight_GBps": step_bytes * K * n / (total_ms / 1e3) / 1e9 / n,
-        "effective_weight_frac_of_hbm": step_bytes / (total_ms / K / 1e3) / 1e9 / peak,
-        "roofline": {"bound": "hbm", "kernel": wl.kernel, "achieved": achieved, "peak": peak,
-                     "unit": "GB/s", "frac": (achieved / peak) if achieved else None,
-                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
-                     "bytes_per_launch": dom_bytes, "avg_launch_ms": dom_avg_ms,
-                     "traffic": traffic},
-        "clocks": clk,
-        "e2e": {"value": e2e_rate, "unit": "tokens/s",
-                "h2d_bytes_per_step": wl.h2d_bytes, "d2h_bytes_per_step": wl.d2h_bytes},
-        "gpu_launches": wl.launches_per_step * K,
-    }
-    if dist.rank == 0 and n == 1 and not args.no_cpu_baseline:
-        done, el, nsteps, cores, _ = time_oracle(wl, args.cpu_seconds)
-        out["cpu_baseline"] = {
-            "value": done / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": (f"{nsteps} tokens of {wl.name} through the scalar C oracle "
-                       f"(OpenMP over output rows), {el:.1f} s"
-                       if isinstance(wl, LlamaDecode) else
-                       f"{nsteps} x one layer of {wl.name} (T={wl.T}) through the scalar C "
-                       f"oracle, counted as 1/{wl.layers} of a step, {el:.1f} s")}
+    cpu_s = 0.0 if args.no_cpu_baseline else args.cpu_seconds
+    wl = make_workload(args.workload, args.tokens, dev)
+    rec = measure(wl, args, dist, stream, cpu_s)
+    del wl
+    out = {"metric": METRIC, "value": rec.pop("value"), "unit": rec.pop("unit"),
+           "n_gpus": dist.world, "steps": args.steps, "warmup": max(args.warmup, 3),
+           "ms_per_step": rec.pop("ms_per_step"), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "int8 x int8 -> int32, fp32 sums", "data": DATA}
+    out.update(rec)
+    if args.workload == "llama2_110m_q8_decode" and not args.no_subs:
+        # the fused MoE feed-forward step (the subject op) on its own workloads
+        subs, packed30 = [], None
+        for name, T in SUB_WORKLOADS:
+            torch.cuda.empty_cache()
+            w = make_workload(name, T, dev, packed=packed30 if name == "moe_30layer" else None)
+            if name == "moe_30layer":
+                packed30 = w.L
+            r = measure(w, args, dist, stream, cpu_s / 3)
+            r["workload"] = f"{name}_t{T}"
+            subs.append(r)
+            del w
+        out["moe_subrecords"] = subs
     if dist.rank == 0:
         print(json.dumps(out))
-    del graphs, e2e_graphs
     dist.close()
 
 

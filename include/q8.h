@@ -295,11 +295,13 @@ q8_status q8_mul_mat_id_fp32(const q8_tensor *W, const float *a, int32_t a_per_s
  *  required), except that there is no ws / ws_bytes.
  *  Limit: the grouping tables must fit the scratch, i.e.
  *  q8_moe_workspace_size(n_tok, n_used, up_gate->n_mat) <= Q8_NOALLOC_SCRATCH_BYTES
- *  (for 128 experts and 8 per token: up to 1983 tokens); larger calls return
+ *  (for 128 experts and 8 per token: up to 1982 tokens); larger calls return
  *  Q8_E_WORKSPACE and launch nothing.
  *  The first call on each device looks up the scratch address on that device
- *  (cudaGetSymbolAddress, with that device current); make that first call
- *  before any stream capture.  Every call shares the one scratch array: calls
+ *  (cudaGetSymbolAddress, with that device current), and so does the first
+ *  call after the device's context was recreated (cudaDeviceReset): the
+ *  address is kept per device together with the id of the context it belongs
+ *  to.  Make that first call before any stream capture.  Every call shares the one scratch array: calls
  *  that overlap on the GPU (other streams, other host threads) race and give
  *  wrong results; serialize them.  The scratch keeps the last call's contents;
  *  nothing in it needs clearing, because the grouping kernel rewrites every
@@ -335,7 +337,10 @@ q8_status q8_moe_combine(const float *y, const float *route_w, int64_t n_tok, in
  *      the intermediates (xq, h, hq, per-slot y) and the grid-barrier words
  *      of the fused layer kernel.  Zero-fill it before its first use; the
  *      calls leave those words at zero (after a wait timeout reported by
- *      q8_check, zero it again).
+ *      q8_check, zero it again).  The barrier words have a fixed place in
+ *      the first 256 bytes, which no call of any shape uses for anything
+ *      else, so a workspace sized for the largest call serves calls of
+ *      every smaller shape in any order.
  * Routed batches of at most 32 pairs (n_tok * n_used) with n_embd <= 4096
  * and n_ff <= 2048 run as ONE cooperative kernel (grouping, up/gate +
  * SwiGLU, a grid barrier, down + combine); the result is bitwise that of
@@ -353,13 +358,40 @@ q8_status q8_moe_ffn(const q8_tensor *up_gate, const q8_tensor *down, const floa
  *    error from the last routed call that used it: an id out of range or
  *    repeated within a token.  The outputs of pairs with out-of-range ids are
  *    then unspecified.
- *  - Q8_E_CUDA if the stream reported an error, or if a streaming kernel on
- *    this device ever gave up waiting (after about 2 s) for a shared-memory
- *    stage; that flag stays set for the life of the process, and results
- *    computed after it are not to be trusted.
+ *  - Q8_E_CUDA if the stream reported an error, or if a kernel on this
+ *    device gave up waiting (after about 2 s) for a shared-memory stage or
+ *    for the other CTAs of its grid; that flag stays set until
+ *    q8_reset_errors clears it, and results computed since it was set are
+ *    not to be trusted.
  * Else Q8_OK.
  */
 q8_status q8_check(const void *ws, void *stream);
+
+/*
+ * q8_reset_errors -- clear the wait-timeout flags (the Q8_E_CUDA condition
+ * of q8_check above) on the current device, so that one timeout does not
+ * poison every later check.  Synchronous; call it while no libq8 kernel is
+ * running on the device.  Routing-id errors live in the caller's workspace
+ * and are rewritten by every routed call; they need no reset.  After a
+ * timeout inside q8_moe_ffn's fused layer kernel, also zero that call's
+ * workspace (its grid-barrier words are left inconsistent).
+ */
+q8_status q8_reset_errors(void);
+
+/*
+ * q8_debug_wait_timeout -- test hook for the bounded waits: runs one wait
+ * that cannot succeed, which gives up after limit_ns nanoseconds, latches the
+ * wait-timeout flag that q8_check reports and returns (the kernel ends; the
+ * device stays usable).
+ *  kind 0: an mbarrier wait on a phase that nothing completes (the wait of
+ *          every streaming kernel's shared-memory ring).
+ *  kind 1: the fused layer kernel's grid barrier with one arrival short; bar
+ *          is a device pointer to two zeroed 32-bit words, which the call
+ *          leaves inconsistent.
+ *  limit_ns: 1e3 .. 1e10.
+ * Clear the flag afterwards with q8_reset_errors.
+ */
+q8_status q8_debug_wait_timeout(int32_t kind, int64_t limit_ns, unsigned *bar, void *stream);
 
 /*
  * q8_debug_block_dots -- test hook: the exact int32 per-block dots of the

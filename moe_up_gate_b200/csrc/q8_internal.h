@@ -68,11 +68,21 @@ q8_status check_tensor(const q8_tensor *W, const char *name, bool need_single);
 // ---------------------------------------------------------------------------
 // Routed-call workspace: int32 words.
 //   [0] error flags  [1] number of experts in the dp4a list  [2] number in the
-//   tensor-core list  [3] pairs  then count[E], offset[E+1], list_small[E],
-//   list_big[E], pairs[P] (pair index p = t * n_used + s, sorted by expert,
-//   then p).
+//   tensor-core list  [3] pairs  [4] [5] the fused layer kernel's grid-barrier
+//   words (arrivals, generation)  [6] [7] unused, then count[E], offset[E+1],
+//   list_small[E], list_big[E], pairs[P] (pair index p = t * n_used + s,
+//   sorted by expert, then p).
+// No grouping writes words 4-7, so the barrier words keep their place and
+// their zero whatever the shape of the calls that share a workspace.
 // ---------------------------------------------------------------------------
-enum : int { WS_ERR = 0, WS_N_SMALL = 1, WS_N_BIG = 2, WS_N_PAIRS = 3, WS_HEADER = 4 };
+enum : int {
+    WS_ERR = 0,
+    WS_N_SMALL = 1,
+    WS_N_BIG = 2,
+    WS_N_PAIRS = 3,
+    WS_BAR = 4,
+    WS_HEADER = 8
+};
 enum : int { ERR_ID_RANGE = 1, ERR_ID_REPEAT = 2 };
 
 struct GroupLayout {
@@ -155,6 +165,11 @@ q8_status read_wait_errors_layer(int *flags);
 q8_status read_wait_errors_matmul(int *flags);
 q8_status read_wait_errors_moe(int *flags);
 q8_status read_wait_errors_tc(int *flags);
+// Zero the wait-timeout flag of each file on the current device.
+q8_status clear_wait_errors_layer();
+q8_status clear_wait_errors_matmul();
+q8_status clear_wait_errors_moe();
+q8_status clear_wait_errors_tc();
 
 // Tensor-core path (q8_tc.cu) for experts with at least kTcMinPairs routed
 // rows: whether a weight view can take it, and the launch over the

@@ -39,6 +39,12 @@ q8_status read_wait_errors_layer(int *flags) {
     return e == cudaSuccess ? Q8_OK : Q8_E_CUDA;
 }
 
+q8_status clear_wait_errors_layer() {
+    const int zero = 0;
+    cudaError_t e = cudaMemcpyToSymbol(g_err_layer, &zero, sizeof(int));
+    return e == cudaSuccess ? Q8_OK : Q8_E_CUDA;
+}
+
 constexpr int kLayerNT = 4;   // activation rows per pass (template bound), several tokens
 
 struct LayerParams {
@@ -74,9 +80,10 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
 // after its CTA's global writes (ordered by a CTA barrier before the call).
 // bar[0] counts arrivals and is reset to 0 by the last one, which then
 // advances the generation bar[1]; the others wait for the generation to move.
-// Bounded: after kWaitLimitNs the wait records Q8_WAIT_TIMEOUT and returns
+// Bounded: after limit_ns the wait records Q8_WAIT_TIMEOUT and returns
 // false (the barrier word is then left inconsistent: q8_check reports it).
-__device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned n, int *err) {
+__device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned n, int *err,
+                                             uint64_t limit_ns = kWaitLimitNs) {
     const unsigned gen = ld_acquire_u32(bar + 1);
     __threadfence();
     const unsigned old = atomicAdd(bar, 1u);
@@ -88,7 +95,7 @@ __device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned n, int *err
     }
     const uint64_t t0 = globaltimer_ns();
     while (ld_acquire_u32(bar + 1) == gen) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             atomicOr(err, Q8_WAIT_TIMEOUT);
             return false;
         }
@@ -522,4 +529,37 @@ q8_status launch_layer(const q8_tensor *up_gate, const q8_tensor *down, const fl
     return Q8_OK;
 }
 
+// Test hook: one bounded wait that cannot succeed.  kind 0: an mbarrier
+// phase that nothing completes; kind 1: the grid barrier with one arrival
+// short (n = gridDim.x + 1).  Both give up after limit_ns, latch
+// Q8_WAIT_TIMEOUT in this file's error word and return.
+__global__ void wait_probe_kernel(int kind, uint64_t limit_ns, unsigned *bar) {
+    __shared__ uint64_t mb;
+    if (kind == 0) {
+        if (threadIdx.x == 0) {
+            mbar_init(&mb, 1);
+            fence_barrier_init();
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) mbar_wait_for(&mb, 0, &g_err_layer, limit_ns);
+    } else {
+        __syncthreads();
+        if (threadIdx.x == 0) grid_barrier(bar, gridDim.x + 1, &g_err_layer, limit_ns);
+    }
+}
+
 }  // namespace q8
+
+using namespace q8;
+
+extern "C" q8_status q8_debug_wait_timeout(int32_t kind, int64_t limit_ns, unsigned *bar,
+                                           void *stream) {
+    Q8_REQUIRE(kind == 0 || kind == 1, Q8_E_SHAPE, "q8_debug_wait_timeout: kind %d", kind);
+    Q8_REQUIRE(limit_ns >= 1000 && limit_ns <= 10000000000LL, Q8_E_SHAPE,
+               "q8_debug_wait_timeout: limit_ns=%lld outside [1e3, 1e10]", (long long)limit_ns);
+    Q8_REQUIRE(kind == 0 || bar != nullptr, Q8_E_NULL, "q8_debug_wait_timeout: bar is NULL");
+    Q8_REQUIRE(((uintptr_t)bar & 3u) == 0, Q8_E_ALIGN, "q8_debug_wait_timeout: bar misaligned");
+    wait_probe_kernel<<<kind == 0 ? 1 : 2, 32, 0, (cudaStream_t)stream>>>(
+        kind, (uint64_t)limit_ns, bar);
+    return launch_status("wait_probe_kernel");
+}

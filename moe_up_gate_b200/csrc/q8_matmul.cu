@@ -23,6 +23,12 @@ q8_status read_wait_errors_matmul(int *flags) {
     return e == cudaSuccess ? Q8_OK : Q8_E_CUDA;
 }
 
+q8_status clear_wait_errors_matmul() {
+    const int zero = 0;
+    cudaError_t e = cudaMemcpyToSymbol(g_err_matmul, &zero, sizeof(int));
+    return e == cudaSuccess ? Q8_OK : Q8_E_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // matmul over the activation rows of each matrix.
 //   dense  (ws == nullptr): matrix 0; activation rows 0..n_dense-1; output

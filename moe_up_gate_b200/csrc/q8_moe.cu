@@ -121,6 +121,12 @@ q8_status read_wait_errors_moe(int *flags) {
     return e == cudaSuccess ? Q8_OK : Q8_E_CUDA;
 }
 
+q8_status clear_wait_errors_moe() {
+    const int zero = 0;
+    cudaError_t e = cudaMemcpyToSymbol(g_err_moe, &zero, sizeof(int));
+    return e == cudaSuccess ? Q8_OK : Q8_E_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // Fused up/gate + SwiGLU on the streaming engine.  A tile is nr/2 gate rows
 // [r0, r0 + nr/2) of one expert and the matching up rows n_ff + r0 ..., both
@@ -380,9 +386,12 @@ static q8_status launch_combine(const float *y, const float *w, int64_t n_tok, i
                       w, (int)n_tok, n_used, (int)n_out, out);
 }
 
-// moe_ffn workspace regions
+// moe_ffn workspace regions.  The grouping region comes first and always
+// holds at least its header, whose words WS_BAR.. are the fused layer
+// kernel's grid-barrier words: a fixed place that no shape-dependent region
+// of any call overlaps.
 struct FfnLayout {
-    size_t group, bar, xq, xd, h, y, total;
+    size_t group, xq, xd, h, y, total;
 };
 
 static FfnLayout ffn_layout(int64_t n_tok, int32_t n_used, int64_t n_mat, int64_t n_embd,
@@ -391,9 +400,7 @@ static FfnLayout ffn_layout(int64_t n_tok, int32_t n_used, int64_t n_mat, int64_
     const int64_t P = n_tok * n_used;
     size_t o = 0;
     L.group = o;
-    o += routed ? group_bytes(P, n_mat) : 0;
-    L.bar = o;  // grid barrier words of the fused layer kernel
-    o += 256;
+    o += routed ? group_bytes(P, n_mat) : 256;
     L.xq = o;
     o += round_up((size_t)n_tok * n_embd, 256);
     L.xd = o;
@@ -525,7 +532,45 @@ static __device__ __align__(256) int32_t g_noalloc_scratch[Q8_NOALLOC_SCRATCH_BY
 
 constexpr int kMaxDevices = 64;
 static std::mutex g_noalloc_mu;
-static void *g_noalloc_addr[kMaxDevices] = {};
+// Per device: the scratch address and the unique id of the context it was
+// looked up in.  The address belongs to the module loaded in that context;
+// when the device's context is recreated (cudaDeviceReset, a new primary
+// context) the module is loaded again, possibly elsewhere, so a changed
+// context id means the address is looked up again.
+struct NoallocAddr {
+    unsigned long long ctx_id;
+    void *addr;
+};
+static NoallocAddr g_noalloc_addr[kMaxDevices] = {};
+
+// The unique id of the calling thread's current context (0: none or unknown),
+// through the driver entry points the runtime exposes (no link-time libcuda).
+typedef int (*CtxGetCurrentFn)(void **);
+typedef int (*CtxGetIdFn)(void *, unsigned long long *);
+static unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static bool resolved = false;
+    if (!resolved) {
+        void *f1 = nullptr, *f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1{}, q2{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) ==
+                cudaSuccess &&
+            q1 == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) == cudaSuccess &&
+            q2 == cudaDriverEntryPointSuccess) {
+            get_current = (CtxGetCurrentFn)f1;
+            get_id = (CtxGetIdFn)f2;
+        }
+        resolved = true;
+    }
+    if (!get_current || !get_id) return 0;
+    void *ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != 0 || ctx == nullptr) return 0;
+    if (get_id(ctx, &id) != 0) return 0;
+    return id;
+}
 
 static q8_status noalloc_scratch_address(void **out) {
     int dev = -1;
@@ -536,15 +581,21 @@ static q8_status noalloc_scratch_address(void **out) {
     Q8_REQUIRE(dev >= 0 && dev < kMaxDevices, Q8_E_UNSUPPORTED,
                "q8_moe_up_gate_swiglu_noalloc: device %d beyond %d", dev, kMaxDevices);
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_addr[dev] == nullptr) {
+    unsigned long long ctx = current_context_id();
+    NoallocAddr &a = g_noalloc_addr[dev];
+    if (ctx == 0 || a.addr == nullptr || a.ctx_id != ctx) {
+        // set-up: the device address of the scratch in this device's current
+        // context (the lookup also makes the primary context current)
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess || p == nullptr)
             Q8_FAIL(Q8_E_CUDA, "q8_moe_up_gate_swiglu_noalloc: cudaGetSymbolAddress: %s",
                     cudaGetErrorString(e));
-        g_noalloc_addr[dev] = p;
+        if (ctx == 0) ctx = current_context_id();
+        a.addr = p;
+        a.ctx_id = ctx;  // 0 (id unknown): looked up again on every call
     }
-    *out = g_noalloc_addr[dev];
+    *out = a.addr;
     return Q8_OK;
 }
 
@@ -719,7 +770,7 @@ q8_status q8_moe_ffn(const q8_tensor *up_gate, const q8_tensor *down, const floa
         int32_t *err = routed ? (int32_t *)(w8 + F.group) : nullptr;
         if (routed && layer_eligible(up_gate, down, n_tok, n_used))
             return launch_layer(up_gate, down, x, n_tok, ids, route_w, n_used, out, h,
-                                (unsigned *)(w8 + F.bar), err, s);
+                                (unsigned *)(w8 + F.group) + WS_BAR, err, s);
         st = q8_moe_up_gate_swiglu_fp32(up_gate, x, n_tok, ids, n_used, h, err, s);
         if (st != Q8_OK) return st;
         if (!routed) return launch_matmul_dense(down, nullptr, nullptr, h, n_tok, out, s);
@@ -750,6 +801,13 @@ q8_status q8_moe_ffn(const q8_tensor *up_gate, const q8_tensor *down, const floa
     st = launch_matmul_routed(down, nullptr, nullptr, h, 1, n_tok, n_used, y, wsg, s);
     if (st != Q8_OK) return st;
     return launch_combine(y, route_w, n_tok, n_used, n_embd, out, s);
+}
+
+q8_status q8_reset_errors(void) {
+    if (clear_wait_errors_matmul() != Q8_OK || clear_wait_errors_moe() != Q8_OK ||
+        clear_wait_errors_tc() != Q8_OK || clear_wait_errors_layer() != Q8_OK)
+        Q8_FAIL(Q8_E_CUDA, "q8_reset_errors: clearing the kernels' wait flags failed");
+    return Q8_OK;
 }
 
 q8_status q8_check(const void *ws, void *stream) {

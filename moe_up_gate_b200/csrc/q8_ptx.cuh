@@ -65,18 +65,25 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 constexpr int Q8_WAIT_TIMEOUT = 1;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
-// Wait for the phase with the given parity to complete; false after ~2 s.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err_word) {
+// Wait for the phase with the given parity to complete; false after
+// limit_ns (the error word then holds Q8_WAIT_TIMEOUT).
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, int *err_word,
+                                              uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         for (int i = 0; i < 256; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             atomicOr(err_word, Q8_WAIT_TIMEOUT);
             return false;
         }
     }
+}
+
+// Wait for the phase with the given parity to complete; false after ~2 s.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err_word) {
+    return mbar_wait_for(bar, parity, err_word, kWaitLimitNs);
 }
 
 // 1-D bulk copy global -> this CTA's shared memory, completing `bytes` of

@@ -65,6 +65,12 @@ q8_status read_wait_errors_tc(int *flags) {
     return e == cudaSuccess ? Q8_OK : Q8_E_CUDA;
 }
 
+q8_status clear_wait_errors_tc() {
+    const int zero = 0;
+    cudaError_t e = cudaMemcpyToSymbol(g_err_tc, &zero, sizeof(int));
+    return e == cudaSuccess ? Q8_OK : Q8_E_CUDA;
+}
+
 struct TcParams {
     CUtensorMap tmap;  // weights as a 2-D int8 tensor [rows_total][k]
     const uint16_t *wd;

@@ -47,7 +47,8 @@ EXPORTS = ["q8_scale_stride", "q8_pack", "q8_pack_up_gate", "q8_quantize_row", "
            "q8_moe_ffn_workspace_size", "q8_moe_ffn", "q8_check", "q8_debug_block_dots",
            "q8_status_string", "q8_last_error", "q8_moe_group",
            "q8_moe_up_gate_swiglu_pregrouped", "q8_mul_mat_id_pregrouped",
-           "q8_moe_up_gate_swiglu_noalloc", "q8_moe_up_gate_swiglu_fp32", "q8_mul_mat_id_fp32"]
+           "q8_moe_up_gate_swiglu_noalloc", "q8_moe_up_gate_swiglu_fp32", "q8_mul_mat_id_fp32",
+           "q8_reset_errors", "q8_debug_wait_timeout"]
 
 
 def lib_path() -> str:
@@ -94,6 +95,8 @@ def load(auto_build: bool = True):
                                                    vp, vp, vp]),
             "q8_moe_up_gate_swiglu_fp32": (st, [P(_Tensor), vp, i64, vp, i32, vp, vp, vp]),
             "q8_mul_mat_id_fp32": (st, [P(_Tensor), vp, i32, i64, vp, i32, vp, vp, vp]),
+            "q8_reset_errors": (st, []),
+            "q8_debug_wait_timeout": (st, [i32, i64, vp, vp]),
             "q8_status_string": (ctypes.c_char_p, [st]),
             "q8_last_error": (ctypes.c_char_p, []),
         }
@@ -367,6 +370,17 @@ def moe_ffn(up_gate: Q8Tensor, down: Q8Tensor, x, ids=None, route_w=None, ws=Non
 
 def check(ws, stream=None):
     _call("q8_check", _ptr(ws), _stream(stream))
+
+
+def reset_errors():
+    """Clear the wait-timeout flags q8_check reports (no kernel may be running)."""
+    _call("q8_reset_errors")
+
+
+def debug_wait_timeout(kind: int, limit_ns: int, bar=None, stream=None):
+    """Test hook: one bounded wait that must give up after limit_ns (kind 0: a
+    shared-memory ring wait; kind 1: the grid barrier, bar = 2 zeroed int32 words)."""
+    _call("q8_debug_wait_timeout", kind, limit_ns, _ptr(bar), _stream(stream))
 
 
 def debug_block_dots(W: Q8Tensor, mat: int, rows: torch.Tensor, xq: torch.Tensor, stream=None):

@@ -163,3 +163,20 @@ def test_gemv_batched_validation(q8):
     assert lib.q8_gemv_batched(arr, 129, 1, None) == 2
     arr[1] = q8._GemvDesc(_tensor(q8), FAKE_ODD.value, FAKE.value)
     assert lib.q8_gemv_batched(arr, 2, 1, None) == 3
+
+
+def test_wait_hook_validation(q8):
+    lib = q8.load()
+    assert lib.q8_debug_wait_timeout(2, 5_000_000, None, None) == 2     # kind
+    assert lib.q8_debug_wait_timeout(0, 10, None, None) == 2            # limit below 1 us
+    assert lib.q8_debug_wait_timeout(0, 10**11, None, None) == 2        # limit above 10 s
+    assert lib.q8_debug_wait_timeout(1, 5_000_000, None, None) == 1     # no barrier words
+    assert lib.q8_debug_wait_timeout(1, 5_000_000, FAKE_ODD, None) == 3
+
+
+def test_noalloc_scratch_capacity(q8):
+    # 128 experts, 8 per token: the grouping tables of 1982 tokens fit the
+    # built-in 64 KiB scratch, those of 1983 do not
+    lib = q8.load()
+    assert lib.q8_moe_workspace_size(1982, 8, 128) <= 65536
+    assert lib.q8_moe_workspace_size(1983, 8, 128) > 65536

@@ -108,3 +108,27 @@ def test_fused_layer_reports_bad_ids():
     out = q8.moe_ffn(UG, DN, x, ids, p, ws=ws)
     q8.check(ws)
     assert torch.equal(out, _chain(UG, DN, x, ids, p)[0])
+
+
+def test_workspace_serves_a_large_then_a_small_call():
+    """One workspace sized for a 256-token call serves a 1-token call next
+    (and back again): the large call's grouping tables cover much of the
+    workspace, but the fused layer kernel's grid-barrier words have a fixed
+    place in the header that no grouping writes, so the small call's barrier
+    starts from zero.  The results equal those on fresh workspaces."""
+    shape = synth.MOE_LAYER
+    big = synth.moe_layer_tensors(951, 0, shape, 256, 1.0, device=DEV)
+    UG = q8.pack(big["up_gate"])
+    DN = q8.pack(big["down"])
+    small = synth.moe_layer_tensors(952, 0, shape, 1, 1.0)
+    xs, ids_s, p_s = small["x"].to(DEV), small["ids"].to(DEV), small["p"].to(DEV)
+    xb, ids_b, p_b = big["x"], big["ids"].to(DEV), big["p"].to(DEV)
+    ws = q8.moe_ffn_workspace(256, 8, 128, 2816, 704, DEV)
+    ref_small = q8.moe_ffn(UG, DN, xs, ids_s, p_s)  # fresh workspaces
+    ref_big = q8.moe_ffn(UG, DN, xb, ids_b, p_b)
+    for _ in range(3):
+        out_b = q8.moe_ffn(UG, DN, xb, ids_b, p_b, ws=ws)
+        out_s = q8.moe_ffn(UG, DN, xs, ids_s, p_s, ws=ws)
+        q8.check(ws)
+        assert torch.equal(out_b, ref_big)
+        assert torch.equal(out_s, ref_small)

@@ -4,11 +4,13 @@ Some callers cannot call cudaMalloc (or any allocating routine) where they run
 the MoE step -- inside an allocator hook, in a plugin whose host forbids device
 allocation, or in a loop that must not touch the allocator -- so libq8 offers a
 variant of the routed up/gate + SwiGLU call that takes no workspace and keeps
-its expert-grouping tables in a built-in device array.  This test calls it
+its expert-grouping tables in a built-in device array.  The tests call it
 through the C ABI twice in a row (different token counts and routing ids, so the
-second call starts from the first call's leftover scratch contents) and checks
+second call starts from the first call's leftover scratch contents) and check
 each result against the workspace-taking entry point q8_moe_up_gate_swiglu,
-within the parity tolerances the other tests use.  This file is collected last.
+within the parity tolerances the other tests use; one case routes 32 tokens to
+one expert so that the tensor-core kernel reads its tables from the built-in
+scratch.  This file is collected last.
 """
 import ctypes
 
@@ -66,6 +68,41 @@ def test_noalloc_matches_workspace_entry_on_two_calls():
         assert np.all(np.abs(host(h) - hr) <= TOL * (np.abs(hr) + 1e-30))
         assert np.array_equal(host(hq), host(ref["hq"]))
         assert np.array_equal(bits(hd), bits(ref["hd"]))
+
+
+def _noalloc(lib, UG, xq, xd, ids, h, hq, hd):
+    n_tok, n_used = ids.shape
+    return lib.q8_moe_up_gate_swiglu_noalloc(
+        ctypes.byref(UG.c()), ctypes.c_void_p(xq.data_ptr()), ctypes.c_void_p(xd.data_ptr()),
+        n_tok, ctypes.c_void_p(ids.data_ptr()), n_used, ctypes.c_void_p(h.data_ptr()),
+        ctypes.c_void_p(hq.data_ptr()), ctypes.c_void_p(hd.data_ptr()), None, None,
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+def test_noalloc_tensor_core_branch():
+    """Without the g/u taps, experts with >= 16 routed rows go to the
+    tensor-core kernel, which reads the tensor-core list and the pair lists
+    from the built-in scratch: slot 0 of all 32 tokens names expert 0.  Two
+    calls in a row with different ids; each equals the workspace entry point
+    bit for bit (the same kernels on the same tables)."""
+    lib = q8.load()
+    n_used, n_ff = 8, 704
+    for n_tok, seed in ((32, 74), (48, 75)):
+        UG, xq, xd, ids = _inputs(n_tok, seed)
+        ids = ids.clone()
+        for t in range(n_tok):  # expert 0 in slot 0 of every token, ids still distinct
+            row = [e for e in ids[t].tolist() if e != 0][: n_used - 1]
+            ids[t] = torch.tensor([0] + row, dtype=torch.int32, device=DEV)
+        counts = torch.bincount(ids.flatten().long(), minlength=128)
+        assert int(counts[0]) == n_tok >= 16
+        ref = q8.moe_up_gate_swiglu(UG, xq, xd, ids, want_hq=True)
+        h = torch.full((n_tok, n_used, n_ff), float("nan"), device=DEV)
+        hq = torch.zeros((n_tok, n_used, n_ff), dtype=torch.int8, device=DEV)
+        hd = torch.zeros((n_tok, n_used, n_ff // 32), dtype=torch.float16, device=DEV)
+        assert _noalloc(lib, UG, xq, xd, ids, h, hq, hd) == 0, lib.q8_last_error()
+        torch.cuda.synchronize()
+        assert torch.equal(h, ref["h"])
+        assert torch.equal(hq, ref["hq"]) and torch.equal(hd, ref["hd"])
 
 
 def test_noalloc_rejects_calls_beyond_the_scratch():
