@@ -334,13 +334,14 @@ q8_status q8_moe_combine(const float *y, const float *route_w, int64_t n_tok, in
  *  n_used == 1), where out = down . quantize(h).
  *  out: fp32 [n_tok][n_embd].
  *  ws: q8_moe_ffn_workspace_size(...) bytes, 256-byte aligned; it also holds
- *      the intermediates (xq, h, hq, per-slot y) and the grid-barrier words
- *      of the fused layer kernel.  Zero-fill it before its first use; the
- *      calls leave those words at zero (after a wait timeout reported by
- *      q8_check, zero it again).  The barrier words have a fixed place in
- *      the first 256 bytes, which no call of any shape uses for anything
- *      else, so a workspace sized for the largest call serves calls of
- *      every smaller shape in any order.
+ *      the intermediates (xq, h, hq, per-slot y) and the grid-barrier
+ *      counter of the fused layer kernel, which every fused call advances by
+ *      its grid size (the device's SM count).  Zero-fill the workspace before
+ *      its first use, use it on one device, and zero it again after a wait
+ *      timeout reported by q8_check.  The counter has a fixed place in the
+ *      first 256 bytes, which no call of any shape uses for anything else, so
+ *      a workspace sized for the largest call serves calls of every smaller
+ *      shape in any order.
  * Routed batches of at most 32 pairs (n_tok * n_used) with n_embd <= 4096
  * and n_ff <= 2048 run as ONE cooperative kernel (grouping, up/gate +
  * SwiGLU, a grid barrier, down + combine); the result is bitwise that of
@@ -351,6 +352,31 @@ size_t q8_moe_ffn_workspace_size(int64_t n_tok, int32_t n_used, int64_t n_mat, i
 q8_status q8_moe_ffn(const q8_tensor *up_gate, const q8_tensor *down, const float *x,
                      int64_t n_tok, const int32_t *ids, const float *route_w, int32_t n_used,
                      float *out, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * q8_route -- the router, the step before the routed calls: routing ids and
+ * routing weights from the activations.  The pages name MoE routing only as
+ * a run-time option ([HADA], opening section on the 2016-Xeon set-up:
+ * 「CPUを考慮したMoEルーティング」); this is the plain top-k router:
+ *    logits[t][e] = sum_i w_router[e][i] * x[t][i], products and sums in fp64;
+ *    ids[t]       = the n_used experts with the largest logits, largest first,
+ *                   equal logits taken by ascending expert index;
+ *    route_w[t]   = softmax over the selected logits only (fp64, stored fp32).
+ *  w_router: fp32 [n_exp][n_embd] (not quantized); x: fp32 [n_tok][n_embd];
+ *            both 16-byte aligned, n_embd a multiple of 4.
+ *  ids: out int32 [n_tok][n_used]; route_w: out fp32 [n_tok][n_used]; they
+ *       feed q8_moe_ffn and the other routed calls directly.
+ *  logits: optional out fp64 [n_tok][n_exp] (NULL: not written).
+ *  Limits: n_exp <= Q8_ROUTE_MAX_EXP, n_used <= min(n_exp, Q8_MAX_USED), and
+ *  the shared-memory plan (16 * n_embd + 33 * n_exp bytes) within 227 KB,
+ *  else Q8_E_SHAPE / Q8_E_UNSUPPORTED.  NaN logits rank as -infinity.
+ * One launch of thread-block clusters (8 CTAs per 4 tokens, the experts split
+ * across the cluster, the top-k read through distributed shared memory).
+ */
+#define Q8_ROUTE_MAX_EXP 1024
+q8_status q8_route(const float *w_router, const float *x, int64_t n_tok, int64_t n_embd,
+                   int64_t n_exp, int32_t n_used, int32_t *ids, float *route_w, double *logits,
+                   void *stream);
 
 /*
  * q8_check -- synchronize `stream` and report errors found on the device:
@@ -386,8 +412,8 @@ q8_status q8_reset_errors(void);
  *  kind 0: an mbarrier wait on a phase that nothing completes (the wait of
  *          every streaming kernel's shared-memory ring).
  *  kind 1: the fused layer kernel's grid barrier with one arrival short; bar
- *          is a device pointer to two zeroed 32-bit words, which the call
- *          leaves inconsistent.
+ *          is a device pointer to a zeroed, 8-byte aligned 64-bit counter,
+ *          which the call leaves off its multiple.
  *  limit_ns: 1e3 .. 1e10.
  * Clear the flag afterwards with q8_reset_errors.
  */

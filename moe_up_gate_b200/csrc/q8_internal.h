@@ -69,7 +69,7 @@ q8_status check_tensor(const q8_tensor *W, const char *name, bool need_single);
 // Routed-call workspace: int32 words.
 //   [0] error flags  [1] number of experts in the dp4a list  [2] number in the
 //   tensor-core list  [3] pairs  [4] [5] the fused layer kernel's grid-barrier
-//   words (arrivals, generation)  [6] [7] unused, then count[E], offset[E+1],
+//   arrival counter (64 bits)  [6] [7] unused, then count[E], offset[E+1],
 //   list_small[E], list_big[E], pairs[P] (pair index p = t * n_used + s,
 //   sorted by expert, then p).
 // No grouping writes words 4-7, so the barrier words keep their place and

@@ -46,6 +46,13 @@ q8_status clear_wait_errors_layer() {
 }
 
 constexpr int kLayerNT = 4;   // activation rows per pass (template bound), several tokens
+// The h bulk copy's mbarrier: after the ring's barriers in the plan's first
+// 256 bytes (full and empty of kMaxStages stages, then the raw slot's two).
+constexpr int kLayerHBar = 2 * kMaxStages * 8 + 16;
+static_assert(kLayerHBar + 8 <= 256, "barrier area");
+// fp32 h of all pairs is copied back in bulk when it takes at most this much
+// shared memory (the copy shares the phase-B region with the other areas)
+constexpr int kLayerHBulkBytes = 24 * 1024;
 
 struct LayerParams {
     const int8_t *ug_q;
@@ -61,48 +68,59 @@ struct LayerParams {
     const float *route_w;
     float *out;
     float *h;       // [P][n_ff] scratch
-    unsigned *bar;  // grid barrier {arrivals, generation}
+    unsigned *bar;  // grid barrier: 64-bit arrival counter (8-byte aligned)
     int32_t *err_out;
     int n_tok, n_used, n_mat;
     int64_t lay_count, lay_offset, lay_list, lay_big, lay_pairs;
     int off_hq, off_hd, off_y, off_inv;  // phase-B areas
+    int off_hf;                          // fp32 h of all pairs, copied in bulk (-1: none)
+    int off_rw;                          // the routing weights [P], staged at the start
     int nrb;                             // down rows per unit
     Plan plan;
 };
 
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 
-// Barrier of all CTAs of a co-resident grid, entered by one thread per CTA
+// Barrier of all n CTAs of a co-resident grid, entered by one thread per CTA
 // after its CTA's global writes (ordered by a CTA barrier before the call).
-// bar[0] counts arrivals and is reset to 0 by the last one, which then
-// advances the generation bar[1]; the others wait for the generation to move.
+// bar: a 64-bit arrival counter (8-byte aligned) that only grows: every
+// launch of n CTAs adds n, so between launches it is a multiple of n (zero
+// before the first use).  A CTA adds one (release) and waits (acquire) until
+// the counter reaches the next multiple of n above its own arrival: one
+// atomic per CTA and no reset, so the last arrival releases the others with
+// its own atomic.
 // Bounded: after limit_ns the wait records Q8_WAIT_TIMEOUT and returns
-// false (the barrier word is then left inconsistent: q8_check reports it).
+// false (the counter is then left off its multiple: q8_check reports it).
 __device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned n, int *err,
                                              uint64_t limit_ns = kWaitLimitNs) {
-    const unsigned gen = ld_acquire_u32(bar + 1);
+    unsigned long long *cnt = reinterpret_cast<unsigned long long *>(bar);
     __threadfence();
-    const unsigned old = atomicAdd(bar, 1u);
-    if (old == n - 1) {
-        atomicExch(bar, 0u);
+    const unsigned long long old = atomicAdd(cnt, 1ull);
+    const unsigned long long target = (old / n + 1) * n;
+    if (old + 1 == target) {
         __threadfence();
-        atomicAdd(bar + 1, 1u);
         return true;
     }
     const uint64_t t0 = globaltimer_ns();
-    while (ld_acquire_u32(bar + 1) == gen) {
+    while (ld_acquire_u64(cnt) < target) {
         if (globaltimer_ns() - t0 > limit_ns) {
             atomicOr(err, Q8_WAIT_TIMEOUT);
             return false;
         }
-        __nanosleep(64);
+        __nanosleep(32);
     }
     __threadfence();
     return true;
+}
+
+// Make this thread's global writes visible to later bulk (async-proxy) reads
+// of the same memory, and order its later bulk reads after what it observed.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // Quantize fp32 rows written in this launch by other CTAs (so loaded at L2,
@@ -147,6 +165,12 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
     extern __shared__ __align__(128) unsigned char smem[];
     Q8_TRACE(0);
     const Ring R = ring_init(smem, p.plan);
+    // the bulk copy of h after the grid barrier completes on its own mbarrier
+    uint64_t *hbar = reinterpret_cast<uint64_t *>(smem + kLayerHBar);
+    if (threadIdx.x == 0) {
+        mbar_init(hbar, 1);
+        fence_barrier_init();
+    }
     Q8_TRACE(1);
     griddep_wait();  // x, ids and route_w may come from the preceding kernel
     griddep_launch_dependents();
@@ -158,6 +182,11 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
         mbar_arrive_expect_tx(R.xfull, (uint32_t)p.k * 4);
         bulk_g2s_keep(R.raw, p.x, (uint32_t)p.k * 4, R.xfull);
     }
+    // the routing weights are read only by the combine at the very end, but
+    // loaded now, while the memory system is idle (ordered by the grouping's
+    // CTA barrier below)
+    float *s_rw = reinterpret_cast<float *>(smem + p.off_rw);
+    for (int i = threadIdx.x; i < p.n_tok * p.n_used; i += blockDim.x) s_rw[i] = p.route_w[i];
     int32_t *tab = reinterpret_cast<int32_t *>(smem + p.plan.off_tab);
     {
         GroupLayout L{};
@@ -308,21 +337,39 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
     }
 
     // ---------------- every CTA's h is written
+    const int P = p.n_tok * p.n_used;
+    if (p.off_hf >= 0) fence_proxy_async_global();  // h is read back by a bulk copy
     sync_all();
     Q8_TRACE(12);
-    if (threadIdx.x == 0) grid_barrier(p.bar, gridDim.x, &g_err_layer);
+    if (threadIdx.x == 0) {
+        grid_barrier(p.bar, gridDim.x, &g_err_layer);
+        if (p.off_hf >= 0) {
+            // all pairs' h [P][n_ff] in one bulk copy (16-byte aligned, a
+            // multiple of 16 bytes): one request stream instead of a load per
+            // thread, each waiting behind the weight stream
+            fence_proxy_async_global();
+            const uint32_t bytes = (uint32_t)P * (uint32_t)p.n_ff * 4u;
+            mbar_arrive_expect_tx(hbar, bytes);
+            bulk_g2s_keep(smem + p.off_hf, p.h, bytes, hbar);
+        }
+    }
     sync_all();
     Q8_TRACE(11);
 
     // every pair's h as Q8_0, in grouped (expert, pair) order
-    const int P = p.n_tok * p.n_used;
     const int n_valid = tab[p.lay_offset + p.n_mat];
     const XStage hs{reinterpret_cast<int8_t *>(smem + p.off_hq),
                     reinterpret_cast<float *>(smem + p.off_hd)};
     int *inv = reinterpret_cast<int *>(smem + p.off_inv);
     float *ybuf = reinterpret_cast<float *>(smem + p.off_y) + (size_t)grp * P * nrb;
-    stage_f32_l2(hs, p.h, p.n_ff, n_valid, [&](int j) { return tab[p.lay_pairs + j]; },
-                 threadIdx.x, kAll);
+    if (p.off_hf >= 0) {
+        mbar_wait(hbar, 0, &g_err_layer);
+        stage_f32_smem8(hs, reinterpret_cast<const float *>(smem + p.off_hf), p.n_ff, n_valid,
+                       [&](int j) { return tab[p.lay_pairs + j]; }, threadIdx.x, kAll);
+    } else {
+        stage_f32_l2(hs, p.h, p.n_ff, n_valid, [&](int j) { return tab[p.lay_pairs + j]; },
+                     threadIdx.x, kAll);
+    }
     for (int i = threadIdx.x; i < P; i += kAll) inv[i] = -1;
     sync_all();
     for (int j = threadIdx.x; j < n_valid; j += kAll) inv[tab[p.lay_pairs + j]] = j;
@@ -377,7 +424,7 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
             float acc = 0.0f;
             for (int s2 = 0; s2 < p.n_used; ++s2) {
                 const int q = inv[t * p.n_used + s2];
-                acc = fmaf(p.route_w[t * p.n_used + s2], q >= 0 ? ybuf[q * nrb + rr] : 0.0f, acc);
+                acc = fmaf(s_rw[t * p.n_used + s2], q >= 0 ? ybuf[q * nrb + rr] : 0.0f, acc);
             }
             p.out[(int64_t)t * p.k + r0 + rr] = acc;
         }
@@ -407,6 +454,7 @@ static bool layer_plan(LayerParams &p, int64_t P, int n_ff, int tq, int td, int 
     const int xmax = xrows;
     const int x_bytes = xmax * p.k + ((xmax * (p.k / QK) * 4 + 15) / 16) * 16;
     const int tab_bytes = ((group_words * 4 + 15) / 16) * 16;
+    const int rw_bytes = (int)((P * 4 + 15) / 16 * 16);
     const int raw_rows = raw ? std::min(xmax, kRawSlotBytes / (4 * p.k)) : 0;
     const int raw_bytes = raw_rows * 4 * p.k;
     int o = 0;
@@ -419,10 +467,16 @@ static bool layer_plan(LayerParams &p, int64_t P, int n_ff, int tq, int td, int 
     o += (int)(P * nrb * 4) * groups;  // one y buffer per consumer group
     const int inv = o;
     o += (int)(P * 4);
+    int hf = -1;
+    if (P * n_ff * 4 <= kLayerHBulkBytes) {
+        o = (o + 15) / 16 * 16;
+        hf = o;
+        o += (int)(P * n_ff * 4);
+    }
     const int union_bytes = (std::max(o, raw_bytes) + 127) / 128 * 128;
     const int stage_qs = round128(tq);
     const int stage_bytes = stage_qs + round128(td);
-    const int fixed = 256 + x_bytes + tab_bytes + union_bytes;
+    const int fixed = 256 + x_bytes + tab_bytes + rw_bytes + union_bytes;
     int stages = (budget - fixed) / stage_bytes;
     if (stages > kMaxStages) stages = kMaxStages;
     if (stages < 2) return false;
@@ -443,7 +497,8 @@ static bool layer_plan(LayerParams &p, int64_t P, int n_ff, int tq, int td, int 
     pl.off_part = pl.off_xd + ((xmax * (p.k / QK) * 4 + 15) / 16) * 16;  // unused
     pl.off_tab = pl.off_part;
     pl.tab_words = group_words;
-    const int off_union = pl.off_tab + tab_bytes;
+    p.off_rw = pl.off_tab + tab_bytes;
+    const int off_union = p.off_rw + rw_bytes;
     pl.raw_rows = raw_rows;
     pl.off_raw = off_union;
     pl.bytes = off_union + union_bytes;
@@ -452,6 +507,7 @@ static bool layer_plan(LayerParams &p, int64_t P, int n_ff, int tq, int td, int 
     p.off_hd = off_union + hd;
     p.off_y = off_union + y;
     p.off_inv = off_union + inv;
+    p.off_hf = hf >= 0 ? off_union + hf : -1;
     p.nrb = nrb;
     return pl.bytes <= budget;
 }
@@ -531,7 +587,7 @@ q8_status launch_layer(const q8_tensor *up_gate, const q8_tensor *down, const fl
 
 // Test hook: one bounded wait that cannot succeed.  kind 0: an mbarrier
 // phase that nothing completes; kind 1: the grid barrier with one arrival
-// short (n = gridDim.x + 1).  Both give up after limit_ns, latch
+// short (n = gridDim.x + 1, counter starting at zero).  Both give up after limit_ns, latch
 // Q8_WAIT_TIMEOUT in this file's error word and return.
 __global__ void wait_probe_kernel(int kind, uint64_t limit_ns, unsigned *bar) {
     __shared__ uint64_t mb;
@@ -558,7 +614,8 @@ extern "C" q8_status q8_debug_wait_timeout(int32_t kind, int64_t limit_ns, unsig
     Q8_REQUIRE(limit_ns >= 1000 && limit_ns <= 10000000000LL, Q8_E_SHAPE,
                "q8_debug_wait_timeout: limit_ns=%lld outside [1e3, 1e10]", (long long)limit_ns);
     Q8_REQUIRE(kind == 0 || bar != nullptr, Q8_E_NULL, "q8_debug_wait_timeout: bar is NULL");
-    Q8_REQUIRE(((uintptr_t)bar & 3u) == 0, Q8_E_ALIGN, "q8_debug_wait_timeout: bar misaligned");
+    Q8_REQUIRE(((uintptr_t)bar & 7u) == 0, Q8_E_ALIGN,
+               "q8_debug_wait_timeout: bar must be 8-byte aligned");
     wait_probe_kernel<<<kind == 0 ? 1 : 2, 32, 0, (cudaStream_t)stream>>>(
         kind, (uint64_t)limit_ns, bar);
     return launch_status("wait_probe_kernel");

@@ -435,7 +435,13 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                                     &g_err_matmul);
                     }
                 };
-                produce(R, tb, te, src, &g_err_matmul, jobs, true);
+                // The activation rows go first: under the weight stream of all
+                // CTAs, a copy queued behind this CTA's first weight tiles lands
+                // microseconds later, and no consumer can start before it.  So
+                // the producer waits for the preceding grid, copies the first
+                // problem's x, then streams the weights in order.
+                griddep_wait();
+                produce(R, tb, te, src, &g_err_matmul, jobs, false);
             } else {
                 produce(R, tb, te, src, &g_err_matmul);
             }

@@ -1,0 +1,236 @@
+// q8_route.cu -- the router: the step before the MoE path, which turns a
+// token's activations into the routing ids and routing weights that the
+// routed calls take as inputs.  The news.hada.io article on Gemma 4 26B-A4B
+// names MoE routing only as a run-time option (its opening section on the
+// 2016-Xeon set-up, 「CPUを考慮したMoEルーティング」); the reading here is the
+// plain top-k router:
+//   logits[t][e] = sum_i w_router[e][i] * x[t][i], every product and sum in
+//                  fp64 (fp32 inputs; each product is exact in fp64);
+//   ids[t]       = the n_used experts with the largest logits, largest first,
+//                  equal logits taken by ascending expert index;
+//   route_w[t]   = softmax over the selected logits only (the largest one
+//                  subtracted before exp, fp64), stored as fp32.
+//
+// One thread-block cluster per group of kRouteTok tokens: the cluster's CTAs
+// split the experts (CTA r takes experts e = r, r + C, ...; a warp per
+// expert row, 16-byte loads, fp64 fma per token, a fixed xor tree), keep the
+// logits in their own shared memory, and after a cluster barrier CTA 0 reads
+// every logit through distributed shared memory; a second cluster barrier
+// keeps every CTA's shared memory alive until then.  CTA 0 then selects the
+// top n_used per token (one warp per token, repeated warp argmax) and forms
+// the weights.  No atomics, no global scratch: the results are deterministic.
+#include <cooperative_groups.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "q8_internal.h"
+#include "q8_ptx.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace q8 {
+
+constexpr int kRouteTok = 4;         // tokens per cluster
+constexpr int kRouteThreads = 256;   // 8 warps
+constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr int kRouteCluster = 8;     // CTAs per cluster (portable size)
+constexpr int kSmemLimitRoute = 227 * 1024;
+
+struct RouteParams {
+    const float *w;  // [n_exp][n_embd]
+    const float *x;  // [n_tok][n_embd]
+    int n_tok, n_embd, n_exp, n_used;
+    int32_t *ids;    // [n_tok][n_used]
+    float *route_w;  // [n_tok][n_used]
+    double *logits;  // [n_tok][n_exp] or nullptr
+    int off_lg;      // shared-memory offsets (bytes)
+    int off_sel;
+};
+
+// Larger logit first; equal logits by the lower expert index (a total order
+// on (value, index); NaN logits count as -infinity, so the order stays total).
+__device__ __forceinline__ bool route_before(double a, int ia, double b, int ib) {
+    return a > b || (a == b && ia < ib);
+}
+
+__global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_constant__ RouteParams p) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const int C = (int)cluster.num_blocks();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = (int)(blockIdx.x / C) * kRouteTok;
+    const int nt = min(kRouteTok, p.n_tok - t0);
+    float *xs = reinterpret_cast<float *>(smem);
+    double *lg = reinterpret_cast<double *>(smem + p.off_lg);  // [kRouteTok][n_exp], own experts only
+    griddep_wait();  // x may come from the preceding kernel
+    griddep_launch_dependents();
+    const int n4 = p.n_embd / 4;
+    for (int i = threadIdx.x; i < nt * n4; i += kRouteThreads) {
+        const int t = i / n4, c = i - t * n4;
+        reinterpret_cast<float4 *>(xs)[t * n4 + c] =
+            reinterpret_cast<const float4 *>(p.x + (int64_t)(t0 + t) * p.n_embd)[c];
+    }
+    __syncthreads();
+    // logits of this CTA's experts: warp per expert row
+    for (int e = rank + C * warp; e < p.n_exp; e += C * kRouteWarps) {
+        const float4 *wr = reinterpret_cast<const float4 *>(p.w + (int64_t)e * p.n_embd);
+        double acc[kRouteTok];
+#pragma unroll
+        for (int t = 0; t < kRouteTok; ++t) acc[t] = 0.0;
+        for (int c = lane; c < n4; c += 32) {
+            const float4 wv = __ldg(wr + c);
+#pragma unroll
+            for (int t = 0; t < kRouteTok; ++t) {
+                if (t < nt) {
+                    const float4 xv = reinterpret_cast<const float4 *>(xs)[t * n4 + c];
+                    acc[t] = fma((double)wv.x, (double)xv.x, acc[t]);
+                    acc[t] = fma((double)wv.y, (double)xv.y, acc[t]);
+                    acc[t] = fma((double)wv.z, (double)xv.z, acc[t]);
+                    acc[t] = fma((double)wv.w, (double)xv.w, acc[t]);
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < kRouteTok; ++t) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+        }
+        if (lane == 0)
+            for (int t = 0; t < nt; ++t) lg[t * p.n_exp + e] = acc[t];
+    }
+    if (p.logits) {
+        for (int i = threadIdx.x; i < nt * p.n_exp; i += kRouteThreads) {
+            const int t = i / p.n_exp, e = i - t * p.n_exp;
+            if (e % C == rank) p.logits[(int64_t)(t0 + t) * p.n_exp + e] = lg[i];
+        }
+    }
+    cluster.sync();  // every CTA's logits are written (release / acquire)
+    if (rank == 0) {
+        // gather the other CTAs' logits into this CTA's array (each expert's
+        // slot is written by exactly one CTA), NaN as -infinity
+        for (int i = threadIdx.x; i < nt * p.n_exp; i += kRouteThreads) {
+            const int e = i % p.n_exp;
+            const double v = e % C == 0 ? lg[i] : cluster.map_shared_rank(lg, e % C)[i];
+            lg[i] = v != v ? -INFINITY : v;
+        }
+        __syncthreads();
+    }
+    cluster.sync();  // CTA 0 is done reading the others' shared memory
+    if (rank == 0 && warp < nt) {
+        // token t0 + warp: repeated warp argmax over the not-yet-selected experts
+        const int t = warp;
+        unsigned char *sel = smem + p.off_sel + t * p.n_exp;
+        for (int e = lane; e < p.n_exp; e += 32) sel[e] = 0;
+        __syncwarp();
+        auto logit = [&](int e) -> double { return lg[t * p.n_exp + e]; };
+        double first = 0.0, mine = -INFINITY;  // lane k keeps the k-th selected logit
+        for (int k = 0; k < p.n_used; ++k) {
+            double bv = -INFINITY;
+            int bi = p.n_exp;  // no candidate yet
+            for (int e = lane; e < p.n_exp; e += 32) {
+                if (sel[e]) continue;
+                const double v = logit(e);
+                if (bi == p.n_exp || route_before(v, e, bv, bi)) {
+                    bv = v;
+                    bi = e;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (oi < p.n_exp && (bi == p.n_exp || route_before(ov, oi, bv, bi))) {
+                    bv = ov;
+                    bi = oi;
+                }
+            }
+            // n_used <= n_exp: some expert is always left, so bi < n_exp
+            if (lane == 0) {
+                sel[bi] = 1;
+                p.ids[(int64_t)(t0 + t) * p.n_used + k] = bi;
+            }
+            if (k == 0) first = bv;
+            if (lane == k) mine = bv;
+            __syncwarp();
+        }
+        // softmax over the selected logits (largest first), fp64
+        const double ex = lane < p.n_used ? exp(mine - first) : 0.0;
+        double sum = ex;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane < p.n_used) p.route_w[(int64_t)(t0 + t) * p.n_used + lane] = (float)(ex / sum);
+    }
+}
+
+}  // namespace q8
+
+using namespace q8;
+
+extern "C" q8_status q8_route(const float *w_router, const float *x, int64_t n_tok,
+                              int64_t n_embd, int64_t n_exp, int32_t n_used, int32_t *ids,
+                              float *route_w, double *logits, void *stream) {
+    const char *fn = "q8_route";
+    Q8_REQUIRE(w_router && x && ids && route_w, Q8_E_NULL, "%s: NULL pointer", fn);
+    Q8_REQUIRE(n_tok >= 1 && n_tok <= (1LL << 24), Q8_E_SHAPE, "%s: n_tok=%lld", fn,
+               (long long)n_tok);
+    Q8_REQUIRE(n_embd >= 4 && n_embd % 4 == 0 && n_embd <= Q8_MAX_K, Q8_E_SHAPE,
+               "%s: n_embd=%lld must be a multiple of 4 in [4, %d]", fn, (long long)n_embd,
+               Q8_MAX_K);
+    Q8_REQUIRE(n_exp >= 1 && n_exp <= Q8_ROUTE_MAX_EXP, Q8_E_SHAPE, "%s: n_exp=%lld (1..%d)", fn,
+               (long long)n_exp, Q8_ROUTE_MAX_EXP);
+    Q8_REQUIRE(n_used >= 1 && n_used <= Q8_MAX_USED && n_used <= n_exp, Q8_E_SHAPE,
+               "%s: n_used=%d (1..min(n_exp, %d))", fn, n_used, Q8_MAX_USED);
+    Q8_REQUIRE(aligned16(w_router) && aligned16(x), Q8_E_ALIGN,
+               "%s: w_router and x must be 16-byte aligned", fn);
+    Q8_REQUIRE(((uintptr_t)ids & 3u) == 0 && ((uintptr_t)route_w & 3u) == 0 &&
+                   ((uintptr_t)logits & 7u) == 0,
+               Q8_E_ALIGN, "%s: ids/route_w/logits misaligned", fn);
+    RouteParams p{};
+    p.w = w_router;
+    p.x = x;
+    p.n_tok = (int)n_tok;
+    p.n_embd = (int)n_embd;
+    p.n_exp = (int)n_exp;
+    p.n_used = n_used;
+    p.ids = ids;
+    p.route_w = route_w;
+    p.logits = logits;
+    const int C = kRouteCluster;
+    const int x_bytes = kRouteTok * (int)n_embd * 4;
+    p.off_lg = (x_bytes + 15) / 16 * 16;
+    const int lg_bytes = kRouteTok * (int)n_exp * 8;
+    p.off_sel = p.off_lg + lg_bytes;
+    const int smem = p.off_sel + kRouteTok * (int)n_exp;
+    Q8_REQUIRE(smem <= kSmemLimitRoute, Q8_E_UNSUPPORTED, "%s: shared-memory plan too large", fn);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        Q8_FAIL(Q8_E_CUDA, "%s: no current device", fn);
+    if (!smem_opted_in((const void *)route_kernel, dev)) {
+        cudaError_t e = cudaFuncSetAttribute(route_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSmemLimitRoute);
+        if (e != cudaSuccess)
+            Q8_FAIL(Q8_E_CUDA, "%s: shared-memory attribute: %s", fn, cudaGetErrorString(e));
+        set_smem_opted_in((const void *)route_kernel, dev);
+    }
+    const int groups = (int)((n_tok + kRouteTok - 1) / kRouteTok);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(groups * C));
+    cfg.blockDim = dim3(kRouteThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = (cudaStream_t)stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, route_kernel, p);
+    if (e != cudaSuccess) Q8_FAIL(Q8_E_CUDA, "%s: launch: %s", fn, cudaGetErrorString(e));
+    return Q8_OK;
+}

@@ -575,35 +575,55 @@ __device__ __forceinline__ void stage_f32(const XStage &xs, const float *__restr
     }
 }
 
+// Quantize n fp32 rows held in shared memory (row j at src + arow(j) * k)
+// into the stage by the Q8_0 rule, eight threads per 32-block: thread i of an
+// aligned group of eight takes elements 4i..4i+3, the block's amax comes from
+// three xor shuffles inside the group, and each thread quantizes its own four
+// values.  Every element goes through the same operations as in the
+// one-thread form (amax is an exact maximum), so the bits are the same; the
+// dependent chain per thread is a quarter as long.  tid/nthr: this thread's
+// index among the nthr threads (whole warps) that share the work.
+template <class RowFn>
+__device__ __forceinline__ void stage_f32_smem8(const XStage &xs, const float *src, int k, int n,
+                                                RowFn arow, int tid, int nthr) {
+    const int nb = k / QK;
+    const int total = n * nb;
+    const int grp = tid >> 3, part = tid & 7;
+    const int ngrp = nthr >> 3;
+    for (int base = 0; base < total; base += ngrp) {  // the same trip count in every lane
+        const int blk = base + grp;
+        const bool live = blk < total;
+        int j = 0, b = 0;
+        float4 f = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (live) {
+            j = blk / nb;
+            b = blk - j * nb;
+            f = reinterpret_cast<const float4 *>(src + (size_t)arow(j) * k + b * QK)[part];
+        }
+        float amax = fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w)));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+        if (live) {
+            const float d32 = block_scale(amax);
+            const float id = block_inv_scale(d32);
+            const uint32_t w = ((uint32_t)quantize_one(f.x, id) & 0xffu) |
+                               (((uint32_t)quantize_one(f.y, id) & 0xffu) << 8) |
+                               (((uint32_t)quantize_one(f.z, id) & 0xffu) << 16) |
+                               (((uint32_t)quantize_one(f.w, id) & 0xffu) << 24);
+            *reinterpret_cast<uint32_t *>(xs.q + (size_t)j * k + b * QK + 4 * part) = w;
+            if (part == 0) xs.dx[(size_t)j * nb + b] = scale_value(scale_bits(d32));
+        }
+    }
+}
+
 // Quantize the n fp32 rows of the raw slot (row j at raw + j * k) into the
-// stage: stage_f32's rule, from shared memory, one consumer thread per block
-// (no cross-lane steps, so a thread's blocks are independent chains).
-// tid/nthr: this thread's index among the nthr threads that share the work
-// (default: the consumer threads).
+// stage (stage_f32_smem8).  tid/nthr: this thread's index among the nthr
+// threads (whole warps) that share the work (default: the consumer threads).
 __device__ __forceinline__ void stage_f32_raw(const XStage &xs, const float *raw, int k, int n,
                                               int tid = -1, int nthr = kCT) {
-    const int nb = k / QK;
-    if (tid < 0) tid = threadIdx.x;
-    for (int blk = tid; blk < n * nb; blk += nthr) {
-        const int j = blk / nb;
-        const int b = blk - j * nb;
-        const float4 *src = reinterpret_cast<const float4 *>(raw + (size_t)j * k + b * QK);
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float4 f = src[i];
-            v[4 * i] = f.x;
-            v[4 * i + 1] = f.y;
-            v[4 * i + 2] = f.z;
-            v[4 * i + 3] = f.w;
-        }
-        uint32_t q[8];
-        const float d32 = quantize_block_thread(v, q);
-        uint4 *dst = reinterpret_cast<uint4 *>(xs.q + (size_t)j * k + b * QK);
-        dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
-        dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
-        xs.dx[(size_t)j * nb + b] = scale_value(scale_bits(d32));
-    }
+    stage_f32_smem8(xs, raw, k, n, [](int j) { return j; }, tid < 0 ? (int)threadIdx.x : tid,
+                    nthr);
 }
 
 // Consumer side of an activation job of nx rows (fp32 af, rows arow(j)):

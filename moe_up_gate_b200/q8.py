@@ -48,7 +48,7 @@ EXPORTS = ["q8_scale_stride", "q8_pack", "q8_pack_up_gate", "q8_quantize_row", "
            "q8_status_string", "q8_last_error", "q8_moe_group",
            "q8_moe_up_gate_swiglu_pregrouped", "q8_mul_mat_id_pregrouped",
            "q8_moe_up_gate_swiglu_noalloc", "q8_moe_up_gate_swiglu_fp32", "q8_mul_mat_id_fp32",
-           "q8_reset_errors", "q8_debug_wait_timeout"]
+           "q8_reset_errors", "q8_debug_wait_timeout", "q8_route"]
 
 
 def lib_path() -> str:
@@ -96,6 +96,7 @@ def load(auto_build: bool = True):
             "q8_moe_up_gate_swiglu_fp32": (st, [P(_Tensor), vp, i64, vp, i32, vp, vp, vp]),
             "q8_mul_mat_id_fp32": (st, [P(_Tensor), vp, i32, i64, vp, i32, vp, vp, vp]),
             "q8_reset_errors": (st, []),
+            "q8_route": (st, [vp, vp, i64, i64, i64, i32, vp, vp, vp, vp]),
             "q8_debug_wait_timeout": (st, [i32, i64, vp, vp]),
             "q8_status_string": (ctypes.c_char_p, [st]),
             "q8_last_error": (ctypes.c_char_p, []),
@@ -370,6 +371,22 @@ def moe_ffn(up_gate: Q8Tensor, down: Q8Tensor, x, ids=None, route_w=None, ws=Non
 
 def check(ws, stream=None):
     _call("q8_check", _ptr(ws), _stream(stream))
+
+
+def route(w_router, x, n_used: int, want_logits=False, ids=None, route_w=None, stream=None):
+    """Router: fp32 w_router [n_exp, n_embd], x [n_tok, n_embd] -> (ids int32
+    [n_tok, n_used], route_w fp32 [n_tok, n_used][, logits fp64 [n_tok, n_exp]])."""
+    n_tok, n_embd = x.shape
+    n_exp = w_router.shape[0]
+    if ids is None:
+        ids = torch.empty((n_tok, n_used), dtype=torch.int32, device=x.device)
+    if route_w is None:
+        route_w = torch.empty((n_tok, n_used), dtype=torch.float32, device=x.device)
+    logits = (torch.empty((n_tok, n_exp), dtype=torch.float64, device=x.device)
+              if want_logits else None)
+    _call("q8_route", _ptr(w_router), _ptr(x), n_tok, n_embd, n_exp, n_used, _ptr(ids),
+          _ptr(route_w), _ptr(logits), _stream(stream))
+    return (ids, route_w, logits) if want_logits else (ids, route_w)
 
 
 def reset_errors():

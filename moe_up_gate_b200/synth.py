@@ -29,6 +29,8 @@ experts per token):
   3  dense up_gate [4096 -> 2*14336] + down [14336 -> 4096], 1 and 8 tokens
   4  MoE layer: n_embd 2816, n_ff 704, 128 experts, top-8, 1 and 16 tokens
   5  30 MoE layers of workload 4's shape, 1/4/16/64/256 tokens
+  (and the feed-forward layers of workload 2 with separate gate (w1) and up
+  (w3) weights packed into one combined up/gate tensor: llama_ffn_tensors)
 """
 from __future__ import annotations
 
@@ -104,6 +106,21 @@ def llama_matvec_set():
             out.append((f"l{layer}.{name}", rows, k))
     out.append(("classifier", LLAMA_VOCAB, d))
     return out
+
+
+LLAMA_FFN = MoeShape(n_embd=LLAMA_DIM, n_ff=LLAMA_HIDDEN, n_exp=1, n_used=1)
+
+
+def llama_ffn_tensors(layer: int, n_tok: int, device="cpu"):
+    """fp32 tensors of one Llama-2-110M-shaped feed-forward layer with separate
+    gate and up weights: w1 (gate) and w3 (up) [2048, 768], w2 (down)
+    [768, 2048], x [n_tok, 768] ~ N(0, 1); the seeds of the w1, w3, w2
+    matvecs of the decode set's layer (workload 2, tensors 4, 5, 6)."""
+    w1 = normal((LLAMA_HIDDEN, LLAMA_DIM), seed_of(2, layer, 4), W_STD, device)
+    w3 = normal((LLAMA_HIDDEN, LLAMA_DIM), seed_of(2, layer, 5), W_STD, device)
+    w2 = normal((LLAMA_DIM, LLAMA_HIDDEN), seed_of(2, layer, 6), W_STD, device)
+    x = normal((n_tok, LLAMA_DIM), seed_of(2, layer, 7), 1.0, device)
+    return dict(w1=w1, w3=w3, w2=w2, x=x)
 
 
 def moe_layer_tensors(c: int, layer: int, shape: MoeShape, n_tok: int, x_std: float,

@@ -180,3 +180,25 @@ def test_noalloc_scratch_capacity(q8):
     lib = q8.load()
     assert lib.q8_moe_workspace_size(1982, 8, 128) <= 65536
     assert lib.q8_moe_workspace_size(1983, 8, 128) > 65536
+
+
+def test_route_validation(q8):
+    lib = q8.load()
+    ok = dict(n_tok=2, n_embd=64, n_exp=16, n_used=4)
+
+    def call(w=FAKE, x=FAKE, ids=FAKE, rw=FAKE, lg=None, **kw):
+        a = dict(ok, **kw)
+        return lib.q8_route(w, x, a["n_tok"], a["n_embd"], a["n_exp"], a["n_used"], ids, rw, lg,
+                            None)
+
+    assert call(w=None) == 1
+    assert call(ids=None) == 1
+    assert call(n_tok=0) == 2
+    assert call(n_embd=62) == 2                 # not a multiple of 4
+    assert call(n_exp=0) == 2
+    assert call(n_exp=1025) == 2                # above Q8_ROUTE_MAX_EXP
+    assert call(n_used=17, n_exp=16) == 2       # more than the experts
+    assert call(n_used=33, n_exp=64) == 2       # above Q8_MAX_USED
+    assert call(x=FAKE_ODD) == 3
+    assert call(lg=ctypes.c_void_p(0x10004)) == 3  # logits 8-byte aligned
+    assert call(n_embd=16384, n_exp=1024) == 5  # shared-memory plan too large

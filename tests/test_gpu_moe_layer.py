@@ -4,7 +4,7 @@ SwiGLU, grid barrier, down projection + combine).  Its output must be bitwise
 the chain of separate calls (same row sums, same h quantization, same combine
 order), whose stages are pinned to the oracle elsewhere; here the down outputs
 are also held to the oracle with P3 on sampled rows, the barrier words must be
-left at zero, repeated calls must agree, and bad ids must be reported."""
+left on a multiple of the grid size, repeated calls must agree, and bad ids must be reported."""
 import numpy as np
 import pytest
 import torch
@@ -51,7 +51,7 @@ def test_fused_layer_equals_chain(n_exp, n_ff, n_embd, n_tok, n_used):
     q8.check(ws)
     ref, r, y = _chain(UG, DN, x, ids, p)
     assert torch.equal(out, ref)
-    # again with the same workspace: the barrier words were left at zero
+    # again with the same workspace: the barrier counter was left on a multiple of the grid
     out2 = q8.moe_ffn(UG, DN, x, ids, p, ws=ws)
     assert torch.equal(out2, out)
     # P3 on the down outputs of sampled rows against the oracle (from the
@@ -79,7 +79,8 @@ def test_fused_layer_equals_chain(n_exp, n_ff, n_embd, n_tok, n_used):
 
 def test_fused_layer_many_calls_one_workspace():
     """Layers of a decode step reuse one workspace back to back (the grid
-    barrier's generation keeps counting, its arrival word returns to 0)."""
+    barrier's arrival counter keeps counting, a multiple of the grid between
+    calls)."""
     t, UG, DN, ids, p = _layer(128, 704, 2816, 1, 8, seed=931)
     x = t["x"].to(DEV)
     ws = q8.moe_ffn_workspace(1, 8, 128, 2816, 704, DEV)

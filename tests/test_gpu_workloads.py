@@ -179,3 +179,50 @@ def test_config5_sweep_layers(T):
     _issue_and_check(wl, sorted({0, T // 2, T - 1}))
     if T == synth.MOE_SWEEP_TOKENS[-1]:
         _SWEEP_PACKED.clear()
+
+
+def test_llama_ffn_separate_gate_up_fused():
+    """The Llama-2-110M feed-forward layers with separate gate (w1) and up
+    (w3) weights: packed once into the combined up/gate tensor, they run as
+    one dense fused up/gate + SwiGLU per layer, then w2.  h is held to the
+    oracle's separate-weights path (two GEMVs, then silu(g) * u), the down
+    projection to P3 on the oracle's quantization of the GPU's h."""
+    wl = bench.MoeWorkload(DEV, "llama2_110m_ffn", 1, layer_ids=[0, 11])
+    D, F = synth.LLAMA_DIM, synth.LLAMA_HIDDEN
+    wl.h.fill_(float("nan"))
+    wl.out.fill_(float("nan"))
+    hs = []
+    # the workload shares one h buffer across layers: issue layer by layer
+    for li, l in enumerate(wl.layer_ids):
+        UG, DN = wl.L[li]
+        t = synth.llama_ffn_tensors(l, 1, device=DEV)
+        gq, gd = oracle.quantize_rows(t["w1"].cpu().numpy())
+        uq, ud = oracle.quantize_rows(t["w3"].cpu().numpy())
+        # P1: the combined tensor holds the gate rows, then the up rows
+        assert np.array_equal(host(UG.qs)[:F], gq) and np.array_equal(host(UG.qs)[F:], uq)
+        assert np.array_equal(canon_d(UG.d, D)[:F], gd) and np.array_equal(canon_d(UG.d, D)[F:], ud)
+        x = wl.x[0][li]
+        assert torch.equal(x.cpu(), t["x"].cpu())
+        h = q8.moe_up_gate_swiglu_fp32(UG, x, None)
+        out = torch.full((1, D), float("nan"), device=DEV)
+        q8.gemv_batched([(DN, h.reshape(1, F), out)], n_tok=1)
+        torch.cuda.synchronize()
+        xq, xd = oracle.quantize_rows(t["x"].cpu().numpy())
+        h_ref, g_ref, u_ref = oracle.up_gate_swiglu_split(gq, gd, uq, ud, xq, xd, None,
+                                                          want_gu=True)
+        Sg = S_norm(gq, gd, xq, xd)
+        Su = S_norm(uq, ud, xq, xd)
+        bound = _h_bound(g_ref[:, 0], u_ref[:, 0], h_ref[:, 0], Sg, Su)
+        assert np.all(np.abs(host(h).reshape(1, F) - h_ref[:, 0]) <= bound)
+        hq, hd = oracle.quantize_rows(host(h).reshape(1, F))
+        dq, dd = oracle.quantize_rows(t["w2"].cpu().numpy())
+        assert np.array_equal(host(DN.qs), dq)
+        y_ref = oracle.gemv(dq, dd, hq, hd)
+        assert_p3(host(out), y_ref, S_norm(dq, dd, hq, hd), f"w2 layer {l}")
+        hs.append(out)
+    # the workload's own step gives the same outputs (the last layer's h is
+    # the shared buffer's final content)
+    wl.issue(0, bench.NoMarks())
+    torch.cuda.synchronize()
+    for li in range(len(wl.layer_ids)):
+        assert torch.equal(wl.out[li], hs[li])
