@@ -100,20 +100,19 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
         if (lane == 0)
             for (int t = 0; t < nt; ++t) lg[t * p.n_exp + e] = acc[t];
     }
+    cluster.sync();  // every CTA's logits are written (release / acquire)
     if (p.logits) {
         for (int i = threadIdx.x; i < nt * p.n_exp; i += kRouteThreads) {
             const int t = i / p.n_exp, e = i - t * p.n_exp;
             if (e % C == rank) p.logits[(int64_t)(t0 + t) * p.n_exp + e] = lg[i];
         }
     }
-    cluster.sync();  // every CTA's logits are written (release / acquire)
     if (rank == 0) {
         // gather the other CTAs' logits into this CTA's array (each expert's
-        // slot is written by exactly one CTA), NaN as -infinity
+        // slot is written by exactly one CTA; this CTA's own slots stay)
         for (int i = threadIdx.x; i < nt * p.n_exp; i += kRouteThreads) {
             const int e = i % p.n_exp;
-            const double v = e % C == 0 ? lg[i] : cluster.map_shared_rank(lg, e % C)[i];
-            lg[i] = v != v ? -INFINITY : v;
+            if (e % C != 0) lg[i] = cluster.map_shared_rank(lg, e % C)[i];
         }
         __syncthreads();
     }
@@ -124,7 +123,10 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
         unsigned char *sel = smem + p.off_sel + t * p.n_exp;
         for (int e = lane; e < p.n_exp; e += 32) sel[e] = 0;
         __syncwarp();
-        auto logit = [&](int e) -> double { return lg[t * p.n_exp + e]; };
+        auto logit = [&](int e) -> double {  // NaN ranks as -infinity
+            const double v = lg[t * p.n_exp + e];
+            return v != v ? -INFINITY : v;
+        };
         double first = 0.0, mine = -INFINITY;  // lane k keeps the k-th selected logit
         for (int k = 0; k < p.n_used; ++k) {
             double bv = -INFINITY;
