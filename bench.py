@@ -5,9 +5,8 @@ Default workload: one single-token decode step of the Llama-2-110M-shaped Q8_0
 matvec set (12 layers x {wq, wk, wv, wo 768x768, w1, w3 2048x768, w2 768x2048}
 + classifier 32000x768, 85 matvecs, batch 1), the Q8_0 int8 decode that the
 "narray-llm" README measures.  Every matvec gets its own seeded N(0,1) x and
-the set runs as one step: one q8_gemv_batched launch with its scheduling
-workspace (each problem quantizes its x to Q8_0 inside the kernel, then
-streams its weights).  The default run also reports the fused MoE
+the set runs as one step: one q8_gemv_batched launch (each problem quantizes
+its x to Q8_0 inside the kernel, then streams its weights).  The default run also reports the fused MoE
 feed-forward step on its own workloads (moe_subrecords).
 
 Other workloads (--workload): gemv_768, dense_ffn (--tokens 1|8),
@@ -224,7 +223,7 @@ class NoMarks:
 class LlamaDecode:
     """85 Q8_0 matvecs of one Llama-2-110M-shaped decode step, one batched launch."""
     name = "llama2_110m_q8_decode"
-    kernel = "gemv_dyn_kernel"
+    kernel = "gemv_batched_kernel"
 
     def __init__(self, dev, tokens=None, gemv768=False, host_only=False):
         import torch
@@ -273,8 +272,6 @@ class LlamaDecode:
         self.x = self.x_host.to(dev)
         self.y = [torch.empty((1, rows), dtype=torch.float32, device=dev) for _, rows, _ in mats]
         self.out_host = torch.empty(mats[-1][1], dtype=torch.float32).pin_memory()
-        # the scheduling workspace of q8_gemv_batched (chunks taken from a counter)
-        self.gemv_ws = q8.gemv_workspace(dev)
         packed = []
         for (_, rows, k), (ws, _) in zip(mats, seeds):
             w = synth.normal((rows, k), ws, std=synth.W_STD, device=dev)
@@ -296,7 +293,7 @@ class LlamaDecode:
         W = self.W[i % self.copies]
         probs = [(Wm, self.x[off:off + Wm.k], y) for Wm, off, y in zip(W, self.offs, self.y)]
         marks.begin()
-        self.q8.gemv_batched(probs, n_tok=1, ws=self.gemv_ws)
+        self.q8.gemv_batched(probs, n_tok=1)
         marks.end()
 
     def unique_bytes(self, i):
@@ -453,7 +450,6 @@ class MoeWorkload:
         self.ids = [ih.to(dev) for ih in self.ids_host]
         self.p = [ph.to(dev) for ph in self.p_host]
         self.ws = q8.moe_workspace(tokens, Uu, E, dev) if self.routed else None
-        self.gemv_ws = q8.gemv_workspace(dev)
         self.xq = torch.empty((tokens, D), dtype=torch.int8, device=dev)
         self.xd = torch.empty((tokens, D // 32), dtype=torch.float16, device=dev)
         self.h = torch.empty((P, F), dtype=torch.float32, device=dev)
@@ -514,7 +510,7 @@ class MoeWorkload:
                     marks.begin()
                     q8.moe_up_gate_swiglu_fp32(UG, x, None, h=self.h)
                     marks.end()
-                    q8.gemv_batched([(DN, self.h, self.out[l])], n_tok=T, ws=self.gemv_ws)
+                    q8.gemv_batched([(DN, self.h, self.out[l])], n_tok=T)
             return
         for l, (UG, DN) in enumerate(layers):
             x = self.x[s][l]

@@ -35,6 +35,7 @@ constexpr int kRouteTok = 4;         // tokens per cluster
 constexpr int kRouteThreads = 256;   // 8 warps
 constexpr int kRouteWarps = kRouteThreads / 32;
 constexpr int kRouteCluster = 8;     // CTAs per cluster (portable size)
+constexpr int kRouteUnroll = 8;      // router-row loads in flight per lane
 constexpr int kSmemLimitRoute = 227 * 1024;
 
 struct RouteParams {
@@ -79,16 +80,26 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
         double acc[kRouteTok];
 #pragma unroll
         for (int t = 0; t < kRouteTok; ++t) acc[t] = 0.0;
-        for (int c = lane; c < n4; c += 32) {
-            const float4 wv = __ldg(wr + c);
+        // kRouteUnroll row loads in flight per lane, then their products in
+        // order (a fixed order per n_embd: the sums are deterministic)
+        for (int c0 = lane; c0 < n4; c0 += 32 * kRouteUnroll) {
+            float4 wv[kRouteUnroll];
 #pragma unroll
-            for (int t = 0; t < kRouteTok; ++t) {
-                if (t < nt) {
-                    const float4 xv = reinterpret_cast<const float4 *>(xs)[t * n4 + c];
-                    acc[t] = fma((double)wv.x, (double)xv.x, acc[t]);
-                    acc[t] = fma((double)wv.y, (double)xv.y, acc[t]);
-                    acc[t] = fma((double)wv.z, (double)xv.z, acc[t]);
-                    acc[t] = fma((double)wv.w, (double)xv.w, acc[t]);
+            for (int u = 0; u < kRouteUnroll; ++u)
+                wv[u] = c0 + 32 * u < n4 ? __ldg(wr + c0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < kRouteUnroll; ++u) {
+                const int c = c0 + 32 * u;
+                if (c >= n4) break;
+#pragma unroll
+                for (int t = 0; t < kRouteTok; ++t) {
+                    if (t < nt) {
+                        const float4 xv = reinterpret_cast<const float4 *>(xs)[t * n4 + c];
+                        acc[t] = fma((double)wv[u].x, (double)xv.x, acc[t]);
+                        acc[t] = fma((double)wv[u].y, (double)xv.y, acc[t]);
+                        acc[t] = fma((double)wv[u].z, (double)xv.z, acc[t]);
+                        acc[t] = fma((double)wv[u].w, (double)xv.w, acc[t]);
+                    }
                 }
             }
         }
