@@ -684,7 +684,6 @@ def gpu_id(local_rank: int) -> str:
 # of them changes)
 KERNEL_SOURCES = {
     "gemv_batched_kernel": ["q8_matmul.cu"],
-    "gemv_dyn_kernel": ["q8_matmul.cu"],
     "route_kernel": ["q8_route.cu"],
     "up_gate_kernel": ["q8_moe.cu"],
     "moe_layer_kernel": ["q8_layer.cu"],

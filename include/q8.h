@@ -167,25 +167,15 @@ q8_status q8_gemv(const q8_tensor *W, const int8_t *xq, const uint16_t *xd, int6
  *  descs: HOST array of n_desc problems (copied into the launch parameters;
  *         the array may be reused as soon as the call returns).
  *  n_desc: 1 .. Q8_MAX_GEMV_DESC.  n_tok: activation rows per problem, >= 1.
- *  ws, ws_bytes: optional scheduling workspace (device, 16-byte aligned, at
- *         least Q8_GEMV_WS_BYTES, zero-filled before its first use; NULL for
- *         none).  With it, the CTAs take the problems' tiles in chunks from a
- *         counter there, so that all of them finish together; without it each
- *         CTA has a fixed run of tiles.  The outputs are the same bits either
- *         way.  Every call leaves the counter at zero; a call that overlaps
- *         another on the GPU needs its own workspace (calls in order on one
- *         stream may share one).  After a wait timeout reported by q8_check,
- *         zero it again.
  */
-#define Q8_GEMV_WS_BYTES 256
 typedef struct {
     q8_tensor W;      /* n_mat == 1                                  */
     const float *x;   /* fp32 [n_tok][W.k], 16-byte aligned          */
     float *y;         /* out fp32 [n_tok][W.rows]                    */
 } q8_gemv_desc;
 
-q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_tok, void *ws,
-                          size_t ws_bytes, void *stream);
+q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_tok,
+                          void *stream);
 
 /*
  * Workspace for the routed (MoE) calls: expert grouping tables and the

@@ -527,170 +527,6 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
 }
 
 // ---------------------------------------------------------------------------
-// Batched GEMV with a dynamic schedule.  The tiles of every problem are cut
-// into chunks (a chunk never spans two problems; chunks get smaller towards
-// the end of the list).  CTA b starts with chunk b; after that every CTA
-// takes the next chunk from a counter in the caller's workspace, one atomic
-// ahead, so CTAs that the memory system serves faster take more of the work
-// and all of them finish together.  The producer writes each stage's tile
-// (problem, tile) into a header word next to the ring barriers; after the
-// last chunk it marks the next stage as the end.  The consumers follow the
-// headers.  Row sums are those of the static kernel (the order depends only
-// on k), so the outputs are bitwise the same.  The last CTA to finish puts
-// the counters back to zero for the next call on the same stream (a call
-// touches them only after its grid-dependency wait).
-// ---------------------------------------------------------------------------
-constexpr int kGemvChunkMax = 4096;
-constexpr int kGemvDynMaxGrid = 512;
-constexpr int kStageHdrOff = 2 * kMaxStages * 8 + 16;  // after the ring's barriers
-static_assert(kStageHdrOff + kMaxStages * 4 <= 256, "header area");
-
-struct GemvChunk {
-    uint8_t problem;
-    uint8_t ntiles;
-    uint16_t first;  // first tile within the problem
-};
-
-struct GemvDynParams {
-    int n_desc;
-    int n_tok;
-    int n_chunks;
-    int grid;
-    unsigned *ws;  // [0] chunks taken after the static ones, [1] finished CTAs
-    Plan plan;
-    GemvProblem pr[Q8_MAX_GEMV_DESC];
-    GemvChunk ch[kGemvChunkMax];
-};
-
-template <int NT>
-__global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
-    gemv_dyn_kernel(const __grid_constant__ GemvDynParams p) {
-    extern __shared__ __align__(128) unsigned char smem[];
-    Q8_TRACE(0);
-    const Ring R = ring_init(smem, p.plan);
-    int *hdr = reinterpret_cast<int *>(smem + kStageHdrOff);
-    Q8_TRACE(1);
-    griddep_launch_dependents();
-    if ((threadIdx.x >> 5) == kCW) {
-        if ((threadIdx.x & 31) == 0) {
-            // the activations and the counter may be written by the preceding
-            // grid; the activation rows go first, then the weights
-            griddep_wait();
-            Q8_TRACE(20);
-            int c = blockIdx.x, it = 0, cur = -1;
-            XJobs J;
-            while (c < p.n_chunks) {
-                const unsigned nxt = atomicAdd(p.ws, 1u);  // used once this chunk is issued
-                const GemvChunk ch = p.ch[c];
-                const GemvProblem &q = p.pr[ch.problem];
-                const Geo g = geo_for_k(q.k, NT);
-                if (R.raw_rows > 0 && ch.problem != cur)
-                    produce_job(R, J, ch.problem, 0, p.n_tok, q.k,
-                                [&](int j) { return q.x + (int64_t)j * q.k; }, &g_err_matmul);
-                cur = ch.problem;
-                for (int i = 0; i < ch.ntiles; ++i, ++it) {
-                    const int s = it % R.stages, round = it / R.stages;
-                    if (round > 0) mbar_wait(&R.empty[s], (round - 1) & 1, &g_err_matmul);
-                    Q8_TRACE(21);
-                    const int tile = ch.first + i;
-                    const int r0 = tile * g.nr;
-                    const int rows = min(g.nr, q.rows - r0);
-                    hdr[s] = (ch.problem << 16) | tile;
-                    const uint32_t qb = (uint32_t)(rows * q.k), db = (uint32_t)(rows * q.ld_d * 2);
-                    mbar_arrive_expect_tx(&R.full[s], qb + db);
-                    bulk_g2s(R.qs(s), q.wq + (int64_t)r0 * q.k, qb, &R.full[s]);
-                    bulk_g2s(R.d(s), q.wd + (int64_t)r0 * q.ld_d, db, &R.full[s]);
-                }
-                c = p.grid + (int)nxt;
-            }
-            // the end marker: a stage with no copies
-            const int s = it % R.stages, round = it / R.stages;
-            if (round > 0) mbar_wait(&R.empty[s], (round - 1) & 1, &g_err_matmul);
-            hdr[s] = -1;
-            mbar_arrive(&R.full[s]);
-            Q8_TRACE(22);
-        }
-        return;
-    }
-    griddep_wait();
-    Q8_TRACE(2);
-    const XStage xs{reinterpret_cast<int8_t *>(smem + p.plan.off_xq),
-                    reinterpret_cast<float *>(smem + p.plan.off_xd)};
-    float *part0 = reinterpret_cast<float *>(smem + p.plan.off_part);
-    const int nx = p.n_tok;  // one activation group (nx <= the stage's rows)
-    int buf = 0, staged = -1;
-    XJobs J;
-    bool unsynced = false;  // passes without a barrier since the last one
-    for (int it = 0;; ++it) {
-        const int s = it % R.stages;
-        mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_matmul);
-        Q8_TRACE(6);
-        const int h = hdr[s];
-        if (h < 0) break;
-        const int prob = h >> 16, tile = h & 0xffff;
-        const GemvProblem &q = p.pr[prob];
-        const Geo g = geo_for_k(q.k, NT);
-        const int r0 = tile * g.nr;
-        const int rows_valid = min(g.nr, q.rows - r0);
-        if (prob != staged) {
-            // after passes without a barrier every warp must be done with the
-            // staged rows before they are replaced
-            if (unsynced) named_bar_sync(kBarConsumers, kCT);
-            unsynced = false;
-            stage_job_f32(R, J, xs, q.x, q.k, nx, [&](int j) { return j; }, &g_err_matmul);
-            named_bar_sync(kBarConsumers, kCT);
-            Q8_TRACE(7);
-            staged = prob;
-        }
-        for (int tg = 0; tg < nx; tg += NT) {
-            const int n = min(NT, nx - tg);
-            float *part = part0 + buf * kPartRows * NT;
-            with_nt<NT>(n, [&](auto ntc) {
-                constexpr int NTC = decltype(ntc)::value;
-                if (g.wpr == 1) {
-                    warp_rows<NTC>(R.qs(s), R.d(s), q.k, q.ld_d, g, xs, tg, n,
-                                   [&](int row, int tt, float v) {
-                                       if (row < rows_valid && tt < n)
-                                           q.y[(int64_t)(tg + tt) * q.rows + r0 + row] = v;
-                                   });
-                    Q8_TRACE(8);
-                    if (tg + NT >= nx) {
-                        __syncwarp();
-                        if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
-                    }
-                    unsynced = true;
-                    return;
-                }
-                warp_rows_to_part<NTC>(R.qs(s), R.d(s), q.k, q.ld_d, g, xs, tg, n, part);
-                Q8_TRACE(8);
-                if (tg + NT >= nx) {
-                    __syncwarp();
-                    if ((threadIdx.x & 31) == 0) mbar_arrive(&R.empty[s]);
-                }
-                named_bar_sync(kBarConsumers, kCT);
-                for (int i = threadIdx.x; i < rows_valid * n; i += kCT) {
-                    const int row = i / n;
-                    const int tt = i - row * n;
-                    q.y[(int64_t)(tg + tt) * q.rows + r0 + row] = part_sum<NTC>(part, g, row, tt);
-                }
-            });
-            buf ^= 1;
-        }
-    }
-    // every consumer warp has seen the end: count this CTA as finished; the
-    // last one puts the counters back to zero
-    named_bar_sync(kBarConsumers, kCT);
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned done = atomicAdd(p.ws + 1, 1u);
-        if (done == gridDim.x - 1) {
-            atomicExch(p.ws, 0u);
-            atomicExch(p.ws + 1, 0u);
-        }
-    }
-}
-
-// ---------------------------------------------------------------------------
 // Test hook: per-block int32 dots through block_dot.
 // A row index outside [0, n_w_rows) writes INT32_MIN for each of its blocks
 // and reads nothing.
@@ -716,58 +552,6 @@ __global__ void block_dots_kernel(const int8_t *__restrict__ wq, int k, int64_t 
         const uint4 x0 = *reinterpret_cast<const uint4 *>(x);
         const uint4 x1 = *reinterpret_cast<const uint4 *>(x + 16);
         isum[i] = block_dot(w0, w1, x0, x1);
-    }
-}
-
-// The dynamic-schedule launch (ws given): chunks of the problems' tiles,
-// larger first, CTA b starting with chunk b.  Q8_E_UNSUPPORTED when the call
-// does not suit it (several activation groups, too many chunks or tiles):
-// the caller then runs the static split.
-q8_status launch_gemv_dyn(const GemvBatchParams &sp, int n_desc, int64_t n_tok, int nt,
-                          unsigned *ws, cudaStream_t s) {
-    static_assert(sizeof(GemvDynParams) < 32000, "kernel parameter block too large");
-    if (n_tok > sp.plan.xmax) return Q8_E_UNSUPPORTED;
-    GemvDynParams p{};
-    p.n_desc = n_desc;
-    p.n_tok = (int)n_tok;
-    p.plan = sp.plan;
-    p.ws = ws;
-    int64_t total = 0;
-    for (int i = 0; i < n_desc; ++i) {
-        p.pr[i] = sp.pr[i];
-        const Geo g = geo_for_k(p.pr[i].k, nt);
-        const int64_t t = (p.pr[i].rows + g.nr - 1) / g.nr;
-        if (t > 65535) return Q8_E_UNSUPPORTED;
-        total += t;
-    }
-    // chunk sizes: 8 tiles for the first 60% of the tiles, then 4, 2 and 1
-    int64_t done = 0;
-    int n = 0;
-    for (int i = 0; i < n_desc; ++i) {
-        const Geo g = geo_for_k(p.pr[i].k, nt);
-        const int t = (p.pr[i].rows + g.nr - 1) / g.nr;
-        for (int f = 0; f < t;) {
-            const double frac = (double)done / (double)total;
-            const int want = frac < 0.60 ? 8 : frac < 0.85 ? 4 : frac < 0.95 ? 2 : 1;
-            const int c = std::min(want, t - f);
-            if (n >= kGemvChunkMax) return Q8_E_UNSUPPORTED;
-            p.ch[n].problem = (uint8_t)i;
-            p.ch[n].ntiles = (uint8_t)c;
-            p.ch[n].first = (uint16_t)f;
-            ++n;
-            f += c;
-            done += c;
-        }
-    }
-    p.n_chunks = n;
-    const int grid = (int)std::max<int64_t>(
-        1, std::min<int64_t>(std::min<int64_t>((int64_t)num_sms() * p.plan.ctas, n), kGemvDynMaxGrid));
-    p.grid = grid;
-    switch (nt) {
-        case 1: return launch_stream(gemv_dyn_kernel<1>, grid, p.plan.bytes, s, p, "gemv_dyn");
-        case 2: return launch_stream(gemv_dyn_kernel<2>, grid, p.plan.bytes, s, p, "gemv_dyn");
-        case 4: return launch_stream(gemv_dyn_kernel<4>, grid, p.plan.bytes, s, p, "gemv_dyn");
-        default: return launch_stream(gemv_dyn_kernel<8>, grid, p.plan.bytes, s, p, "gemv_dyn");
     }
 }
 
@@ -833,8 +617,8 @@ q8_status q8_mul_mat_id_pregrouped(const q8_tensor *W, const int8_t *aq, const u
                             false, n_used, y, ws, ws_bytes, (cudaStream_t)stream);
 }
 
-q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_tok, void *ws,
-                          size_t ws_bytes, void *stream) {
+q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_tok,
+                          void *stream) {
     Q8_REQUIRE(descs != nullptr, Q8_E_NULL, "q8_gemv_batched: descs is NULL");
     Q8_REQUIRE(n_desc >= 1 && n_desc <= Q8_MAX_GEMV_DESC, Q8_E_SHAPE,
                "q8_gemv_batched: n_desc=%d", n_desc);
@@ -873,17 +657,10 @@ q8_status q8_gemv_batched(const q8_gemv_desc *descs, int32_t n_desc, int64_t n_t
         max_td = std::max(max_td, td);
     }
     Q8_REQUIRE(tiles < (1LL << 31), Q8_E_SHAPE, "q8_gemv_batched: too many tiles");
-    Q8_REQUIRE(ws == nullptr || (ws_bytes >= Q8_GEMV_WS_BYTES && ((uintptr_t)ws & 15u) == 0),
-               Q8_E_WORKSPACE, "q8_gemv_batched: workspace below %d bytes or not 16-byte aligned",
-               Q8_GEMV_WS_BYTES);
     p.total_tiles = (int)tiles;
     if (!make_plan(max_tq, max_td, max_k, (int)std::min<int64_t>(n_tok, kMaxXRows), nt, &p.plan,
                    0, true))
         Q8_FAIL(Q8_E_UNSUPPORTED, "q8_gemv_batched: k=%d does not fit the plan", max_k);
-    if (ws != nullptr) {
-        q8_status st = launch_gemv_dyn(p, n_desc, n_tok, nt, (unsigned *)ws, (cudaStream_t)stream);
-        if (st != Q8_E_UNSUPPORTED) return st;  // else: the static split below
-    }
     const int grid = (int)std::max<int64_t>(
         1, std::min<int64_t>(std::min<int64_t>((int64_t)num_sms() * p.plan.ctas, tiles),
                              kGemvMaxGrid));

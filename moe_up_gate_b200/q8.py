@@ -76,7 +76,7 @@ def load(auto_build: bool = True):
             "q8_pack_up_gate": (st, [vp, vp, i64, i64, i64, vp, vp, i64, vp]),
             "q8_quantize_row": (st, [vp, i64, i64, vp, vp, vp]),
             "q8_gemv": (st, [P(_Tensor), vp, vp, i64, vp, vp]),
-            "q8_gemv_batched": (st, [P(_GemvDesc), i32, i64, vp, sz, vp]),
+            "q8_gemv_batched": (st, [P(_GemvDesc), i32, i64, vp]),
             "q8_moe_workspace_size": (sz, [i64, i32, i64]),
             "q8_moe_up_gate_swiglu": (st, [P(_Tensor), vp, vp, i64, vp, i32, vp, vp, vp, vp, vp,
                                            vp, sz, vp]),
@@ -232,22 +232,12 @@ def gemv(W: Q8Tensor, xq: torch.Tensor, xd: torch.Tensor, y: torch.Tensor | None
     return y
 
 
-GEMV_WS_BYTES = 256
-
-
-def gemv_workspace(device="cuda") -> torch.Tensor:
-    """The batched GEMV's scheduling workspace (zero-filled)."""
-    return torch.zeros(GEMV_WS_BYTES, dtype=torch.uint8, device=device)
-
-
-def gemv_batched(problems, n_tok: int = 1, ws=None, stream=None):
-    """problems: list of (Q8Tensor, x fp32 [n_tok, k], y fp32 [n_tok, rows]) on the device.
-    ws: optional scheduling workspace (gemv_workspace()): chunks taken dynamically."""
+def gemv_batched(problems, n_tok: int = 1, stream=None):
+    """problems: list of (Q8Tensor, x fp32 [n_tok, k], y fp32 [n_tok, rows]) on the device."""
     arr = (_GemvDesc * len(problems))()
     for i, (W, x, y) in enumerate(problems):
         arr[i] = _GemvDesc(W.c(), x.data_ptr(), y.data_ptr())
-    _call("q8_gemv_batched", arr, len(problems), n_tok, _ptr(ws), 0 if ws is None else ws.numel(),
-          _stream(stream))
+    _call("q8_gemv_batched", arr, len(problems), n_tok, _stream(stream))
 
 
 def moe_workspace(n_tok: int, n_used: int, n_mat: int, device="cuda") -> torch.Tensor:

@@ -158,14 +158,11 @@ def test_gemv_batched_validation(q8):
     arr = (q8._GemvDesc * 2)()
     arr[0] = q8._GemvDesc(_tensor(q8), FAKE.value, FAKE.value)
     arr[1] = q8._GemvDesc(_tensor(q8, n_mat=3), FAKE.value, FAKE.value)
-    assert lib.q8_gemv_batched(arr, 2, 1, None, 0, None) == 2
-    assert lib.q8_gemv_batched(arr, 0, 1, None, 0, None) == 2
-    assert lib.q8_gemv_batched(arr, 129, 1, None, 0, None) == 2
+    assert lib.q8_gemv_batched(arr, 2, 1, None) == 2
+    assert lib.q8_gemv_batched(arr, 0, 1, None) == 2
+    assert lib.q8_gemv_batched(arr, 129, 1, None) == 2
     arr[1] = q8._GemvDesc(_tensor(q8), FAKE_ODD.value, FAKE.value)
-    assert lib.q8_gemv_batched(arr, 2, 1, None, 0, None) == 3
-    arr[1] = q8._GemvDesc(_tensor(q8), FAKE.value, FAKE.value)
-    assert lib.q8_gemv_batched(arr, 2, 1, FAKE, 64, None) == 7          # workspace too small
-    assert lib.q8_gemv_batched(arr, 2, 1, ctypes.c_void_p(0x10004), 256, None) == 7  # alignment
+    assert lib.q8_gemv_batched(arr, 2, 1, None) == 3
 
 
 def test_wait_hook_validation(q8):

@@ -80,30 +80,3 @@ def test_gemv_on_row_view():
     full = host(q8.gemv(W, xq, xd))
     assert np.array_equal(y, full[:, 32:72])
 
-
-def test_gemv_batched_dynamic_schedule_same_bits():
-    """With a scheduling workspace the CTAs take chunks of tiles from a counter
-    (CTAs finish together); the outputs are the bits of the fixed split, the
-    counter is back at zero after every call, and repeated calls on one
-    workspace agree (the Llama-2-110M matvec set at one token, and a batch of
-    3 rows)."""
-    mats = synth.llama_matvec_set()[:15] + [("classifier", 32000, 768)]
-    for n_tok in (1, 3):
-        probs_s, probs_d = [], []
-        for i, (_, rows, k) in enumerate(mats):
-            W = q8.pack(synth.normal((rows, k), seed=1500 + i, std=0.02).to(DEV))
-            x = synth.normal((n_tok, k), seed=1600 + i).to(DEV)
-            probs_s.append((W, x, torch.full((n_tok, rows), float("nan"), device=DEV)))
-            probs_d.append((W, x, torch.full((n_tok, rows), float("nan"), device=DEV)))
-        ws = q8.gemv_workspace(DEV)
-        q8.gemv_batched(probs_s, n_tok=n_tok)
-        for rep in range(3):
-            q8.gemv_batched(probs_d, n_tok=n_tok, ws=ws)
-            torch.cuda.synchronize()
-            assert int(ws.count_nonzero()) == 0
-            for (_, _, ys), (_, _, yd) in zip(probs_s, probs_d):
-                assert not torch.isnan(yd).any()
-                assert torch.equal(ys.view(torch.int32), yd.view(torch.int32))
-            for _, _, yd in probs_d:
-                yd.fill_(float("nan"))
-        q8.check(None)
