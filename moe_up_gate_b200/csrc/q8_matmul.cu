@@ -395,6 +395,79 @@ struct GemvBatchParams {
 };
 
 
+// One decode row (n_tok == 1) through the tiles [t0, t1) of one problem whose
+// rows a warp takes whole (k <= 4096), with RPW rows per warp and ITERS 32-block
+// steps per row.  The same arithmetic, in the same order, as warp_rows (so the
+// same bits): per lane, block sums scaled and added in block order, then the
+// reduce-scatter tree.  What it saves is the generic path's per-tile work:
+// the problem is held in registers, the lane's activation blocks are loaded
+// once for the whole run, the row addresses are fixed per warp, and there is
+// one tile loop with no dispatch inside.  Returns the ring position after t1.
+template <int RPW, int ITERS>
+__device__ __forceinline__ int gemv_run(const Ring &R, const XStage &xs, const GemvProblem &q,
+                                        const Geo &g, int64_t t0, int64_t t1, int it) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int k = q.k, nb = k / QK, ld_d = q.ld_d;
+    const int h0 = ((lane >> 2) & 1) * 16, h1 = 16 - h0;
+    const int row0 = warp * RPW;
+    uint4 xa[ITERS], xb[ITERS];
+    float dx[ITERS];
+#pragma unroll
+    for (int i = 0; i < ITERS; ++i) {
+        const int kb = i * 32 + lane;
+        xa[i] = xb[i] = make_uint4(0u, 0u, 0u, 0u);
+        dx[i] = 0.0f;
+        if (kb < nb) {
+            xa[i] = *reinterpret_cast<const uint4 *>(xs.q + kb * QK + h0);
+            xb[i] = *reinterpret_cast<const uint4 *>(xs.q + kb * QK + h1);
+            dx[i] = xs.dx[kb];
+        }
+    }
+    constexpr int VP = pow2_ceil(RPW);
+    const int idx = reduce_scatter_index<VP>(lane);
+    const bool writer = (lane & (32 / VP - 1)) == 0 && idx < RPW;
+    for (int64_t t = t0; t < t1; ++t, ++it) {
+        const int s = it % R.stages;
+        mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_matmul);
+        Q8_TRACE(6);
+        const int r0 = (int)(t - q.tile_begin) * g.nr;
+        const int8_t *sq = R.qs(s) + (size_t)row0 * k;
+        const uint16_t *sd = R.d(s) + (size_t)row0 * ld_d;
+        float acc[RPW];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) acc[r] = 0.0f;
+#pragma unroll
+        for (int i = 0; i < ITERS; ++i) {
+            const int kb = i * 32 + lane;
+            if (kb < nb) {
+                uint4 w0[RPW], w1[RPW];
+                float dw[RPW];
+#pragma unroll
+                for (int r = 0; r < RPW; ++r) {
+                    const int8_t *wp = sq + (size_t)r * k + kb * QK;
+                    w0[r] = *reinterpret_cast<const uint4 *>(wp + h0);
+                    w1[r] = *reinterpret_cast<const uint4 *>(wp + h1);
+                    dw[r] = scale_value(sd[(size_t)r * ld_d + kb]);
+                }
+#pragma unroll
+                for (int r = 0; r < RPW; ++r) {
+                    const int sum = block_dot(w0[r], w1[r], xa[i], xb[i]);
+                    acc[r] = fmaf(dw[r] * dx[i], small_int_to_float(sum), acc[r]);
+                }
+            }
+        }
+        float a[VP];
+#pragma unroll
+        for (int i = 0; i < VP; ++i) a[i] = i < RPW ? acc[i] : 0.0f;
+        const float v = warp_reduce_scatter<VP>(a);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&R.empty[s]);
+        Q8_TRACE(8);
+        if (writer && row0 + idx < q.rows - r0 && row0 + idx < g.nr) q.y[r0 + row0 + idx] = v;
+    }
+    return it;
+}
+
 template <int NT>
 __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     gemv_batched_kernel(const __grid_constant__ GemvBatchParams p) {
@@ -460,6 +533,37 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     bool unsynced = false;  // passes without a barrier since the last one
     for (int64_t t = tb; t < te; ++t, ++it) {
         while (cur + 1 < p.n_desc && p.pr[cur + 1].tile_begin <= t) ++cur;
+        if constexpr (NT == 1) {
+            // one decode row, whole rows per warp: the run of this problem's
+            // tiles in one tight loop (gemv_run)
+            const GemvProblem qv = p.pr[cur];
+            const Geo gv = geo_for_k(qv.k, 1);
+            if (p.n_tok == 1 && gv.wpr == 1) {
+                const int64_t t1 =
+                    cur + 1 < p.n_desc ? min(te, (int64_t)p.pr[cur + 1].tile_begin) : te;
+                if (cur != staged) {
+                    if (unsynced) named_bar_sync(kBarConsumers, kCT);
+                    stage_job_f32(R, J, xs, qv.x, qv.k, 1, [](int j) { return j; },
+                                  &g_err_matmul);
+                    named_bar_sync(kBarConsumers, kCT);
+                    Q8_TRACE(7);
+                    staged = cur;
+                    staged_grp = 0;
+                }
+                if (gv.rpw == 5)
+                    it = gemv_run<5, 1>(R, xs, qv, gv, t, t1, it);
+                else if (gv.rpw == 4)
+                    it = gemv_run<4, 1>(R, xs, qv, gv, t, t1, it);
+                else if (gv.rpw == 2)
+                    it = gemv_run<2, 2>(R, xs, qv, gv, t, t1, it);
+                else
+                    it = gemv_run<1, 4>(R, xs, qv, gv, t, t1, it);
+                unsynced = true;
+                t = t1 - 1;  // the loop's increments step to t1 and keep it
+                --it;
+                continue;
+            }
+        }
         const GemvProblem &q = p.pr[cur];
         const Geo g = geo_for_k(q.k, NT);
         const int s = it % R.stages;
