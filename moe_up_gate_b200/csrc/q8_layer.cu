@@ -152,6 +152,87 @@ __device__ __forceinline__ void stage_f32_l2(const XStage &xs, const float *src,
     }
 }
 
+// Phase A at one decode token, with x staged once for all experts: a consumer
+// group's up/gate tiles in one tight loop, the lane's activation blocks held
+// in registers for the whole phase.  The arithmetic and its order are those
+// of warp_pairs (dot_rows over gate row row0 + i and up row half + row0 + i,
+// then the reduce-scatter tree), so h has the same bits; the per-tile
+// dispatch of the generic path is gone.
+template <int RPW, int ITERS, int G>
+__device__ __forceinline__ void layer_pairs_run(const Ring &R, const XStage &xs,
+                                                const LayerParams &p, const int32_t *tab,
+                                                int tpm, int half, int64_t ta0, int64_t ta1,
+                                                int grp, int w8) {
+    const int lane = threadIdx.x & 31;
+    const int k = p.k, nb = k / QK, ld_d = (int)p.ug_ld_d;
+    const int h0 = ((lane >> 2) & 1) * 16, h1 = 16 - h0;
+    constexpr int H = RPW / 2;
+    const int row0 = w8 * H;
+    uint4 xa[ITERS], xb[ITERS];
+    float dx[ITERS];
+#pragma unroll
+    for (int i = 0; i < ITERS; ++i) {
+        const int kb = i * 32 + lane;
+        xa[i] = xb[i] = make_uint4(0u, 0u, 0u, 0u);
+        dx[i] = 0.0f;
+        if (kb < nb) {
+            xa[i] = *reinterpret_cast<const uint4 *>(xs.q + kb * QK + h0);
+            xb[i] = *reinterpret_cast<const uint4 *>(xs.q + kb * QK + h1);
+            dx[i] = xs.dx[kb];
+        }
+    }
+    constexpr int VP = pow2_ceil(RPW);
+    const int idx = reduce_scatter_index<VP>(lane);
+    const int up_idx = idx + H;
+    const int up_lane = reduce_scatter_lane<VP>(up_idx < VP ? up_idx : 0);
+    const bool writer = (lane & (32 / VP - 1)) == 0 && idx < H;
+    for (int64_t t = ta0 + grp; t < ta1; t += G) {
+        const int it = (int)(t - ta0);
+        const int s = it % R.stages;
+        mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_layer);
+        Q8_TRACE(6);
+        const int mi = (int)(t / tpm), ti = (int)(t % tpm);
+        const int e = tab[p.lay_list + mi];
+        const int pr = tab[p.lay_pairs + tab[p.lay_offset + e]];  // one pair per expert
+        const int r0 = ti * half;
+        const int8_t *sq = R.qs(s);
+        const uint16_t *sd = R.d(s);
+        float acc[RPW];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) acc[r] = 0.0f;
+#pragma unroll
+        for (int i = 0; i < ITERS; ++i) {
+            const int kb = i * 32 + lane;
+            if (kb < nb) {
+                uint4 w0[RPW], w1[RPW];
+                float dw[RPW];
+#pragma unroll
+                for (int r = 0; r < RPW; ++r) {
+                    const int srow = r < H ? row0 + r : half + row0 + (r - H);
+                    const int8_t *wp = sq + (size_t)srow * k + kb * QK;
+                    w0[r] = *reinterpret_cast<const uint4 *>(wp + h0);
+                    w1[r] = *reinterpret_cast<const uint4 *>(wp + h1);
+                    dw[r] = scale_value(sd[(size_t)srow * ld_d + kb]);
+                }
+#pragma unroll
+                for (int r = 0; r < RPW; ++r) {
+                    const int sum = block_dot(w0[r], w1[r], xa[i], xb[i]);
+                    acc[r] = fmaf(dw[r] * dx[i], small_int_to_float(sum), acc[r]);
+                }
+            }
+        }
+        float a[VP];
+#pragma unroll
+        for (int i = 0; i < VP; ++i) a[i] = i < RPW ? acc[i] : 0.0f;
+        const float v = warp_reduce_scatter<VP>(a);
+        const float u = __shfl_sync(0xffffffffu, v, up_lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&R.empty[s]);
+        Q8_TRACE(8);
+        if (writer) p.h[(int64_t)pr * p.n_ff + r0 + row0 + idx] = v / (1.0f + expf(-v)) * u;
+    }
+}
+
 // G consumer groups of kCW warps share one ring: group g takes every G-th
 // tile of phase A and every G-th unit of phase B (G = 2 doubles the warps
 // that hide each other's latency, at one CTA per SM).  G > 1 needs the
@@ -291,7 +372,26 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
         sync_all();
         Q8_TRACE(7);
     }
-    for (int64_t t = ta0 + grp; t < ta1; t += G) {
+    bool phase_a_done = false;
+    if constexpr (NT == 1) {
+        if (x_once) {
+            // one decode token: every expert has one pair and reads the one
+            // staged x row
+            const int iters = (p.k / QK + 31) / 32;
+            if (ga.rpw == 2 && iters == 1)
+                layer_pairs_run<2, 1, G>(R, xs, p, tab, tpm, half, ta0, ta1, grp, w8);
+            else if (ga.rpw == 2 && iters == 2)
+                layer_pairs_run<2, 2, G>(R, xs, p, tab, tpm, half, ta0, ta1, grp, w8);
+            else if (ga.rpw == 2 && iters == 3)
+                layer_pairs_run<2, 3, G>(R, xs, p, tab, tpm, half, ta0, ta1, grp, w8);
+            else if (ga.rpw == 2)
+                layer_pairs_run<2, 4, G>(R, xs, p, tab, tpm, half, ta0, ta1, grp, w8);
+            else
+                layer_pairs_run<4, 1, G>(R, xs, p, tab, tpm, half, ta0, ta1, grp, w8);
+            phase_a_done = true;
+        }
+    }
+    for (int64_t t = ta0 + grp; t < ta1 && !phase_a_done; t += G) {
         const int it = (int)(t - ta0);
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_layer);

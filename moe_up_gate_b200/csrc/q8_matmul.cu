@@ -550,12 +550,22 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                     staged = cur;
                     staged_grp = 0;
                 }
-                if (gv.rpw == 5)
+                // 32-block steps per row: 1 (k <= 1024), 2 (k <= 2048) or 4
+                const int iters = qv.k <= 1024 ? 1 : qv.k <= 2048 ? 2 : 4;
+                if (gv.rpw == 5 && iters == 1)
                     it = gemv_run<5, 1>(R, xs, qv, gv, t, t1, it);
-                else if (gv.rpw == 4)
+                else if (gv.rpw == 4 && iters == 1)
                     it = gemv_run<4, 1>(R, xs, qv, gv, t, t1, it);
-                else if (gv.rpw == 2)
+                else if (gv.rpw == 3 && iters == 1)
+                    it = gemv_run<3, 1>(R, xs, qv, gv, t, t1, it);
+                else if (gv.rpw == 2 && iters == 1)
+                    it = gemv_run<2, 1>(R, xs, qv, gv, t, t1, it);
+                else if (gv.rpw == 2 && iters == 2)
                     it = gemv_run<2, 2>(R, xs, qv, gv, t, t1, it);
+                else if (gv.rpw == 1 && iters == 1)
+                    it = gemv_run<1, 1>(R, xs, qv, gv, t, t1, it);
+                else if (gv.rpw == 1 && iters == 2)
+                    it = gemv_run<1, 2>(R, xs, qv, gv, t, t1, it);
                 else
                     it = gemv_run<1, 4>(R, xs, qv, gv, t, t1, it);
                 unsynced = true;
