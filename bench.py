@@ -408,7 +408,11 @@ class MoeWorkload:
             # the whole layer when it is fused)
             self.up_gate_bytes.append((tot if self.fused else ug) / self.layers)
         self.tokens_per_step = tokens
-        self.small = P <= 1024 and E <= 512
+        # the paths q8_moe_ffn takes: the fp32 calls for dense batches up to
+        # 1024 rows and routed batches up to 32 pairs (the fused kernel
+        # when it applies); larger routed batches group once (tensor cores
+        # for the experts with at least 4 rows)
+        self.small = P <= 1024 and E <= 512 and (not self.routed or P <= 32)
         self.config = {"workload": kind, "tokens": tokens, "layers": self.layers, "n_embd": D,
                        "n_ff": F, "n_experts": E, "n_used": Uu,
                        "mean_weight_bytes_per_step": statistics.mean(self.step_bytes),
@@ -469,7 +473,7 @@ class MoeWorkload:
         elif self.routed:
             # quantize x, group, up/gate (dp4a + tensor cores), quantize h,
             # down (dp4a + tensor cores), combine; the timed unit is the
-            # up/gate step: tc_kernel for the experts with >= 16 rows and
+            # up/gate step: tc_kernel for the experts with >= 4 rows and
             # up_gate_kernel for the rest
             self.kernel = "up_gate_step"
             self.launches_per_step = self.layers * 8
@@ -801,21 +805,26 @@ def measure(wl, args, dist, stream, cpu_seconds):
     flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=wl.dev) \
         if getattr(wl, "flush", False) else None
 
-    # one CUDA graph per step index, without timing marks (the step rate), and
-    # one per timed step with event marks around the dominant launches (the
-    # kernel time); the marks are kept out of the step-rate graphs
+    # CUDA graphs without timing marks for the step rate: one per warm-up
+    # step, and the K timed steps in one graph (back to back on the device,
+    # no host replay between steps) unless an L2 flush must run between
+    # them (then one graph per step); and one graph per timed step with
+    # event marks around the dominant launches (the kernel time), kept out of
+    # the step-rate graphs
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         wl.issue(0, NoMarks())  # eager warm-up (sets kernel attributes)
     torch.cuda.synchronize()
 
-    def capture(i, m, input_set=None):
+    def capture(i, m, input_set=None, n_steps=1):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            wl.issue(i, m, input_set)
+            for j in range(i, i + n_steps):
+                wl.issue(j, m, input_set)
         return g
 
-    graphs = [capture(i, NoMarks()) for i in range(W + K)]
+    graphs = [capture(i, NoMarks()) for i in range(W + (K if flush is not None else 0))]
+    timed_graph = capture(W, NoMarks(), n_steps=K) if flush is None else None
     marks = [Marks(wl.dominant_launches) for _ in range(K)]
     mgraphs = [capture(W + i, marks[i]) for i in range(K)]
     torch.cuda.synchronize()
@@ -834,18 +843,22 @@ def measure(wl, args, dist, stream, cpu_seconds):
     st_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     en_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
 
-    def timed_steps(step):
+    def timed_steps(step, all_steps=None):
         """K steps, bracketed by a barrier + synchronize on both sides; ms of
         device time, max over ranks.  Timed by one pair of events around the K
-        steps, or, when an L2 flush runs between steps, by a pair around each
-        step (the flush stays outside the timed intervals)."""
+        steps (all_steps() issues them at once when given, else step(i) each),
+        or, when an L2 flush runs between steps, by a pair around each step
+        (the flush stays outside the timed intervals)."""
         torch.cuda.synchronize()
         dist.barrier()
         with torch.cuda.stream(stream):
             if flush is None:
                 ev[0].record(stream)
-                for i in range(K):
-                    step(i)
+                if all_steps is not None:
+                    all_steps()
+                else:
+                    for i in range(K):
+                        step(i)
                 ev[1].record(stream)
             else:
                 for i in range(K):
@@ -860,6 +873,8 @@ def measure(wl, args, dist, stream, cpu_seconds):
         return dist.max(ms)
 
     def one_round():
+        if timed_graph is not None:
+            return timed_steps(None, all_steps=timed_graph.replay)
         return timed_steps(lambda i: graphs[W + i].replay())
 
     torch.cuda.nvtx.range_push("timed")
@@ -923,7 +938,8 @@ def measure(wl, args, dist, stream, cpu_seconds):
         "config": dict(wl.config, parallelism=f"replicas x{n}"),
         "timing": {"rounds": len(round_ms),
                    "round_ms_min_median_max": [min(round_ms), total_ms, max(round_ms)],
-                   "step_timer": ("one event pair around each round of K steps"
+                   "step_timer": ("one event pair around each round of K steps (the K steps "
+                                  "replayed as one CUDA graph)"
                                   if flush is None else
                                   "an event pair around each step (the L2 flush between "
                                   "steps is not timed)")},
@@ -951,7 +967,7 @@ def measure(wl, args, dist, stream, cpu_seconds):
                        f"{nsteps} x one layer of {wl.name} (T={wl.T}) through the scalar C "
                        f"oracle (the first {wl.o_tok} of its tokens), counted as "
                        f"1/{wl.layers} of a step, {el:.1f} s")}
-    del graphs, mgraphs, e2e_graphs
+    del graphs, timed_graph, mgraphs, e2e_graphs
     return out
 
 

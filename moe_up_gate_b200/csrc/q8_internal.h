@@ -173,8 +173,11 @@ q8_status clear_wait_errors_tc();
 
 // Tensor-core path (q8_tc.cu) for experts with at least kTcMinPairs routed
 // rows: whether a weight view can take it, and the launch over the
-// tensor-core list of a grouping workspace.
-constexpr int kTcMinPairs = 16;
+// tensor-core list of a grouping workspace.  From 4 rows on, a 16-column MMA
+// pass (padded) costs less per weight byte than the dp4a kernel: the
+// 128-expert layer at 256 tokens ran 1.3x faster than with a 16-row
+// threshold.
+constexpr int kTcMinPairs = 4;
 // Dense calls (one matrix) with kTcMinDense..kTcMaxDense activation rows go
 // to the tensor cores too (one pass over the weights): launch_tc with
 // ws == nullptr.

@@ -92,19 +92,27 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
 // before the first use).  A CTA adds one (release) and waits (acquire) until
 // the counter reaches the next multiple of n above its own arrival: one
 // atomic per CTA and no reset, so the last arrival releases the others with
-// its own atomic.
+// its own atomic.  The add is acquire-release at GPU scope and the polls are
+// acquire loads: the adds form one release sequence, so a CTA that reads the
+// final count has seen every CTA's writes before its arrival (the CTA
+// barrier before the call makes them the arriving thread's), with no
+// separate fences.
 // Bounded: after limit_ns the wait records Q8_WAIT_TIMEOUT and returns
 // false (the counter is then left off its multiple: q8_check reports it).
+__device__ __forceinline__ unsigned long long atom_add_acq_rel_u64(unsigned long long *p,
+                                                                   unsigned long long v) {
+    unsigned long long old;
+    asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v)
+                 : "memory");
+    return old;
+}
+
 __device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned n, int *err,
                                              uint64_t limit_ns = kWaitLimitNs) {
     unsigned long long *cnt = reinterpret_cast<unsigned long long *>(bar);
-    __threadfence();
-    const unsigned long long old = atomicAdd(cnt, 1ull);
+    const unsigned long long old = atom_add_acq_rel_u64(cnt, 1ull);
     const unsigned long long target = (old / n + 1) * n;
-    if (old + 1 == target) {
-        __threadfence();
-        return true;
-    }
+    if (old + 1 == target) return true;
     const uint64_t t0 = globaltimer_ns();
     while (ld_acquire_u64(cnt) < target) {
         if (globaltimer_ns() - t0 > limit_ns) {
@@ -113,7 +121,6 @@ __device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned n, int *err
         }
         __nanosleep(32);
     }
-    __threadfence();
     return true;
 }
 
@@ -255,6 +262,7 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
     Q8_TRACE(1);
     griddep_wait();  // x, ids and route_w may come from the preceding kernel
     griddep_launch_dependents();
+    Q8_TRACE(2);
     // One token (the NT == 1 variant): every routed expert reads the same x
     // row, so the producer fetches it before the grouping and it is staged
     // once for the whole of phase A.
@@ -263,11 +271,13 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
         mbar_arrive_expect_tx(R.xfull, (uint32_t)p.k * 4);
         bulk_g2s_keep(R.raw, p.x, (uint32_t)p.k * 4, R.xfull);
     }
-    // the routing weights are read only by the combine at the very end, but
-    // loaded now, while the memory system is idle (ordered by the grouping's
-    // CTA barrier below)
+    // the routing weights are read only by the combine at the very end: their
+    // copy starts now, asynchronously (the grouping's read of the ids does not
+    // wait behind it), and the issuing threads wait for it before the grid
+    // barrier
     float *s_rw = reinterpret_cast<float *>(smem + p.off_rw);
-    for (int i = threadIdx.x; i < p.n_tok * p.n_used; i += blockDim.x) s_rw[i] = p.route_w[i];
+    for (int i = threadIdx.x; i < p.n_tok * p.n_used; i += blockDim.x) cp_async4(s_rw + i, p.route_w + i);
+    cp_async_commit();
     int32_t *tab = reinterpret_cast<int32_t *>(smem + p.plan.off_tab);
     {
         GroupLayout L{};
@@ -438,6 +448,7 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
 
     // ---------------- every CTA's h is written
     const int P = p.n_tok * p.n_used;
+    cp_async_wait<0>();  // this thread's part of the routing weights has landed
     if (p.off_hf >= 0) fence_proxy_async_global();  // h is read back by a bulk copy
     sync_all();
     Q8_TRACE(12);
@@ -464,6 +475,7 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
     float *ybuf = reinterpret_cast<float *>(smem + p.off_y) + (size_t)grp * P * nrb;
     if (p.off_hf >= 0) {
         mbar_wait(hbar, 0, &g_err_layer);
+        Q8_TRACE(14);
         stage_f32_smem8(hs, reinterpret_cast<const float *>(smem + p.off_hf), p.n_ff, n_valid,
                        [&](int j) { return tab[p.lay_pairs + j]; }, threadIdx.x, kAll);
     } else {
@@ -513,11 +525,13 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
                     });
                 }
             }
+            Q8_TRACE(13);
             __syncwarp();
             if (lane == 0) mbar_arrive(&R.empty[s]);
             Q8_TRACE(8);
         }
         sync_grp();
+        Q8_TRACE(15);
         for (int i = gtid; i < p.n_tok * nrv; i += kCT) {
             const int t = i / nrv;
             const int rr = i - t * nrv;

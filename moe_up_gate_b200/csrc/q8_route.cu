@@ -11,14 +11,17 @@
 //   route_w[t]   = softmax over the selected logits only (the largest one
 //                  subtracted before exp, fp64), stored as fp32.
 //
-// One thread-block cluster per group of kRouteTok tokens: the cluster's CTAs
-// split the experts (CTA r takes experts e = r, r + C, ...; a warp per
-// expert row, 16-byte loads, fp64 fma per token, a fixed xor tree), keep the
-// logits in their own shared memory, and after a cluster barrier CTA 0 reads
-// every logit through distributed shared memory; a second cluster barrier
-// keeps every CTA's shared memory alive until then.  CTA 0 then selects the
-// top n_used per token (one warp per token, repeated warp argmax) and forms
-// the weights.  No atomics, no global scratch: the results are deterministic.
+// One thread-block cluster per group of up to kRouteTok tokens: the
+// cluster's CTAs split the experts (CTA r takes experts e = r, r + C, ...; a
+// warp per expert row, 16-byte loads, fp64 fma per token, a fixed xor tree),
+// keep the logits in their own shared memory, and after a cluster barrier
+// CTA 0 reads every logit through distributed shared memory; a second cluster
+// barrier keeps every CTA's shared memory alive until then.  CTA 0 then
+// selects the top n_used per token (one warp per token, repeated warp argmax)
+// and forms the weights.  The group's activations are staged once as fp64
+// (exact), so the inner loop is one fp64 fma per weight and token plus one
+// conversion per weight.  No atomics, no global scratch: the results are
+// deterministic.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -31,9 +34,8 @@ namespace cg = cooperative_groups;
 
 namespace q8 {
 
-constexpr int kRouteTok = 4;         // tokens per cluster
-constexpr int kRouteThreads = 256;   // 8 warps
-constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr int kRouteTok = 4;         // most tokens per cluster
+constexpr int kRouteThreads = 512;   // most threads per CTA (16 warps)
 constexpr int kRouteCluster = 8;     // CTAs per cluster (portable size)
 constexpr int kRouteUnroll = 8;      // router-row loads in flight per lane
 constexpr int kSmemLimitRoute = 227 * 1024;
@@ -42,6 +44,7 @@ struct RouteParams {
     const float *w;  // [n_exp][n_embd]
     const float *x;  // [n_tok][n_embd]
     int n_tok, n_embd, n_exp, n_used;
+    int tpc;         // tokens per cluster (1..kRouteTok; fewer when n_embd is long)
     int32_t *ids;    // [n_tok][n_used]
     float *route_w;  // [n_tok][n_used]
     double *logits;  // [n_tok][n_exp] or nullptr
@@ -61,21 +64,26 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
     const int rank = (int)cluster.block_rank();
     const int C = (int)cluster.num_blocks();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t0 = (int)(blockIdx.x / C) * kRouteTok;
-    const int nt = min(kRouteTok, p.n_tok - t0);
-    float *xs = reinterpret_cast<float *>(smem);
-    double *lg = reinterpret_cast<double *>(smem + p.off_lg);  // [kRouteTok][n_exp], own experts only
+    const int t0 = (int)(blockIdx.x / C) * p.tpc;
+    const int nt = min(p.tpc, p.n_tok - t0);
+    // x of token t as fp64 pairs: element 4c, 4c+1 at xa[t * n4 + c], 4c+2,
+    // 4c+3 at xb[t * n4 + c] (lane-consecutive 16-byte loads, no bank conflicts)
+    const int n4 = p.n_embd / 4;
+    double2 *xa = reinterpret_cast<double2 *>(smem);
+    double2 *xb = xa + (size_t)p.tpc * n4;
+    double *lg = reinterpret_cast<double *>(smem + p.off_lg);  // [tpc][n_exp], own experts only
+    const int n_warps = (int)(blockDim.x >> 5);
     griddep_wait();  // x may come from the preceding kernel
     griddep_launch_dependents();
-    const int n4 = p.n_embd / 4;
-    for (int i = threadIdx.x; i < nt * n4; i += kRouteThreads) {
+    for (int i = threadIdx.x; i < nt * n4; i += blockDim.x) {
         const int t = i / n4, c = i - t * n4;
-        reinterpret_cast<float4 *>(xs)[t * n4 + c] =
-            reinterpret_cast<const float4 *>(p.x + (int64_t)(t0 + t) * p.n_embd)[c];
+        const float4 v = reinterpret_cast<const float4 *>(p.x + (int64_t)(t0 + t) * p.n_embd)[c];
+        xa[i] = make_double2((double)v.x, (double)v.y);
+        xb[i] = make_double2((double)v.z, (double)v.w);
     }
     __syncthreads();
     // logits of this CTA's experts: warp per expert row
-    for (int e = rank + C * warp; e < p.n_exp; e += C * kRouteWarps) {
+    for (int e = rank + C * warp; e < p.n_exp; e += C * n_warps) {
         const float4 *wr = reinterpret_cast<const float4 *>(p.w + (int64_t)e * p.n_embd);
         double acc[kRouteTok];
 #pragma unroll
@@ -91,14 +99,15 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
             for (int u = 0; u < kRouteUnroll; ++u) {
                 const int c = c0 + 32 * u;
                 if (c >= n4) break;
+                const double w0 = wv[u].x, w1 = wv[u].y, w2 = wv[u].z, w3 = wv[u].w;
 #pragma unroll
                 for (int t = 0; t < kRouteTok; ++t) {
                     if (t < nt) {
-                        const float4 xv = reinterpret_cast<const float4 *>(xs)[t * n4 + c];
-                        acc[t] = fma((double)wv[u].x, (double)xv.x, acc[t]);
-                        acc[t] = fma((double)wv[u].y, (double)xv.y, acc[t]);
-                        acc[t] = fma((double)wv[u].z, (double)xv.z, acc[t]);
-                        acc[t] = fma((double)wv[u].w, (double)xv.w, acc[t]);
+                        const double2 a = xa[t * n4 + c], b = xb[t * n4 + c];
+                        acc[t] = fma(w0, a.x, acc[t]);
+                        acc[t] = fma(w1, a.y, acc[t]);
+                        acc[t] = fma(w2, b.x, acc[t]);
+                        acc[t] = fma(w3, b.y, acc[t]);
                     }
                 }
             }
@@ -108,12 +117,15 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
         }
-        if (lane == 0)
-            for (int t = 0; t < nt; ++t) lg[t * p.n_exp + e] = acc[t];
+        if (lane == 0) {
+#pragma unroll
+            for (int t = 0; t < kRouteTok; ++t)
+                if (t < nt) lg[t * p.n_exp + e] = acc[t];
+        }
     }
     cluster.sync();  // every CTA's logits are written (release / acquire)
     if (p.logits) {
-        for (int i = threadIdx.x; i < nt * p.n_exp; i += kRouteThreads) {
+        for (int i = threadIdx.x; i < nt * p.n_exp; i += blockDim.x) {
             const int t = i / p.n_exp, e = i - t * p.n_exp;
             if (e % C == rank) p.logits[(int64_t)(t0 + t) * p.n_exp + e] = lg[i];
         }
@@ -121,7 +133,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
     if (rank == 0) {
         // gather the other CTAs' logits into this CTA's array (each expert's
         // slot is written by exactly one CTA; this CTA's own slots stay)
-        for (int i = threadIdx.x; i < nt * p.n_exp; i += kRouteThreads) {
+        for (int i = threadIdx.x; i < nt * p.n_exp; i += blockDim.x) {
             const int e = i % p.n_exp;
             if (e % C != 0) lg[i] = cluster.map_shared_rank(lg, e % C)[i];
         }
@@ -211,11 +223,16 @@ extern "C" q8_status q8_route(const float *w_router, const float *x, int64_t n_t
     p.route_w = route_w;
     p.logits = logits;
     const int C = kRouteCluster;
-    const int x_bytes = kRouteTok * (int)n_embd * 4;
+    // tokens per cluster: as many as fit (up to kRouteTok), the fp64 rows of
+    // x, the logits and the selection flags of each
+    const int per_tok = (int)n_embd * 8 + (int)n_exp * 9 + 32;
+    p.tpc = std::min<int>(kRouteTok, kSmemLimitRoute / per_tok);
+    Q8_REQUIRE(p.tpc >= 1, Q8_E_UNSUPPORTED, "%s: shared-memory plan too large", fn);
+    const int x_bytes = p.tpc * (int)n_embd * 8;  // two double2 arrays (xa, xb)
     p.off_lg = (x_bytes + 15) / 16 * 16;
-    const int lg_bytes = kRouteTok * (int)n_exp * 8;
+    const int lg_bytes = p.tpc * (int)n_exp * 8;
     p.off_sel = p.off_lg + lg_bytes;
-    const int smem = p.off_sel + kRouteTok * (int)n_exp;
+    const int smem = p.off_sel + p.tpc * (int)n_exp;
     Q8_REQUIRE(smem <= kSmemLimitRoute, Q8_E_UNSUPPORTED, "%s: shared-memory plan too large", fn);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
@@ -228,10 +245,13 @@ extern "C" q8_status q8_route(const float *w_router, const float *x, int64_t n_t
             Q8_FAIL(Q8_E_CUDA, "%s: shared-memory attribute: %s", fn, cudaGetErrorString(e));
         set_smem_opted_in((const void *)route_kernel, dev);
     }
-    const int groups = (int)((n_tok + kRouteTok - 1) / kRouteTok);
+    const int groups = (int)((n_tok + p.tpc - 1) / p.tpc);
+    // a few clusters (decode): 16 warps per CTA, one router row each at 128
+    // experts; many: 8 warps, so that two CTAs share an SM
+    const int threads = (int64_t)groups * C * 2 <= num_sms() ? kRouteThreads : kRouteThreads / 2;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)(groups * C));
-    cfg.blockDim = dim3(kRouteThreads);
+    cfg.blockDim = dim3((unsigned)threads);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = (cudaStream_t)stream;
     cudaLaunchAttribute attr[2];

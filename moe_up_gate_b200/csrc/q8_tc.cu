@@ -15,9 +15,9 @@
 // Q8_0 block (M=128, N=16/32, K=32) lands in its own tensor-memory slot
 // (16 slots: the MMAs run up to four chunks ahead of the epilogue), because
 // each block has its own pair of scales and the int32 sum cannot run across
-// blocks; eight epilogue warps read the slots back, scale by d_w * d_x in
-// fp32 and accumulate in block order.  Every wait is bounded (q8_ptx.cuh);
-// tensor memory is freed before exit.
+// blocks; sixteen epilogue warps read the slots back, scale each block sum by
+// d_w (rounded once) and add d_x times that to the fp32 sums in block order.
+// Every wait is bounded (q8_ptx.cuh); tensor memory is freed before exit.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -39,15 +39,17 @@ constexpr int kTcB = kTcN * 128;    // B part: kTcN rows x 128 bytes (core matri
 constexpr int kTcStage = 20480;     // kTcA + kTcB
 constexpr int kTcDxRing = 8;        // entries of the activation-scale ring, one per K chunk
 constexpr int kTcDx = kTcN * 4 * 4; // an entry: the chunk's 4 blocks' scales d_x, fp32 [block][row]
-constexpr int kTcDm = kTcN * 4 * 4; // then -kTcMagic * d_x, fp32 [block][row]
 constexpr int kTcDh = kTcN * 4 * 2; // then d_x as copied, fp16 [row][block]
-constexpr int kTcDxEntry = kTcDx + kTcDm + kTcDh;
-// A block sum |v| < 2^22 becomes the fp32 kTcMagic + v by adding v to the
-// bits of kTcMagic.  kTcMagic * d_x is exact in fp32 (d_x is an fp16 value,
-// 11 significant bits), so fma(kTcMagic + v, d_x, -kTcMagic * d_x) is v * d_x
-// rounded once.
+constexpr int kTcDxEntry = kTcDx + kTcDh;
+// Block scaling.  Every tensor-memory slot holds the bits of kTcMagic before
+// its MMA, which accumulates onto them: a block sum |v| < 2^22 then reads
+// back as the fp32 value kTcMagic + v, exactly.  kTcMagic * d_w is exact in
+// fp32 (d_w is an fp16 value, 11 significant bits), so
+// fma(kTcMagic + v, d_w, -kTcMagic * d_w) is v * d_w rounded once; the
+// epilogue then adds d_x times that to the row's sum and writes kTcMagic back
+// into the slot for its next block.
 constexpr float kTcMagic = 12582912.0f;  // 1.5 * 2^23
-constexpr int kTcMagicBits = 0x4B400000;
+constexpr uint32_t kTcMagicBits = 0x4B400000u;
 constexpr int kTcLag = 3;           // chunks a builder keeps in flight before it reports one
 constexpr int kTcEpiWarps = 16;
 constexpr int kTcCw = kTcN * 4 / kTcEpiWarps;  // activation rows (columns) per epilogue warp
@@ -104,25 +106,12 @@ __device__ __forceinline__ float tc_silu(float z) { return z / (1.0f + expf(-z))
 __device__ __forceinline__ void tmem_ld_cols(uint32_t addr, uint32_t (&v)[16]) { tmem_ld16(addr, v); }
 __device__ __forceinline__ void tmem_ld_cols(uint32_t addr, uint32_t (&v)[8]) { tmem_ld8(addr, v); }
 
-// Pairs of fp32 in one 64-bit register pair, for the packed sm_100 form of
-// fma: each lane of the pair is rounded exactly as the scalar instruction
-// rounds it, at half the instruction count.
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-// Two block sums |v| < 2^22 as the fp32 values 1.5 * 2^23 + v (exact).
-__device__ __forceinline__ uint64_t f2_biased(uint32_t a, uint32_t b) {
-    return f2_pack(__int_as_float((int)a + kTcMagicBits), __int_as_float((int)b + kTcMagicBits));
+// Set this thread's kTcCw columns of a slot back to kTcMagic.
+__device__ __forceinline__ void tmem_rebias(uint32_t addr) {
+    if constexpr (kTcCw == 8)
+        tmem_fill8(addr, kTcMagicBits);
+    else
+        tmem_fill16(addr, kTcMagicBits);
 }
 
 // The CTA's work items, in order: (expert of the tensor-core list, pass of
@@ -155,19 +144,27 @@ struct TcWalk {
         it.n = min(kTcN, it.cnt - it.c0);
         it.npad = (it.n + 15) / 16 * 16;
     }
-    // the item with index i (sequential scan of the expert list)
-    __device__ __forceinline__ TcItem seek(int64_t i) const {
+    // the item with index i, given first[mi] = the passes of the experts
+    // before mi (first[n_big] = all of them): a binary search
+    __device__ __forceinline__ TcItem seek(int64_t i, const int *first) const {
         TcItem it{};
-        int64_t before = 0;
-        for (it.mi = 0; it.mi < n_big; ++it.mi) {
-            const int64_t cnt = (int64_t)passes(it.mi) * n_tiles;
-            if (i < before + cnt) break;
-            before += cnt;
+        if (i >= (int64_t)first[n_big] * n_tiles) {
+            it.mi = n_big;
+            return it;
         }
-        const int64_t r = i - before;
+        int lo = 0, hi = n_big;  // first[lo] * n_tiles <= i < first[hi] * n_tiles
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if ((int64_t)first[mid] * n_tiles <= i)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        it.mi = lo;
+        const int64_t r = i - (int64_t)first[lo] * n_tiles;
         it.pass = (int)(r / n_tiles);
         it.tile = (int)(r % n_tiles);
-        if (it.mi < n_big) fill(it);
+        fill(it);
         return it;
     }
     __device__ __forceinline__ void next(TcItem &it) const {
@@ -179,11 +176,6 @@ struct TcWalk {
             }
         }
         if (it.mi < n_big) fill(it);
-    }
-    __device__ __forceinline__ int64_t total() const {
-        int64_t t = 0;
-        for (int mi = 0; mi < n_big; ++mi) t += (int64_t)passes(mi) * n_tiles;
-        return t;
     }
 };
 
@@ -202,18 +194,40 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // the 128-byte-swizzled stages need 1024-byte alignment
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    Q8_TRACE(0);
     griddep_launch_dependents();
     griddep_wait();  // the grouping tables and the activations come from earlier kernels
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool upgate = p.n_ff > 0;
     const int k = p.k, nb = k / QK, nkc = (k + 127) / 128;
     TcWalk W{&p, p.n_dense > 0 ? 1 : p.ws[WS_N_BIG], upgate ? p.n_ff / 64 : (p.rows + 127) / 128};
-    // the item count, by one lane per warp (a scan of the expert list)
-    int64_t total = 0;
-    if (lane == 0) total = W.total();
-    total = __shfl_sync(0xffffffffu, total, 0);
+    // The walk: every tensor-core expert's pass count (loaded by all
+    // threads at once), then their running sum by warp 0, in the ring's
+    // memory before the ring is used (n_big <= 4096 ints).
+    int *first = reinterpret_cast<int *>(smem);
+    for (int mi = threadIdx.x; mi < W.n_big; mi += blockDim.x) first[mi] = W.passes(mi);
+    __syncthreads();
+    if (warp == 0) {
+        int run = 0;
+        for (int base = 0; base < W.n_big; base += 32) {
+            const int v = base + lane < W.n_big ? first[base + lane] : 0;
+            int inc = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += u;
+            }
+            if (base + lane < W.n_big) first[base + lane] = run + inc - v;
+            run += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) first[W.n_big] = run;
+    }
+    __syncthreads();
+    const int64_t total = (int64_t)first[W.n_big] * W.n_tiles;
     const int64_t i0 = total * blockIdx.x / gridDim.x, i1 = total * (blockIdx.x + 1) / gridDim.x;
-    if (i0 >= i1) return;  // uniform: before any barrier
+    TcItem it = W.seek(i0, first);
+    __syncthreads();       // the ring's memory is free again
+    if (i0 >= i1) return;  // uniform: before any other barrier
 
     unsigned char *ring = smem;
     float *xchg = reinterpret_cast<float *>(smem + p.off_xchg);
@@ -258,8 +272,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+    // every slot starts at kTcMagic (an epilogue warp sets its lane quarter's
+    // columns of each slot; the MMAs accumulate onto them)
+    if (warp >= 2 && warp < 2 + kTcEpiWarps) {
+        const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) +
+                            (uint32_t)(((warp - 2) >> 2) * kTcCw);
+        for (int sl = 0; sl < kTcSlots; ++sl) tmem_rebias(ta + (uint32_t)(sl * kTcN));
+        tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
-    TcItem it = W.seek(i0);
     int g = 0;   // K chunks so far (ring position)
     // asynchronous builders: the chunks whose copies have been reported
     int reported = 0;
@@ -270,15 +294,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
         const int s = pc % p.stages, e = pc % kTcDxRing;
         unsigned char *dxe = dx_entry(e);
         const int j = (threadIdx.x - (2 + kTcEpiWarps) * 32) >> 1, h = threadIdx.x & 1;
-        const uint32_t two =
-            *reinterpret_cast<const uint32_t *>(dxe + kTcDx + kTcDm + j * 8 + h * 4);
+        const uint32_t two = *reinterpret_cast<const uint32_t *>(dxe + kTcDx + j * 8 + h * 4);
         float *dxs = reinterpret_cast<float *>(dxe);
-        float *dms = reinterpret_cast<float *>(dxe + kTcDx);
-        const float d0 = scale_value((uint16_t)(two & 0xffffu)), d1 = scale_value((uint16_t)(two >> 16));
-        dxs[(2 * h) * kTcN + j] = d0;
-        dxs[(2 * h + 1) * kTcN + j] = d1;
-        dms[(2 * h) * kTcN + j] = -kTcMagic * d0;
-        dms[(2 * h + 1) * kTcN + j] = -kTcMagic * d1;
+        dxs[(2 * h) * kTcN + j] = scale_value((uint16_t)(two & 0xffffu));
+        dxs[(2 * h + 1) * kTcN + j] = scale_value((uint16_t)(two >> 16));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -316,6 +335,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 for (int kc = 0; kc < nkc; ++kc) {
                     const int gg = g + kc, s = gg % p.stages;
                     if (gg >= p.stages) mbar_wait(&empty[s], (gg / p.stages - 1) & 1, &g_err_tc);
+                    Q8_TRACE(15);
                     mbar_arrive_expect_tx(&full[s], kTcA);
                     unsigned char *dst = ring + (size_t)s * kTcStage;
                     if (upgate) {
@@ -347,6 +367,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             for (int kc = 0; kc < nkc; ++kc) {
                 const int gg = g + kc, s = gg % p.stages;
                 builder_wait(gg);
+                Q8_TRACE(13);
                 unsigned char *bst = ring + (size_t)s * kTcStage + kTcA;
                 // nb is even, so both blocks of the pair are present or neither
                 if (xrow && 2 * h < nb - kc * 4) {
@@ -354,7 +375,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     for (int c = 4 * h; c < 4 * h + 4; ++c)
                         cp_async16(bst + (c * ngrp + (j >> 3)) * 128 + (j & 7) * 16,
                                    xrow + kc * 128 + c * 16);
-                    cp_async4(dx_entry(gg % kTcDxRing) + kTcDx + kTcDm + j * 8 + h * 4,
+                    cp_async4(dx_entry(gg % kTcDxRing) + kTcDx + j * 8 + h * 4,
                               dxrow + kc * 4 + 2 * h);
                 }
                 cp_async_commit();
@@ -410,7 +431,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     *reinterpret_cast<uint4 *>(bst + (c * ngrp + (j >> 3)) * 128 + (j & 7) * 16) = lo;
                     *reinterpret_cast<uint4 *>(bst + ((c + 1) * ngrp + (j >> 3)) * 128 + (j & 7) * 16) = hi;
                     dxs[b4 * kTcN + j] = dx;  // [block][row]: a warp's rows are contiguous
-                    dxs[kTcN * 4 + b4 * kTcN + j] = -kTcMagic * dx;
                 }
                 fence_proxy_async_smem();  // generic-proxy writes, read by the tensor cores
                 __syncwarp();
@@ -431,7 +451,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 for (int kc = 0; kc < nkc; ++kc) {
                     const int gg = g + kc, s = gg % p.stages, grp = gg % kTcGroups;
                     mbar_wait(&full[s], (gg / p.stages) & 1, &g_err_tc);
+                    Q8_TRACE(9);
                     if (gg >= kTcGroups) mbar_wait(&sempty[grp], (gg / kTcGroups - 1) & 1, &g_err_tc);
+                    Q8_TRACE(11);
                     tc_fence_after();
                     const uint32_t a_base = smem_u32(ring + (size_t)s * kTcStage);
                     uint64_t adesc = smem_desc(a_base, 16, 1024, 2);
@@ -439,13 +461,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     uint32_t dt = tmem + (uint32_t)(grp * 4 * kTcN);
                     const int gn = min(4, nb - kc * 4);
                     for (int b4 = 0; b4 < gn; ++b4) {
-                        mma_i8(dt, adesc, bdesc, idesc, 0);
+                        mma_i8(dt, adesc, bdesc, idesc, 1);  // onto kTcMagic
                         adesc += 2;  // 32 bytes along K within the swizzled rows
                         bdesc += bstep;
                         dt += kTcN;
                     }
                     tc_commit(&sfull[grp]);   // the chunk's slots hold its block sums
                     tc_commit(&empty[s]);     // the stage is free once these MMAs are done
+                    Q8_TRACE(12);
                 }
             }
             __syncwarp();
@@ -466,16 +489,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
             const bool active = part * kTcCw < it.npad;
             mbar_wait(&dfull[d], (int)((ii / 2) & 1), &g_err_tc);
             const uint16_t *drow = dws(d) + (size_t)row * p.ld_d;
-            uint64_t acc2[kTcCw / 2];  // activation rows (2t2, 2t2 + 1) of the warp's kTcCw
+            float acc[kTcCw];  // the warp's kTcCw activation rows of this thread's weight row
 #pragma unroll
-            for (int t2 = 0; t2 < kTcCw / 2; ++t2) acc2[t2] = 0ull;  // +0.0f in both lanes
+            for (int t = 0; t < kTcCw; ++t) acc[t] = 0.0f;
             for (int kc = 0; kc < nkc; ++kc) {
                 const int gg = g + kc, grp = gg % kTcGroups;
                 const int gn = min(4, nb - kc * 4);
                 const int e = gg % kTcDxRing;
                 mbar_wait(&xfull[e], (gg / kTcDxRing) & 1, &g_err_tc);
+                Q8_TRACE(6);
                 const float *dxs = reinterpret_cast<const float *>(dx_entry(e));
                 mbar_wait(&sfull[grp], (gg / kTcGroups) & 1, &g_err_tc);
+                Q8_TRACE(7);
                 tc_fence_after();
                 uint32_t v[4][kTcCw];
                 if (active) {
@@ -486,6 +511,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                         if (i < gn) tmem_ld_cols(ta + (uint32_t)(i * kTcN), v[i]);
                     }
                     tmem_ld_wait();
+                    // the slots start over from kTcMagic for the next chunk's MMAs
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (i < gn) tmem_rebias(ta + (uint32_t)(i * kTcN));
+                    }
+                    tmem_st_wait();
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -500,36 +531,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     for (int i = 0; i < 4; ++i) {
                         if (i < gn) {
                             const float dw = row_ok ? scale_value(dwh[i]) : 0.0f;
-                            // the block's kTcCw activation scales and their
-                            // -kTcMagic multiples: 16-byte loads
+                            const float dm = -kTcMagic * dw;  // exact
+                            // the block's kTcCw activation scales: 16-byte loads;
+                            // acc[t] = fma(dx[t], round(v[t] * dw), acc[t]) (scalar fma:
+                            // the packed f32x2 form measured 3% slower here)
                             const float4 *dx4 =
                                 reinterpret_cast<const float4 *>(dxs + i * kTcN + part * kTcCw);
-                            const float4 *dm4 = reinterpret_cast<const float4 *>(
-                                dxs + kTcN * 4 + i * kTcN + part * kTcCw);
-                            const uint64_t dw2 = f2_pack(dw, dw);
-                            // acc[t] = fma(dw, round(v[t] * dx[t]), acc[t]), two rows at a time
 #pragma unroll
                             for (int q4 = 0; q4 < kTcCw / 4; ++q4) {
-                                const float4 f = dx4[q4], m = dm4[q4];
+                                const float4 f = dx4[q4];
                                 const int t = 4 * q4;
-                                const uint64_t vd01 = f2_fma(f2_biased(v[i][t], v[i][t + 1]),
-                                                             f2_pack(f.x, f.y), f2_pack(m.x, m.y));
-                                const uint64_t vd23 = f2_fma(f2_biased(v[i][t + 2], v[i][t + 3]),
-                                                             f2_pack(f.z, f.w), f2_pack(m.z, m.w));
-                                acc2[2 * q4] = f2_fma(dw2, vd01, acc2[2 * q4]);
-                                acc2[2 * q4 + 1] = f2_fma(dw2, vd23, acc2[2 * q4 + 1]);
+                                acc[t] = fmaf(f.x, fmaf(__uint_as_float(v[i][t]), dw, dm), acc[t]);
+                                acc[t + 1] = fmaf(f.y, fmaf(__uint_as_float(v[i][t + 1]), dw, dm), acc[t + 1]);
+                                acc[t + 2] = fmaf(f.z, fmaf(__uint_as_float(v[i][t + 2]), dw, dm), acc[t + 2]);
+                                acc[t + 3] = fmaf(f.w, fmaf(__uint_as_float(v[i][t + 3]), dw, dm), acc[t + 3]);
                             }
                         }
                     }
                 }
+                Q8_TRACE(8);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&xempty[e]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&dempty[d]);
-            float acc[kTcCw];
-#pragma unroll
-            for (int t2 = 0; t2 < kTcCw / 2; ++t2) f2_unpack(acc2[t2], acc[2 * t2], acc[2 * t2 + 1]);
             // ---- outputs
             if (upgate) {
                 if (row >= 64 && active) {
@@ -549,6 +574,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     }
                 }
                 named_bar_sync(2, kTcEpiWarps * 32);  // xchg is free for the next item
+                Q8_TRACE(10);
             } else if (row_ok && active) {
 #pragma unroll
                 for (int t = 0; t < kTcCw; ++t) {
@@ -658,6 +684,9 @@ q8_status launch_tc(const q8_tensor *W, bool upgate, const int8_t *aq, const uin
     if (stages > 8) stages = 8;
     if (stages < 3) Q8_FAIL(Q8_E_UNSUPPORTED, "tensor-core path: k=%lld too large", (long long)W->k);
     if (stages <= kTcLag) p.x_async = 0;  // a builder's lag must stay below the ring depth
+    // the walk's running sums sit in the ring's memory at the start
+    if ((max_big + 1) * 4 > (int64_t)stages * kTcStage)
+        Q8_FAIL(Q8_E_UNSUPPORTED, "tensor-core path: %lld experts", (long long)max_big);
     p.stages = stages;
     p.dws_bytes = dws_bytes;
     p.off_dx = stages * kTcStage;

@@ -201,4 +201,5 @@ def test_route_validation(q8):
     assert call(n_used=33, n_exp=64) == 2       # above Q8_MAX_USED
     assert call(x=FAKE_ODD) == 3
     assert call(lg=ctypes.c_void_p(0x10004)) == 3  # logits 8-byte aligned
-    assert call(n_embd=16384, n_exp=1024) == 5  # shared-memory plan too large
+    # the longest rows with the most experts fit one token per cluster, so no
+    # valid shape is refused for its shared-memory plan

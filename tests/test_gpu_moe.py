@@ -275,26 +275,51 @@ def test_bad_ids_reported_without_fault():
     q8.check(ws)
 
 
+TC_MIN_ROWS = 4  # the library's tensor-core threshold (routed rows per expert)
+
+
 @pytest.mark.parametrize("n_exp,n_ff,n_embd,n_tok,n_used", [
     (128, 704, 2816, 1, 8), (128, 704, 2816, 16, 8), (16, 64, 128, 5, 4), (1, 64, 256, 3, 1),
     (32, 96, 2048, 33, 2)])
 def test_fp32_entry_points_match_workspace_path(n_exp, n_ff, n_embd, n_tok, n_used):
     """The small-batch fp32 calls (quantize in the kernel, group in every CTA)
-    give bitwise the results of quantize + grouping + the Q8_0 calls."""
+    give bitwise the results of quantize + grouping + the Q8_0 calls on the
+    dp4a kernels: the up/gate reference asks for the g/u taps, which keep
+    every expert on dp4a; in the down projection the experts with at least
+    TC_MIN_ROWS rows take the tensor cores (P3 against the fp32 entry, whose
+    dp4a sums differ only in the fp32 accumulation order), the rest bitwise."""
     t, UG, DN, ids, p = _layer(n_exp, n_ff, n_embd, n_tok, n_used, seed=300 + n_tok + n_exp)
     x = t["x"].to(DEV)
     xq, xd = q8.quantize_row(x)
-    ref = q8.moe_up_gate_swiglu(UG, xq, xd, ids, want_hq=True)
+    ref = q8.moe_up_gate_swiglu(UG, xq, xd, ids, want_hq=True, want_gu=True)
     h = q8.moe_up_gate_swiglu_fp32(UG, x, ids)
     assert torch.equal(h, ref["h"])
     if ids is not None:
         y = q8.mul_mat_id_fp32(DN, h.reshape(-1, n_ff), ids, True)
-        y2 = q8.mul_mat_id(DN, ref["hq"].reshape(-1, n_ff), ref["hd"].reshape(-1, n_ff // 32),
-                           ids, True)
-        assert torch.equal(y, y2)
-        # the whole step through q8_moe_ffn takes the same kernels
+        hq, hd = ref["hq"].reshape(-1, n_ff), ref["hd"].reshape(-1, n_ff // 32)
+        y2 = q8.mul_mat_id(DN, hq, hd, ids, True)
+        counts = torch.bincount(ids.flatten().long(), minlength=n_exp)
+        dp4a = counts[ids.long()] < TC_MIN_ROWS  # [n_tok, n_used]
+        assert torch.equal(y[dp4a], y2[dp4a])
+        wq, wd = _w_host(DN)
+        hqh = host(hq).reshape(n_tok, n_used, n_ff)
+        hdh = bits(hd).reshape(n_tok, n_used, n_ff // 32)
+        idh, yh, y2h = host(ids), host(y), host(y2)
+        for t_, s in zip(*np.nonzero(~host(dp4a))):
+            e = idh[t_, s]
+            S = S_norm(wq[e], wd[e], hqh[t_, s][None], hdh[t_, s][None])[0]
+            assert np.all(np.abs(yh[t_, s] - y2h[t_, s]) <= 2 * TOL * S + 1e-30)
+        # the whole step through q8_moe_ffn: up to 32 pairs one fused kernel
+        # on dp4a (the fp32 chain's bits); above, the grouped Q8_0 calls
+        # (tensor cores for the experts with at least TC_MIN_ROWS rows)
         out = q8.moe_ffn(UG, DN, x, ids, p)
-        assert torch.equal(out, q8.moe_combine(y2, p))
+        if n_tok * n_used <= 32:
+            assert torch.equal(out, q8.moe_combine(y, p))
+        else:
+            r2 = q8.moe_up_gate_swiglu(UG, xq, xd, ids, want_hq=True)
+            y3 = q8.mul_mat_id(DN, r2["hq"].reshape(-1, n_ff),
+                               r2["hd"].reshape(-1, n_ff // 32), ids, True)
+            assert torch.equal(out, q8.moe_combine(y3, p))
 
 
 def test_fp32_entry_reports_bad_ids():

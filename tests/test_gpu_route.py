@@ -48,6 +48,8 @@ def _check(w, x, n_used, ids, rw, lg):
     (5, 4096, 1024, 32),     # the most experts and the most per token
     (3, 128, 9, 9),          # n_used == n_exp: every expert, in order
     (4, 96, 33, 1),          # n_used == 1: weight 1
+    (7, 8192, 32, 4),        # rows long enough that 3 tokens share a cluster
+    (2, 16384, 64, 8),       # the longest rows: one token per cluster
 ])
 def test_route_matches_oracle(n_tok, n_embd, n_exp, n_used):
     w = synth.normal((n_exp, n_embd), seed=1300 + n_exp, std=synth.W_STD).to(DEV)

@@ -1,13 +1,14 @@
 """The arithmetic identities the tensor-core epilogue relies on to scale an
-int32 Q8_0 block sum v by an activation scale d_x with one fused multiply-add
-(csrc/q8_tc.cu, "Block scaling"):
+int32 Q8_0 block sum v by an fp16 block scale d (the weight row's d_w) with
+one fused multiply-add (csrc/q8_tc.cu, "Block scaling"):
 
   1. adding v to the bit pattern of M = 1.5 * 2^23 gives the fp32 value M + v
      exactly, for every |v| < 2^22 (a block sum is at most 32 * 128 * 128);
-  2. M * d_x is exact in fp32 for every finite fp16 value d_x, so -M * d_x
-     can be stored beside d_x;
-  3. hence fma(M + v, d_x, -M * d_x) = v * d_x rounded once to fp32, the
-     same value as the plain product fp32(v) * d_x.
+     the MMA forms it by accumulating v onto tensor memory that holds M's bits;
+  2. M * d is exact in fp32 for every finite fp16 value d, so -M * d costs
+     one exact multiply;
+  3. hence fma(M + v, d, -M * d) = v * d rounded once to fp32, the same
+     value as the plain product fp32(v) * d.
 
 Checked exhaustively over the fp16 values and over a sweep of v, with the
 fused multiply-add emulated exactly in fp64 (the operands' product needs at
