@@ -38,7 +38,7 @@
  *  - Accuracy: block dots are exact int32; every fp32 output of a matmul lies
  *    within 1e-5 * sum|w * x| (the sum of the dequantized products' magnitudes)
  *    of the exact value of its definition.  Which kernel runs depends on the
- *    shape: experts with >= 16 routed rows in a call, and dense calls with
+ *    shape: experts with >= 4 routed rows in a call, and dense calls with
  *    16..32 activation rows, run on the int8 tensor cores
  *    (tcgen05.mma.kind::i8) when 128 <= k <= 4096 (and, for up/gate, n_ff is
  *    a multiple of 64, and no g_out/u_out is asked for); the rest run on
@@ -334,7 +334,7 @@ q8_status q8_moe_combine(const float *y, const float *route_w, int64_t n_tok, in
  *  n_used == 1), where out = down . quantize(h).
  *  out: fp32 [n_tok][n_embd].
  *  ws: q8_moe_ffn_workspace_size(...) bytes, 256-byte aligned; it also holds
- *      the intermediates (xq, h, hq, per-slot y) and the grid-barrier
+ *      the intermediates (grouping, xq, h, hq, per-slot y) and the grid-barrier
  *      counter of the fused layer kernel, which every fused call advances by
  *      its grid size (the device's SM count).  Zero-fill the workspace before
  *      its first use, use it on one device, and zero it again after a wait
@@ -345,7 +345,11 @@ q8_status q8_moe_combine(const float *y, const float *route_w, int64_t n_tok, in
  * Routed batches of at most 32 pairs (n_tok * n_used) with n_embd <= 4096
  * and n_ff <= 2048 run as ONE cooperative kernel (grouping, up/gate +
  * SwiGLU, a grid barrier, down + combine); the result is bitwise that of
- * the separate calls.
+ * the separate calls.  Larger routed batches run quantize + q8_moe_group +
+ * q8_moe_up_gate_swiglu_pregrouped (h quantized once) +
+ * q8_mul_mat_id_pregrouped + q8_moe_combine, with the same results as those
+ * calls.  Dense batches of up to Q8_SMALL_BATCH_PAIRS rows run the _fp32
+ * calls.
  */
 size_t q8_moe_ffn_workspace_size(int64_t n_tok, int32_t n_used, int64_t n_mat, int64_t n_embd,
                                  int64_t n_ff);
@@ -367,10 +371,11 @@ q8_status q8_moe_ffn(const q8_tensor *up_gate, const q8_tensor *down, const floa
  *  ids: out int32 [n_tok][n_used]; route_w: out fp32 [n_tok][n_used]; they
  *       feed q8_moe_ffn and the other routed calls directly.
  *  logits: optional out fp64 [n_tok][n_exp] (NULL: not written).
- *  Limits: n_exp <= Q8_ROUTE_MAX_EXP, n_used <= min(n_exp, Q8_MAX_USED), and
- *  the shared-memory plan (16 * n_embd + 33 * n_exp bytes) within 227 KB,
- *  else Q8_E_SHAPE / Q8_E_UNSUPPORTED.  NaN logits rank as -infinity.
- * One launch of thread-block clusters (8 CTAs per 4 tokens, the experts split
+ *  Limits: n_exp <= Q8_ROUTE_MAX_EXP, n_used <= min(n_exp, Q8_MAX_USED),
+ *  else Q8_E_SHAPE.  NaN logits rank as -infinity.
+ * One launch of thread-block clusters (8 CTAs per group of up to 4 tokens,
+ * fewer when one token's fp64 activations, logits and flags,
+ * 8 * n_embd + 9 * n_exp bytes, leave no room for more; the experts split
  * across the cluster, the top-k read through distributed shared memory).
  */
 #define Q8_ROUTE_MAX_EXP 1024

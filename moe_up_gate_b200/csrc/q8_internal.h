@@ -180,7 +180,9 @@ q8_status clear_wait_errors_tc();
 constexpr int kTcMinPairs = 4;
 // Dense calls (one matrix) with kTcMinDense..kTcMaxDense activation rows go
 // to the tensor cores too (one pass over the weights): launch_tc with
-// ws == nullptr.
+// ws == nullptr.  (4 rows, the routed experts' line, measured no faster
+// for the dense 8-row up/gate of fp32 activations: their quantization in the
+// gathering warps then costs what the dp4a kernel saves.)
 constexpr int kTcMinDense = 16;
 constexpr int kTcMaxDense = 32;
 bool tc_eligible(const q8_tensor *W, bool upgate);

@@ -378,7 +378,7 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
     XJobs J;
     if (x_once) {
         mbar_wait(R.xfull, 0, &g_err_layer);
-        stage_f32_raw(xs, R.raw, p.k, 1, threadIdx.x, kAll);
+        stage_f32_smem_tpb<2>(xs, R.raw, p.k, 1, [](int j) { return j; }, threadIdx.x, kAll);
         sync_all();
         Q8_TRACE(7);
     }
@@ -476,15 +476,22 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
     if (p.off_hf >= 0) {
         mbar_wait(hbar, 0, &g_err_layer);
         Q8_TRACE(14);
-        stage_f32_smem8(hs, reinterpret_cast<const float *>(smem + p.off_hf), p.n_ff, n_valid,
-                       [&](int j) { return tab[p.lay_pairs + j]; }, threadIdx.x, kAll);
+        stage_f32_smem_tpb<2>(hs, reinterpret_cast<const float *>(smem + p.off_hf), p.n_ff,
+                              n_valid, [&](int j) { return tab[p.lay_pairs + j]; }, threadIdx.x,
+                              kAll);
+        Q8_TRACE(16);
     } else {
         stage_f32_l2(hs, p.h, p.n_ff, n_valid, [&](int j) { return tab[p.lay_pairs + j]; },
                      threadIdx.x, kAll);
     }
-    for (int i = threadIdx.x; i < P; i += kAll) inv[i] = -1;
-    sync_all();
-    for (int j = threadIdx.x; j < n_valid; j += kAll) inv[tab[p.lay_pairs + j]] = j;
+    // inv[pair] = its position in the grouped order (-1: an invalid pair);
+    // at most kLayerMaxPairs pairs, so one pass of a short scan
+    for (int i = threadIdx.x; i < P; i += kAll) {
+        int q = -1;
+        for (int j = 0; j < n_valid; ++j)
+            if (tab[p.lay_pairs + j] == i) q = j;
+        inv[i] = q;
+    }
     sync_all();
     Q8_TRACE(7);
 

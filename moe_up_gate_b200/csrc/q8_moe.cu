@@ -23,23 +23,31 @@ namespace q8 {
 // lists of experts with pairs (split at big_threshold) and the pairs sorted
 // by expert then by pair index (a stable counting sort: one warp walks the
 // pairs in order, 32 at a time, ranking equal experts with __match_any_sync).
+// When they fit (staged), the ids are read from global memory once, by all
+// threads, into shared memory, so the checks and the warp's walk read them
+// there.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) group_kernel(const int32_t *__restrict__ ids, int n_tok,
                                                      int n_used, int n_mat, int big_threshold,
-                                                     int32_t *__restrict__ ws, GroupLayout L) {
+                                                     int staged, int32_t *__restrict__ ws,
+                                                     GroupLayout L) {
     extern __shared__ int sm_group[];
     int *cnt = sm_group;
     int *cursor = sm_group + n_mat;
+    int *sid = sm_group + 2 * n_mat;  // the ids, when staged
     __shared__ int s_err;
     const int P = n_tok * n_used;
     griddep_wait();  // ids may come from, and ws may still be read by, earlier kernels
     griddep_launch_dependents();
     for (int e = threadIdx.x; e < n_mat; e += blockDim.x) cnt[e] = 0;
+    if (staged)
+        for (int p = threadIdx.x; p < P; p += blockDim.x) sid[p] = ids[p];
     if (threadIdx.x == 0) s_err = 0;
     __syncthreads();
+    const int32_t *idv = staged ? sid : ids;
     int err = 0;
     for (int p = threadIdx.x; p < P; p += blockDim.x) {
-        const int e = ids[p];
+        const int e = idv[p];
         if (e < 0 || e >= n_mat) {
             err |= ERR_ID_RANGE;
             continue;
@@ -48,7 +56,7 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t *__restrict__
         const int t = p / n_used;
         const int s = p - t * n_used;
         for (int s2 = 0; s2 < s; ++s2)
-            if (ids[t * n_used + s2] == e) err |= ERR_ID_REPEAT;
+            if (idv[t * n_used + s2] == e) err |= ERR_ID_REPEAT;
     }
     if (err) atomicOr(&s_err, err);
     __syncthreads();
@@ -92,7 +100,7 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t *__restrict__
         // stable scatter of the valid pairs
         for (int base = 0; base < P; base += 32) {
             const int p = base + lane;
-            const int e = p < P ? ids[p] : -1;
+            const int e = p < P ? idv[p] : -1;
             const bool valid = e >= 0 && e < n_mat;
             const int key = valid ? e : n_mat + lane;  // invalid lanes match nobody
             const unsigned m = __match_any_sync(0xffffffffu, key);
@@ -108,9 +116,14 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t *__restrict__
 q8_status launch_group(const int32_t *ids, int64_t n_tok, int32_t n_used, int64_t n_mat,
                        int32_t big_threshold, int32_t *ws, cudaStream_t s) {
     const GroupLayout L = group_layout(n_tok * n_used, n_mat);
-    const size_t smem = (size_t)2 * n_mat * sizeof(int);
+    const int64_t P = n_tok * n_used;
+    // counts and cursors (n_mat <= 4096: at most 32 KB), then the ids when the
+    // whole stays inside the 48 KB a launch gets without an opt-in
+    const int64_t base = 2 * n_mat * (int64_t)sizeof(int);
+    const bool staged = base + P * (int64_t)sizeof(int) + 256 <= 48 * 1024;
+    const size_t smem = (size_t)(base + (staged ? P * (int64_t)sizeof(int) : 0));
     return launch_pdl("group_kernel", group_kernel, dim3(1), dim3(1024), smem, s, ids, (int)n_tok,
-                      n_used, (int)n_mat, big_threshold, ws, L);
+                      n_used, (int)n_mat, big_threshold, staged ? 1 : 0, ws, L);
 }
 
 // Wait timeouts of the kernels in this file (read by q8_check).

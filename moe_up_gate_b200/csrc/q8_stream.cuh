@@ -361,36 +361,33 @@ __device__ __forceinline__ void group_small_warp(const int32_t *__restrict__ ids
     const int e = live ? ids[lane] : -1;
     const bool valid = live && e >= 0 && e < n_mat;
     int err = (live && !valid) ? ERR_ID_RANGE : 0;
+    const unsigned lt = (1u << lane) - 1u;
+    // the lanes naming the same expert (invalid lanes match nobody)
+    const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : n_mat + lane);
+    const bool first = valid && (peers & lt) == 0u;
+    const unsigned vb = __ballot_sync(0xffffffffu, valid);
+    const unsigned firsts = __ballot_sync(0xffffffffu, first);
+    // a repeat: an earlier slot of the same token names the same expert
     const int tok0 = live ? (lane / n_used) * n_used : 0;
-    int rank = 0, cnt_e = 0, dpos = 0;
-    bool first = true;
+    const unsigned tok_mask = (unsigned)((((uint64_t)1 << n_used) - 1u) << tok0);
+    if (valid && (peers & lt & tok_mask) != 0u) err |= ERR_ID_REPEAT;
+    // rank: the valid pairs of smaller experts, then this expert's earlier
+    // pairs; dpos: the distinct smaller experts
+    int rank = __popc(peers & lt), dpos = 0;
 #pragma unroll
     for (int s2 = 0; s2 < 32; ++s2) {
         const int e2 = __shfl_sync(0xffffffffu, e, s2);
-        const bool v2 = __shfl_sync(0xffffffffu, valid ? 1 : 0, s2) != 0;
-        if (!valid || !v2) continue;
-        if (e2 < e || (e2 == e && s2 < lane)) ++rank;
-        if (e2 == e) {
-            ++cnt_e;
-            if (s2 < lane) {
-                first = false;
-                if (s2 >= tok0) err |= ERR_ID_REPEAT;
-            }
+        if (e2 < e) {
+            rank += (int)((vb >> s2) & 1u);
+            dpos += (int)((firsts >> s2) & 1u);
         }
     }
-    const unsigned firsts = __ballot_sync(0xffffffffu, valid && first);
-#pragma unroll
-    for (int s2 = 0; s2 < 32; ++s2) {
-        const int e2 = __shfl_sync(0xffffffffu, e, s2);
-        if (((firsts >> s2) & 1u) && e2 < e) ++dpos;
-    }
     if (valid) tab[L.pairs + rank] = lane;
-    if (valid && first) {
+    if (first) {
         tab[L.list_small + dpos] = e;
-        tab[L.count + e] = cnt_e;
+        tab[L.count + e] = __popc(peers);
         tab[L.offset + e] = rank;
     }
-    const unsigned vb = __ballot_sync(0xffffffffu, valid);
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) err |= __shfl_xor_sync(0xffffffffu, err, o);
     if (lane == 0) {
@@ -612,6 +609,59 @@ __device__ __forceinline__ void stage_f32_smem8(const XStage &xs, const float *s
                                (((uint32_t)quantize_one(f.z, id) & 0xffu) << 16) |
                                (((uint32_t)quantize_one(f.w, id) & 0xffu) << 24);
             *reinterpret_cast<uint32_t *>(xs.q + (size_t)j * k + b * QK + 4 * part) = w;
+            if (part == 0) xs.dx[(size_t)j * nb + b] = scale_value(scale_bits(d32));
+        }
+    }
+}
+
+// The same with TPB threads per 32-block (TPB = 2, 4 or 8): fewer rounds of
+// the block's scale divisions when the rows are few and the threads many
+// (8 rows of 704 take one round of 2 threads per block among 512 threads,
+// against three of 8).  amax is exact and every code is formed as in
+// quantize_block_thread, so the bits do not depend on TPB.
+template <int TPB, class RowFn>
+__device__ __forceinline__ void stage_f32_smem_tpb(const XStage &xs, const float *src, int k,
+                                                   int n, RowFn arow, int tid, int nthr) {
+    static_assert(TPB == 2 || TPB == 4 || TPB == 8, "threads per block");
+    constexpr int F4 = 8 / TPB;  // float4s of the block per thread
+    const int nb = k / QK;
+    const int total = n * nb;
+    const int grp = tid / TPB, part = tid % TPB;
+    const int ngrp = nthr / TPB;
+    for (int base = 0; base < total; base += ngrp) {  // the same trip count in every lane
+        const int blk = base + grp;
+        const bool live = blk < total;
+        int j = 0, b = 0;
+        float4 f[F4];
+#pragma unroll
+        for (int i = 0; i < F4; ++i) f[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (live) {
+            j = blk / nb;
+            b = blk - j * nb;
+            const float4 *p4 = reinterpret_cast<const float4 *>(src + (size_t)arow(j) * k + b * QK);
+#pragma unroll
+            for (int i = 0; i < F4; ++i) f[i] = p4[part * F4 + i];
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < F4; ++i)
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f[i].x), fabsf(f[i].y)),
+                                     fmaxf(fabsf(f[i].z), fabsf(f[i].w))));
+#pragma unroll
+        for (int o = 1; o < TPB; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (live) {
+            const float d32 = block_scale(amax);
+            const float id = block_inv_scale(d32);
+            uint32_t w[F4];
+#pragma unroll
+            for (int i = 0; i < F4; ++i)
+                w[i] = ((uint32_t)quantize_one(f[i].x, id) & 0xffu) |
+                       (((uint32_t)quantize_one(f[i].y, id) & 0xffu) << 8) |
+                       (((uint32_t)quantize_one(f[i].z, id) & 0xffu) << 16) |
+                       (((uint32_t)quantize_one(f[i].w, id) & 0xffu) << 24);
+            uint32_t *dst = reinterpret_cast<uint32_t *>(xs.q + (size_t)j * k + b * QK + 4 * F4 * part);
+#pragma unroll
+            for (int i = 0; i < F4; ++i) dst[i] = w[i];
             if (part == 0) xs.dx[(size_t)j * nb + b] = scale_value(scale_bits(d32));
         }
     }

@@ -41,13 +41,11 @@ constexpr int kTcDxRing = 8;        // entries of the activation-scale ring, one
 constexpr int kTcDx = kTcN * 4 * 4; // an entry: the chunk's 4 blocks' scales d_x, fp32 [block][row]
 constexpr int kTcDh = kTcN * 4 * 2; // then d_x as copied, fp16 [row][block]
 constexpr int kTcDxEntry = kTcDx + kTcDh;
-// Block scaling.  Every tensor-memory slot holds the bits of kTcMagic before
-// its MMA, which accumulates onto them: a block sum |v| < 2^22 then reads
-// back as the fp32 value kTcMagic + v, exactly.  kTcMagic * d_w is exact in
-// fp32 (d_w is an fp16 value, 11 significant bits), so
+// Block scaling.  A block sum |v| < 2^22 becomes the fp32 value kTcMagic + v
+// exactly by an integer add of v to the bits of kTcMagic.  kTcMagic * d_w is
+// exact in fp32 (d_w is an fp16 value, 11 significant bits), so
 // fma(kTcMagic + v, d_w, -kTcMagic * d_w) is v * d_w rounded once; the
-// epilogue then adds d_x times that to the row's sum and writes kTcMagic back
-// into the slot for its next block.
+// epilogue then adds d_x times that to the row's sum.
 constexpr float kTcMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr uint32_t kTcMagicBits = 0x4B400000u;
 constexpr int kTcLag = 3;           // chunks a builder keeps in flight before it reports one
@@ -102,17 +100,15 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ float tc_silu(float z) { return z / (1.0f + expf(-z)); }
 
+// A block sum |v| < 2^22 (int32 bits) as the fp32 value kTcMagic + v, exactly.
+__device__ __forceinline__ float biased(uint32_t v) {
+    return __int_as_float((int)v + (int)kTcMagicBits);
+}
+
 // A warp's kTcCw columns of one slot (this thread's lane).
 __device__ __forceinline__ void tmem_ld_cols(uint32_t addr, uint32_t (&v)[16]) { tmem_ld16(addr, v); }
 __device__ __forceinline__ void tmem_ld_cols(uint32_t addr, uint32_t (&v)[8]) { tmem_ld8(addr, v); }
 
-// Set this thread's kTcCw columns of a slot back to kTcMagic.
-__device__ __forceinline__ void tmem_rebias(uint32_t addr) {
-    if constexpr (kTcCw == 8)
-        tmem_fill8(addr, kTcMagicBits);
-    else
-        tmem_fill16(addr, kTcMagicBits);
-}
 
 // The CTA's work items, in order: (expert of the tensor-core list, pass of
 // kTcN of its rows, weight tile).  Every role walks the same sequence.
@@ -272,17 +268,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    // every slot starts at kTcMagic (an epilogue warp sets its lane quarter's
-    // columns of each slot; the MMAs accumulate onto them)
-    if (warp >= 2 && warp < 2 + kTcEpiWarps) {
-        const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) +
-                            (uint32_t)(((warp - 2) >> 2) * kTcCw);
-        for (int sl = 0; sl < kTcSlots; ++sl) tmem_rebias(ta + (uint32_t)(sl * kTcN));
-        tmem_st_wait();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
 
     int g = 0;   // K chunks so far (ring position)
     // asynchronous builders: the chunks whose copies have been reported
@@ -312,6 +297,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
         if (gg >= kTcDxRing)
             mbar_wait(&xempty[gg % kTcDxRing], (gg / kTcDxRing - 1) & 1, &g_err_tc);
     };
+    // The ring cursor of the single-thread roles (producer, MMA issuer): the
+    // stage of chunk gg, the parity of its phase, and whether the ring has
+    // wrapped (before that every stage is free).  Set once per item and
+    // advanced per chunk, so no division by the stage count per chunk.
+    struct RingCursor {
+        int s, stages;
+        uint32_t ph;
+        bool wrapped;
+        __device__ __forceinline__ RingCursor(int gg, int n)
+            : s(gg % n), stages(n), ph((uint32_t)(gg / n) & 1u), wrapped(gg >= n) {}
+        __device__ __forceinline__ void next() {
+            if (++s == stages) {
+                s = 0;
+                ph ^= 1u;
+                wrapped = true;
+            }
+        }
+    };
     for (int64_t ii = 0; ii < i1 - i0; ++ii, W.next(it)) {
         const int d = (int)(ii & 1);
         const int row0 = it.tile * (upgate ? 64 : 128);
@@ -332,18 +335,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                     mbar_arrive_expect_tx(&dfull[d], bytes);
                     bulk_g2s(dws(d), p.wd + (mrow + row0) * p.ld_d, bytes, &dfull[d]);
                 }
-                for (int kc = 0; kc < nkc; ++kc) {
-                    const int gg = g + kc, s = gg % p.stages;
-                    if (gg >= p.stages) mbar_wait(&empty[s], (gg / p.stages - 1) & 1, &g_err_tc);
+                RingCursor rc(g, p.stages);
+                for (int kc = 0; kc < nkc; ++kc, rc.next()) {
+                    if (rc.wrapped) mbar_wait(&empty[rc.s], rc.ph ^ 1u, &g_err_tc);
                     Q8_TRACE(15);
-                    mbar_arrive_expect_tx(&full[s], kTcA);
-                    unsigned char *dst = ring + (size_t)s * kTcStage;
+                    mbar_arrive_expect_tx(&full[rc.s], kTcA);
+                    unsigned char *dst = ring + (size_t)rc.s * kTcStage;
                     if (upgate) {
-                        tma_load_2d(dst, &p.tmap, kc * 128, (int)(mrow + row0), &full[s]);
+                        tma_load_2d(dst, &p.tmap, kc * 128, (int)(mrow + row0), &full[rc.s]);
                         tma_load_2d(dst + kTcA / 2, &p.tmap, kc * 128, (int)(mrow + p.n_ff + row0),
-                                    &full[s]);
+                                    &full[rc.s]);
                     } else {
-                        tma_load_2d(dst, &p.tmap, kc * 128, (int)(mrow + row0), &full[s]);
+                        tma_load_2d(dst, &p.tmap, kc * 128, (int)(mrow + row0), &full[rc.s]);
                     }
                 }
             }
@@ -364,6 +367,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 xrow = p.aq + r * k;
                 dxrow = p.ad + r * nb;
             }
+
             for (int kc = 0; kc < nkc; ++kc) {
                 const int gg = g + kc, s = gg % p.stages;
                 builder_wait(gg);
@@ -448,26 +452,40 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 const uint32_t idesc = idesc_i8(it.npad);
                 const uint32_t lbo = (uint32_t)(it.npad / 8) * 128;
                 const uint64_t bstep = (uint64_t)((2 * lbo) >> 4);  // next block: 2 core-matrix columns
-                for (int kc = 0; kc < nkc; ++kc) {
-                    const int gg = g + kc, s = gg % p.stages, grp = gg % kTcGroups;
-                    mbar_wait(&full[s], (gg / p.stages) & 1, &g_err_tc);
+                // stage 0's descriptors; stage s adds s * kTcStage / 16 to the
+                // address field (the ring lies below 256 KB: no carry out of it)
+                const uint32_t ring0 = smem_u32(ring);
+                const uint64_t adesc0 = smem_desc(ring0, 16, 1024, 2);
+                const uint64_t bdesc0 = smem_desc(ring0 + kTcA, lbo, 128, 0);
+                RingCursor rc(g, p.stages);
+                for (int kc = 0; kc < nkc; ++kc, rc.next()) {
+                    const int gg = g + kc, grp = gg & (kTcGroups - 1);
+                    mbar_wait(&full[rc.s], rc.ph, &g_err_tc);
                     Q8_TRACE(9);
-                    if (gg >= kTcGroups) mbar_wait(&sempty[grp], (gg / kTcGroups - 1) & 1, &g_err_tc);
+                    if (gg >= kTcGroups) mbar_wait(&sempty[grp], ((gg / kTcGroups) - 1) & 1, &g_err_tc);
                     Q8_TRACE(11);
                     tc_fence_after();
-                    const uint32_t a_base = smem_u32(ring + (size_t)s * kTcStage);
-                    uint64_t adesc = smem_desc(a_base, 16, 1024, 2);
-                    uint64_t bdesc = smem_desc(a_base + kTcA, lbo, 128, 0);
+                    const uint64_t soff = (uint64_t)(rc.s * (kTcStage >> 4));
+                    uint64_t adesc = adesc0 + soff, bdesc = bdesc0 + soff;
                     uint32_t dt = tmem + (uint32_t)(grp * 4 * kTcN);
-                    const int gn = min(4, nb - kc * 4);
-                    for (int b4 = 0; b4 < gn; ++b4) {
-                        mma_i8(dt, adesc, bdesc, idesc, 1);  // onto kTcMagic
-                        adesc += 2;  // 32 bytes along K within the swizzled rows
-                        bdesc += bstep;
-                        dt += kTcN;
+                    if (nb - kc * 4 >= 4) {
+#pragma unroll
+                        for (int b4 = 0; b4 < 4; ++b4) {
+                            mma_i8(dt, adesc, bdesc, idesc, 0);
+                            adesc += 2;  // 32 bytes along K within the swizzled rows
+                            bdesc += bstep;
+                            dt += kTcN;
+                        }
+                    } else {
+                        for (int b4 = 0; b4 < nb - kc * 4; ++b4) {
+                            mma_i8(dt, adesc, bdesc, idesc, 0);
+                            adesc += 2;
+                            bdesc += bstep;
+                            dt += kTcN;
+                        }
                     }
                     tc_commit(&sfull[grp]);   // the chunk's slots hold its block sums
-                    tc_commit(&empty[s]);     // the stage is free once these MMAs are done
+                    tc_commit(&empty[rc.s]);  // the stage is free once these MMAs are done
                     Q8_TRACE(12);
                 }
             }
@@ -511,12 +529,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                         if (i < gn) tmem_ld_cols(ta + (uint32_t)(i * kTcN), v[i]);
                     }
                     tmem_ld_wait();
-                    // the slots start over from kTcMagic for the next chunk's MMAs
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        if (i < gn) tmem_rebias(ta + (uint32_t)(i * kTcN));
-                    }
-                    tmem_st_wait();
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -534,17 +546,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                             const float dm = -kTcMagic * dw;  // exact
                             // the block's kTcCw activation scales: 16-byte loads;
                             // acc[t] = fma(dx[t], round(v[t] * dw), acc[t]) (scalar fma:
-                            // the packed f32x2 form measured 3% slower here)
+                            // the packed f32x2 form measured 3% slower here; biasing v in
+                            // tensor memory, rewritten after every read, 5% slower than
+                            // the integer add)
                             const float4 *dx4 =
                                 reinterpret_cast<const float4 *>(dxs + i * kTcN + part * kTcCw);
 #pragma unroll
                             for (int q4 = 0; q4 < kTcCw / 4; ++q4) {
                                 const float4 f = dx4[q4];
                                 const int t = 4 * q4;
-                                acc[t] = fmaf(f.x, fmaf(__uint_as_float(v[i][t]), dw, dm), acc[t]);
-                                acc[t + 1] = fmaf(f.y, fmaf(__uint_as_float(v[i][t + 1]), dw, dm), acc[t + 1]);
-                                acc[t + 2] = fmaf(f.z, fmaf(__uint_as_float(v[i][t + 2]), dw, dm), acc[t + 2]);
-                                acc[t + 3] = fmaf(f.w, fmaf(__uint_as_float(v[i][t + 3]), dw, dm), acc[t + 3]);
+                                acc[t] = fmaf(f.x, fmaf(biased(v[i][t]), dw, dm), acc[t]);
+                                acc[t + 1] = fmaf(f.y, fmaf(biased(v[i][t + 1]), dw, dm), acc[t + 1]);
+                                acc[t + 2] = fmaf(f.z, fmaf(biased(v[i][t + 2]), dw, dm), acc[t + 2]);
+                                acc[t + 3] = fmaf(f.w, fmaf(biased(v[i][t + 3]), dw, dm), acc[t + 3]);
                             }
                         }
                     }

@@ -58,24 +58,6 @@ __device__ __forceinline__ void tmem_ld8(uint32_t addr, uint32_t (&v)[8]) {
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-// Set 8 (or 16) consecutive 32-bit columns of this thread's lane to one value
-// (32x32b shape).
-__device__ __forceinline__ void tmem_fill8(uint32_t addr, uint32_t val) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1};"
-                 ::"r"(addr), "r"(val)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_fill16(uint32_t addr, uint32_t val) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(addr),
-        "r"(val)
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() {
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
 // ---------------------------------------------------------------------------
 // MMA: D[tmem] = A[smem] x B[smem]^T (int8 x int8 -> int32), M=128, cta_group::1.
 // accumulate == 0 overwrites D.  Issued by one thread.

@@ -4,7 +4,6 @@ one fused multiply-add (csrc/q8_tc.cu, "Block scaling"):
 
   1. adding v to the bit pattern of M = 1.5 * 2^23 gives the fp32 value M + v
      exactly, for every |v| < 2^22 (a block sum is at most 32 * 128 * 128);
-     the MMA forms it by accumulating v onto tensor memory that holds M's bits;
   2. M * d is exact in fp32 for every finite fp16 value d, so -M * d costs
      one exact multiply;
   3. hence fma(M + v, d, -M * d) = v * d rounded once to fp32, the same
