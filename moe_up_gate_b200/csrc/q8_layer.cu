@@ -168,7 +168,7 @@ __device__ __forceinline__ void stage_f32_l2(const XStage &xs, const float *src,
 template <int RPW, int ITERS, int G>
 __device__ __forceinline__ void layer_pairs_run(const Ring &R, const XStage &xs,
                                                 const LayerParams &p, const int32_t *tab,
-                                                int tpm, int half, int64_t ta0, int64_t ta1,
+                                                int tpm, int half, int ta0, int ta1,
                                                 int grp, int w8) {
     const int lane = threadIdx.x & 31;
     const int k = p.k, nb = k / QK, ld_d = (int)p.ug_ld_d;
@@ -193,8 +193,8 @@ __device__ __forceinline__ void layer_pairs_run(const Ring &R, const XStage &xs,
     const int up_idx = idx + H;
     const int up_lane = reduce_scatter_lane<VP>(up_idx < VP ? up_idx : 0);
     const bool writer = (lane & (32 / VP - 1)) == 0 && idx < H;
-    for (int64_t t = ta0 + grp; t < ta1; t += G) {
-        const int it = (int)(t - ta0);
+    for (int t = ta0 + grp; t < ta1; t += G) {
+        const int it = t - ta0;
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_layer);
         Q8_TRACE(6);
@@ -290,6 +290,7 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
     }
     Q8_TRACE(3);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    Q8_TRACE(25);
     const int n_exp = tab[WS_N_SMALL];
     const Geo ga = geo_pair_for_k(p.k);
     const int half = ga.nr / 2;
@@ -298,16 +299,20 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
     const int units = (p.k + nrb - 1) / nrb;
     const int sg_per_unit = (n_exp + kCW - 1) / kCW;
     const int xmax = p.plan.xmax;
-    int64_t ta0, ta1, ub0, ub1;
-    my_tiles((int64_t)n_exp * tpm, &ta0, &ta1);
-    my_tiles(units, &ub0, &ub1);
+    // this CTA's tiles and units (32-bit: at most 32 experts of 2048 / 8 tiles)
+    const int n_tiles_a = n_exp * tpm;
+    const int ta0 = (int)((unsigned)n_tiles_a * blockIdx.x / gridDim.x);
+    const int ta1 = (int)((unsigned)n_tiles_a * (blockIdx.x + 1) / gridDim.x);
+    const int ub0 = (int)((unsigned)units * blockIdx.x / gridDim.x);
+    const int ub1 = (int)((unsigned)units * (blockIdx.x + 1) / gridDim.x);
     auto expert = [&](int i) { return tab[p.lay_list + i]; };
 
     if (warp == kProd) {  // ---------------- producer
+        Q8_TRACE(24);
         if (lane == 0) {
             int it = 0;
             XJobs J;
-            auto jobs = [&](int64_t t, int when) {
+            auto jobs = [&](int t, int when) {
                 const int e = expert((int)(t / tpm));
                 const int cnt = tab[p.lay_count + e];
                 const int32_t *plist = tab + p.lay_pairs + tab[p.lay_offset + e];
@@ -319,7 +324,7 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
                     }, &g_err_layer);
                 }
             };
-            for (int64_t t = ta0; t < ta1; ++t, ++it) {  // phase A: gate/up tiles
+            for (int t = ta0; t < ta1; ++t, ++it) {  // phase A: gate/up tiles
                 const int s = it % R.stages;
                 if (R.raw_rows > 0 && !x_once) jobs(t, 0);
                 if (it >= R.stages) mbar_wait(&R.empty[s], (it / R.stages - 1) & 1, &g_err_layer);
@@ -337,7 +342,7 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
                          &R.full[s]);
                 if (R.raw_rows > 0 && !x_once) jobs(t, 1);
             }
-            for (int64_t u = ub0; u < ub1; ++u) {  // phase B: down rows of every expert
+            for (int u = ub0; u < ub1; ++u) {  // phase B: down rows of every expert
                 const int r0 = (int)u * nrb;
                 const int nrv = min(nrb, p.k - r0);
                 for (int sg = 0; sg < sg_per_unit; ++sg, ++it) {
@@ -401,8 +406,8 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
             phase_a_done = true;
         }
     }
-    for (int64_t t = ta0 + grp; t < ta1 && !phase_a_done; t += G) {
-        const int it = (int)(t - ta0);
+    for (int t = ta0 + grp; t < ta1 && !phase_a_done; t += G) {
+        const int it = t - ta0;
         const int s = it % R.stages;
         mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_layer);
         Q8_TRACE(6);
@@ -497,13 +502,13 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
 
     // ---------------- phase B: y = down . hq, out = sum_s p y
     const Geo gb{nrb * kCW, 1, nrb};
-    const int itb = (int)(ta1 - ta0);  // ring position of the first phase-B stage
+    const int itb = ta1 - ta0;  // ring position of the first phase-B stage
     const int gtid = threadIdx.x - grp * kCT;
-    for (int64_t u = ub0 + grp; u < ub1; u += G) {
+    for (int u = ub0 + grp; u < ub1; u += G) {
         const int r0 = (int)u * nrb;
         const int nrv = min(nrb, p.k - r0);
         for (int sg = 0; sg < sg_per_unit; ++sg) {
-            const int it = itb + (int)(u - ub0) * sg_per_unit + sg;
+            const int it = itb + (u - ub0) * sg_per_unit + sg;
             const int s = it % R.stages;
             mbar_wait(&R.full[s], (it / R.stages) & 1, &g_err_layer);
             Q8_TRACE(6);
@@ -543,6 +548,7 @@ __global__ void __launch_bounds__((G * kCW + 1) * 32, 1)
             const int t = i / nrv;
             const int rr = i - t * nrv;
             float acc = 0.0f;
+#pragma unroll 8
             for (int s2 = 0; s2 < p.n_used; ++s2) {
                 const int q = inv[t * p.n_used + s2];
                 acc = fmaf(s_rw[t * p.n_used + s2], q >= 0 ? ybuf[q * nrb + rr] : 0.0f, acc);
