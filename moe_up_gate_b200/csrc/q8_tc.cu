@@ -504,7 +504,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_kernel(const __grid_constant
                 grow = row0 + row;
                 row_ok = grow < p.rows;
             }
-            const bool active = part * kTcCw < it.npad;
+            // a warp whose columns all lie past the pass's rows (the MMA's N is
+            // padded to 16 or 32) reads and scales nothing (skipping the columns
+            // past the rows inside a warp's part too measured slower)
+            const bool active = part * kTcCw < it.n;
             mbar_wait(&dfull[d], (int)((ii / 2) & 1), &g_err_tc);
             const uint16_t *drow = dws(d) + (size_t)row * p.ld_d;
             float acc[kTcCw];  // the warp's kTcCw activation rows of this thread's weight row
