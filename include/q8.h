@@ -374,8 +374,8 @@ q8_status q8_moe_ffn(const q8_tensor *up_gate, const q8_tensor *down, const floa
  *  Limits: n_exp <= Q8_ROUTE_MAX_EXP, n_used <= min(n_exp, Q8_MAX_USED),
  *  else Q8_E_SHAPE.  NaN logits rank as -infinity.
  * One launch of thread-block clusters (8 CTAs per group of up to 4 tokens,
- * fewer when one token's fp64 activations, logits and flags,
- * 8 * n_embd + 9 * n_exp bytes, leave no room for more; the experts split
+ * fewer when one token's fp64 activations and logits, 8 * n_embd + 8 *
+ * n_exp bytes, leave no room for more; the experts split
  * across the cluster, the top-k read through distributed shared memory).
  */
 #define Q8_ROUTE_MAX_EXP 1024

@@ -48,8 +48,7 @@ struct RouteParams {
     int32_t *ids;    // [n_tok][n_used]
     float *route_w;  // [n_tok][n_used]
     double *logits;  // [n_tok][n_exp] or nullptr
-    int off_lg;      // shared-memory offsets (bytes)
-    int off_sel;
+    int off_lg;      // shared-memory offset (bytes) of the logits
 };
 
 // Larger logit first; equal logits by the lower expert index (a total order
@@ -73,6 +72,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
     double2 *xb = xa + (size_t)p.tpc * n4;
     double *lg = reinterpret_cast<double *>(smem + p.off_lg);  // [tpc][n_exp], own experts only
     const int n_warps = (int)(blockDim.x >> 5);
+    Q8_TRACE(0);
     griddep_wait();  // x may come from the preceding kernel
     griddep_launch_dependents();
     for (int i = threadIdx.x; i < nt * n4; i += blockDim.x) {
@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
         xb[i] = make_double2((double)v.z, (double)v.w);
     }
     __syncthreads();
+    Q8_TRACE(1);
     // logits of this CTA's experts: warp per expert row
     for (int e = rank + C * warp; e < p.n_exp; e += C * n_warps) {
         const float4 *wr = reinterpret_cast<const float4 *>(p.w + (int64_t)e * p.n_embd);
@@ -123,7 +124,9 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
                 if (t < nt) lg[t * p.n_exp + e] = acc[t];
         }
     }
+    Q8_TRACE(2);
     cluster.sync();  // every CTA's logits are written (release / acquire)
+    Q8_TRACE(3);
     if (p.logits) {
         for (int i = threadIdx.x; i < nt * p.n_exp; i += blockDim.x) {
             const int t = i / p.n_exp, e = i - t * p.n_exp;
@@ -139,29 +142,40 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
         }
         __syncthreads();
     }
+    Q8_TRACE(4);
     cluster.sync();  // CTA 0 is done reading the others' shared memory
+    Q8_TRACE(5);
     if (rank == 0 && warp < nt) {
-        // token t0 + warp: repeated warp argmax over the not-yet-selected experts
+        // token t0 + warp: repeated warp argmax over the not-yet-selected
+        // experts.  Lane l owns experts l, l + 32, ... (at most 32: n_exp <=
+        // 1024) and keeps its best unselected one in registers; each round
+        // the warp's best is the next selection, and only its owner lane
+        // looks at its candidates again.
         const int t = warp;
-        unsigned char *sel = smem + p.off_sel + t * p.n_exp;
-        for (int e = lane; e < p.n_exp; e += 32) sel[e] = 0;
-        __syncwarp();
         auto logit = [&](int e) -> double {  // NaN ranks as -infinity
             const double v = lg[t * p.n_exp + e];
             return v != v ? -INFINITY : v;
         };
-        double first = 0.0, mine = -INFINITY;  // lane k keeps the k-th selected logit
-        for (int k = 0; k < p.n_used; ++k) {
-            double bv = -INFINITY;
-            int bi = p.n_exp;  // no candidate yet
-            for (int e = lane; e < p.n_exp; e += 32) {
-                if (sel[e]) continue;
+        uint32_t taken = 0;  // bit c: expert lane + 32 c is selected
+        double lv = -INFINITY;
+        int li = p.n_exp;  // this lane's best unselected expert (n_exp: none)
+        auto rescan = [&]() {
+            lv = -INFINITY;
+            li = p.n_exp;
+            for (int e = lane, c = 0; e < p.n_exp; e += 32, ++c) {
+                if ((taken >> c) & 1u) continue;
                 const double v = logit(e);
-                if (bi == p.n_exp || route_before(v, e, bv, bi)) {
-                    bv = v;
-                    bi = e;
+                if (li == p.n_exp || route_before(v, e, lv, li)) {
+                    lv = v;
+                    li = e;
                 }
             }
+        };
+        rescan();
+        double first = 0.0, mine = -INFINITY;  // lane k keeps the k-th selected logit
+        for (int k = 0; k < p.n_used; ++k) {
+            double bv = lv;
+            int bi = li;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -171,21 +185,25 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
                     bi = oi;
                 }
             }
-            // n_used <= n_exp: some expert is always left, so bi < n_exp
-            if (lane == 0) {
-                sel[bi] = 1;
-                p.ids[(int64_t)(t0 + t) * p.n_used + k] = bi;
-            }
+            // n_used <= n_exp: some expert is always left, so bi < n_exp, and
+            // every lane holds the same (bv, bi)
+            if (lane == 0) p.ids[(int64_t)(t0 + t) * p.n_used + k] = bi;
             if (k == 0) first = bv;
             if (lane == k) mine = bv;
+            if ((bi & 31) == lane) {
+                taken |= 1u << (bi >> 5);
+                rescan();
+            }
             __syncwarp();
         }
+        Q8_TRACE(6);
         // softmax over the selected logits (largest first), fp64
         const double ex = lane < p.n_used ? exp(mine - first) : 0.0;
         double sum = ex;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         if (lane < p.n_used) p.route_w[(int64_t)(t0 + t) * p.n_used + lane] = (float)(ex / sum);
+        Q8_TRACE(7);
     }
 }
 
@@ -224,15 +242,14 @@ extern "C" q8_status q8_route(const float *w_router, const float *x, int64_t n_t
     p.logits = logits;
     const int C = kRouteCluster;
     // tokens per cluster: as many as fit (up to kRouteTok), the fp64 rows of
-    // x, the logits and the selection flags of each
-    const int per_tok = (int)n_embd * 8 + (int)n_exp * 9 + 32;
+    // x and the logits of each
+    const int per_tok = (int)n_embd * 8 + (int)n_exp * 8 + 32;
     p.tpc = std::min<int>(kRouteTok, kSmemLimitRoute / per_tok);
     Q8_REQUIRE(p.tpc >= 1, Q8_E_UNSUPPORTED, "%s: shared-memory plan too large", fn);
     const int x_bytes = p.tpc * (int)n_embd * 8;  // two double2 arrays (xa, xb)
     p.off_lg = (x_bytes + 15) / 16 * 16;
     const int lg_bytes = p.tpc * (int)n_exp * 8;
-    p.off_sel = p.off_lg + lg_bytes;
-    const int smem = p.off_sel + p.tpc * (int)n_exp;
+    const int smem = p.off_lg + lg_bytes;
     Q8_REQUIRE(smem <= kSmemLimitRoute, Q8_E_UNSUPPORTED, "%s: shared-memory plan too large", fn);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
