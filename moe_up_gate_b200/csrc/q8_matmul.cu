@@ -543,7 +543,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                     cur + 1 < p.n_desc ? min(te, (int64_t)p.pr[cur + 1].tile_begin) : te;
                 if (cur != staged) {
                     if (unsynced) named_bar_sync(kBarConsumers, kCT);
-                    stage_job_f32(R, J, xs, qv.x, qv.k, 1, [](int j) { return j; },
+                    stage_job_f32<true>(R, J, xs, qv.x, qv.k, 1, [](int j) { return j; },
                                   &g_err_matmul);
                     named_bar_sync(kBarConsumers, kCT);
                     Q8_TRACE(7);
@@ -590,7 +590,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                 // with the staged rows before they are replaced
                 if (unsynced) named_bar_sync(kBarConsumers, kCT);
                 unsynced = false;
-                stage_job_f32(R, J, xs, q.x, q.k, nx, [&](int j) { return x0 + j; },
+                stage_job_f32<true>(R, J, xs, q.x, q.k, nx, [&](int j) { return x0 + j; },
                               &g_err_matmul);
                 named_bar_sync(kBarConsumers, kCT);
                 Q8_TRACE(7);

@@ -227,7 +227,9 @@ struct UpGateParams {
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 
-template <int NT>
+// Dense: an instantiation for dense calls (no grouping table, no ids), whose
+// activation staging takes the wide form (stage_f32).
+template <int NT, bool Dense>
 __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     up_gate_kernel(const __grid_constant__ UpGateParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -238,8 +240,8 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     const int half_rows = g.nr / 2;
     const int tpm = p.n_ff / half_rows;
     griddep_launch_dependents();
-    const int32_t *tab = p.ws;
-    if (p.ids) {
+    const int32_t *tab = Dense ? nullptr : p.ws;
+    if (!Dense && p.ids) {
         griddep_wait();
         int32_t *stab = reinterpret_cast<int32_t *>(smem + p.plan.off_tab);
         GroupLayout L{};
@@ -339,7 +341,7 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                     return routed ? pr / p.n_used : pr;
                 };
                 if (p.xf)
-                    stage_job_f32(R, J, xs, p.xf, p.k, nx, arow, &g_err_moe);
+                    stage_job_f32<Dense>(R, J, xs, p.xf, p.k, nx, arow, &g_err_moe);
                 else
                     stage_q8(xs, p.xq, p.xd, p.k, nx, arow);
                 named_bar_sync(kBarConsumers, kCT);
@@ -413,11 +415,19 @@ static q8_status launch_up_gate(const UpGateParams &base, RowPlan rp, int64_t sl
     const Geo g = geo_pair_for_k(p.k);
     const int64_t tiles = slots * (p.n_ff / (g.nr / 2));
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * p.plan.ctas, tiles));
+    if (!p.ids && !p.ws) {
+        switch (nt) {
+            case 1: return launch_stream(up_gate_kernel<1, true>, grid, p.plan.bytes, s, p, "up_gate");
+            case 2: return launch_stream(up_gate_kernel<2, true>, grid, p.plan.bytes, s, p, "up_gate");
+            case 4: return launch_stream(up_gate_kernel<4, true>, grid, p.plan.bytes, s, p, "up_gate");
+            default: return launch_stream(up_gate_kernel<8, true>, grid, p.plan.bytes, s, p, "up_gate");
+        }
+    }
     switch (nt) {
-        case 1: return launch_stream(up_gate_kernel<1>, grid, p.plan.bytes, s, p, "up_gate");
-        case 2: return launch_stream(up_gate_kernel<2>, grid, p.plan.bytes, s, p, "up_gate");
-        case 4: return launch_stream(up_gate_kernel<4>, grid, p.plan.bytes, s, p, "up_gate");
-        default: return launch_stream(up_gate_kernel<8>, grid, p.plan.bytes, s, p, "up_gate");
+        case 1: return launch_stream(up_gate_kernel<1, false>, grid, p.plan.bytes, s, p, "up_gate");
+        case 2: return launch_stream(up_gate_kernel<2, false>, grid, p.plan.bytes, s, p, "up_gate");
+        case 4: return launch_stream(up_gate_kernel<4, false>, grid, p.plan.bytes, s, p, "up_gate");
+        default: return launch_stream(up_gate_kernel<8, false>, grid, p.plan.bytes, s, p, "up_gate");
     }
 }
 

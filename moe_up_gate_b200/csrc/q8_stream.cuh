@@ -508,11 +508,66 @@ __device__ __forceinline__ void stage_q8(const XStage &xs, const int8_t *__restr
     }
 }
 
-// Quantize fp32 rows arow(j) of af (k floats apart), j < n, into the stage,
-// one warp per 32-block, by the Q8_0 rule.  Each warp first issues the loads
-// of up to 8 of its blocks, then quantizes them (one memory latency per 8
-// blocks).
+// Quantize fp32 rows arow(j) of af (16-byte aligned, k floats apart), j < n,
+// into the stage with eight threads per 32-block (thread i takes elements
+// 4i..4i+3, as in stage_f32_smem8); each thread issues the loads of kWide of
+// its blocks before it quantizes any, so a stage costs one memory latency
+// per kWide * kCT / 8 blocks (14336 floats: 2) where one warp per block
+// with 8 blocks' loads in flight pays one per 8 blocks of a warp (7).
 template <class RowFn>
+__device__ __forceinline__ void stage_f32_wide(const XStage xs, const float *__restrict__ af,
+                                               int k, int n, RowFn arow) {
+    const int nb = k / QK;
+    const int total = n * nb;
+    constexpr int kWide = 8;
+    constexpr int ngrp = kCT / 8;
+    const int grp = (int)threadIdx.x >> 3, part = (int)threadIdx.x & 7;
+    for (int base = 0; base < total; base += kWide * ngrp) {  // the same trip count in every lane
+        float4 f[kWide];
+#pragma unroll
+        for (int r = 0; r < kWide; ++r) {
+            const int blk = base + r * ngrp + grp;
+            f[r] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (blk < total) {
+                const int j = blk / nb;
+                const int b = blk - j * nb;
+                f[r] = reinterpret_cast<const float4 *>(af + (int64_t)arow(j) * k + b * QK)[part];
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < kWide; ++r) {
+            const int blk = base + r * ngrp + grp;
+            float amax = fmaxf(fmaxf(fabsf(f[r].x), fabsf(f[r].y)),
+                               fmaxf(fabsf(f[r].z), fabsf(f[r].w)));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+            if (blk < total) {
+                const int j = blk / nb;
+                const int b = blk - j * nb;
+                const float d32 = block_scale(amax);
+                const float id = block_inv_scale(d32);
+                const uint32_t w = ((uint32_t)quantize_one(f[r].x, id) & 0xffu) |
+                                   (((uint32_t)quantize_one(f[r].y, id) & 0xffu) << 8) |
+                                   (((uint32_t)quantize_one(f[r].z, id) & 0xffu) << 16) |
+                                   (((uint32_t)quantize_one(f[r].w, id) & 0xffu) << 24);
+                *reinterpret_cast<uint32_t *>(xs.q + (size_t)j * k + b * QK + 4 * part) = w;
+                if (part == 0) xs.dx[(size_t)j * nb + b] = scale_value(scale_bits(d32));
+            }
+        }
+    }
+}
+
+// Quantize fp32 rows arow(j) of af (k floats apart), j < n, into the stage
+// by the Q8_0 rule.  Aligned rows: one thread per 32-block when the blocks
+// are at most kCT, else (Wide) eight threads per block with many blocks'
+// loads in flight per thread.  Otherwise one warp per 32-block, each warp
+// first issuing the loads of up to 8 of its blocks.  amax is an exact
+// maximum and every code is formed as in quantize_block_thread, so the three
+// forms give the same bits.  Wide is for kernels that stage long or many
+// rows (dense matmuls): its loads, inlined, raise the register pressure of
+// the dot loops, which costs the routed kernels more than it saves them.
+template <bool Wide, class RowFn>
 __device__ __forceinline__ void stage_f32(const XStage &xs, const float *__restrict__ af, int k,
                                           int n, RowFn arow) {
     constexpr int kBatch = 8;
@@ -543,6 +598,12 @@ __device__ __forceinline__ void stage_f32(const XStage &xs, const float *__restr
             xs.dx[(size_t)j * nb + b] = scale_value(scale_bits(d32));
         }
         return;
+    }
+    if constexpr (Wide) {
+        if (((uintptr_t)af & 15u) == 0) {
+            stage_f32_wide(xs, af, k, n, arow);
+            return;
+        }
     }
     for (int b0 = threadIdx.x >> 5; b0 < total; b0 += kCW * kBatch) {
         float v[kBatch];
@@ -679,7 +740,7 @@ __device__ __forceinline__ void stage_f32_raw(const XStage &xs, const float *raw
 // Consumer side of an activation job of nx rows (fp32 af, rows arow(j)):
 // from the raw slot when the producer copied them, else from global memory.
 // The caller synchronizes the consumer warps afterwards.
-template <class RowFn>
+template <bool Wide = false, class RowFn>
 __device__ __forceinline__ void stage_job_f32(const Ring &R, XJobs &J, const XStage &xs,
                                               const float *af, int k, int nx, RowFn arow,
                                               int *err) {
@@ -690,7 +751,7 @@ __device__ __forceinline__ void stage_job_f32(const Ring &R, XJobs &J, const XSt
         if ((threadIdx.x & 31) == 0) mbar_arrive(R.xempty);
         ++J.n;
     } else {
-        stage_f32(xs, af, k, nx, arow);
+        stage_f32<Wide>(xs, af, k, nx, arow);
     }
 }
 
