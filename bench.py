@@ -459,6 +459,9 @@ class MoeWorkload:
         self.h = torch.empty((P, F), dtype=torch.float32, device=dev)
         self.hq = torch.empty((P, F), dtype=torch.int8, device=dev)
         self.hd = torch.empty((P, F // 32), dtype=torch.float16, device=dev)
+        # dense h rows longer than the 16 KB raw slot of the streaming
+        # kernels are quantized once before the down GEMV
+        self.h_once = not self.routed and F * 4 > 16 * 1024
         self.y = torch.empty((tokens, Uu, D), dtype=torch.float32, device=dev)
         self.out = torch.empty((self.layers, tokens, D), dtype=torch.float32, device=dev)
         self.out_host = torch.empty((self.layers, tokens, D), dtype=torch.float32).pin_memory()
@@ -469,7 +472,7 @@ class MoeWorkload:
             self.ffn_ws = q8.moe_ffn_workspace(tokens, U, E, D, F, dev)
             self.launches_per_step = self.layers
         elif self.small:
-            self.launches_per_step = self.layers * (3 if self.routed else 2)
+            self.launches_per_step = self.layers * (3 if self.routed or self.h_once else 2)
         elif self.routed:
             # quantize x, group, up/gate (dp4a + tensor cores), quantize h,
             # down (dp4a + tensor cores), combine; the timed unit is the
@@ -500,7 +503,8 @@ class MoeWorkload:
         if self.small:
             # small batches: the fp32 calls (x and h quantized inside the
             # kernels, routing grouped in every CTA), the same kernels
-            # q8_moe_ffn runs: routed 3 launches per layer, dense 2
+            # q8_moe_ffn runs: routed 3 launches per layer, dense 2 (3 when
+            # h is quantized once)
             for l, (UG, DN) in enumerate(layers):
                 x = self.x[s][l]
                 if self.routed:
@@ -514,7 +518,14 @@ class MoeWorkload:
                     marks.begin()
                     q8.moe_up_gate_swiglu_fp32(UG, x, None, h=self.h)
                     marks.end()
-                    q8.gemv_batched([(DN, self.h, self.out[l])], n_tok=T)
+                    if self.h_once:
+                        # h rows longer than a CTA's raw slot: h quantized
+                        # once, then the Q8_0 GEMV (as q8_moe_ffn does)
+                        q8._call("q8_quantize_row", q8._ptr(self.h), T, self.h.shape[1],
+                                 q8._ptr(self.hq), q8._ptr(self.hd), q8._stream())
+                        q8.gemv(DN, self.hq, self.hd, y=self.out[l])
+                    else:
+                        q8.gemv_batched([(DN, self.h, self.out[l])], n_tok=T)
             return
         for l, (UG, DN) in enumerate(layers):
             x = self.x[s][l]

@@ -348,8 +348,10 @@ q8_status q8_moe_combine(const float *y, const float *route_w, int64_t n_tok, in
  * the separate calls.  Larger routed batches run quantize + q8_moe_group +
  * q8_moe_up_gate_swiglu_pregrouped (h quantized once) +
  * q8_mul_mat_id_pregrouped + q8_moe_combine, with the same results as those
- * calls.  Dense batches of up to Q8_SMALL_BATCH_PAIRS rows run the _fp32
- * calls.
+ * calls.  Dense batches of up to Q8_SMALL_BATCH_PAIRS rows run
+ * q8_moe_up_gate_swiglu_fp32 and the down GEMV on fp32 h (n_ff <= 4096) or,
+ * for longer h rows, q8_quantize_row of h and q8_gemv (the same bits: the
+ * down kernel quantizes h by the same rule).
  */
 size_t q8_moe_ffn_workspace_size(int64_t n_tok, int32_t n_used, int64_t n_mat, int64_t n_embd,
                                  int64_t n_ff);

@@ -513,9 +513,9 @@ static FfnLayout ffn_layout(int64_t n_tok, int32_t n_used, int64_t n_mat, int64_
     L.h = o;
     o += round_up((size_t)P * n_ff * 4, 256);
     L.hq = o;
-    o += routed ? round_up((size_t)P * n_ff, 256) : 0;
+    o += round_up((size_t)P * n_ff, 256);
     L.hd = o;
-    o += routed ? round_up((size_t)P * (n_ff / QK) * 2, 256) : 0;
+    o += round_up((size_t)P * (n_ff / QK) * 2, 256);
     L.y = o;
     o += routed ? round_up((size_t)P * n_embd * 4, 256) : 0;
     L.total = o;
@@ -883,14 +883,26 @@ q8_status q8_moe_ffn(const q8_tensor *up_gate, const q8_tensor *down, const floa
     if (small) {
         // Three launches: up/gate (x quantized as it is staged; routed: the
         // grouping built in each CTA from ids), down (h quantized as it is
-        // staged), combine.
+        // staged; dense h rows longer than the raw slot: quantized once
+        // before it), combine (routed).
         int32_t *err = routed ? (int32_t *)(w8 + F.group) : nullptr;
         if (routed && layer_eligible(up_gate, down, n_tok, n_used))
             return launch_layer(up_gate, down, x, n_tok, ids, route_w, n_used, out, h,
                                 (unsigned *)(w8 + F.group) + WS_BAR, err, s);
         st = q8_moe_up_gate_swiglu_fp32(up_gate, x, n_tok, ids, n_used, h, err, s);
         if (st != Q8_OK) return st;
-        if (!routed) return launch_matmul_dense(down, nullptr, nullptr, h, n_tok, out, s);
+        if (!routed) {
+            if (4 * n_ff <= kRawSlotBytes)
+                return launch_matmul_dense(down, nullptr, nullptr, h, n_tok, out, s);
+            // h rows too long for the raw slot: every CTA of the down kernel
+            // would quantize all of h from global memory (a 14336-long row:
+            // about 7 us of each launch), so h is quantized once here
+            int8_t *hq = (int8_t *)(w8 + F.hq);
+            uint16_t *hd = (uint16_t *)(w8 + F.hd);
+            st = q8_quantize_row(h, n_tok, n_ff, hq, hd, s);
+            if (st != Q8_OK) return st;
+            return launch_matmul_dense(down, hq, hd, nullptr, n_tok, out, s);
+        }
         float *y = (float *)(w8 + F.y);
         st = q8_mul_mat_id_fp32(down, h, 1, n_tok, ids, n_used, y, nullptr, s);
         if (st != Q8_OK) return st;

@@ -98,8 +98,13 @@ def test_config3_dense_ffn_full_size(T):
     Su = S_norm(wq[F:], wd[F:], xq, xd)
     bound = _h_bound(g_ref[:, 0], u_ref[:, 0], h_ref[:, 0], Sg, Su)
     assert np.all(np.abs(h - h_ref[:, 0]) <= bound)
-    # the down projection quantizes the fp32 h as it stages it: P5 + P3
+    # the down projection takes h quantized by the Q8_0 rule (P5: bitwise the
+    # oracle's quantization of the GPU's h, checked where h is quantized once
+    # before the GEMV) and P3 on its output
     hq, hd = oracle.quantize_rows(host(wl.h).reshape(T, F))
+    if wl.h_once:
+        assert np.array_equal(host(wl.hq).reshape(T, F), hq)
+        assert np.array_equal(bits(wl.hd).reshape(T, F // 32), hd)
     dq, dd = host(DN.qs), canon_d(DN.d, F)
     y_ref = oracle.gemv(dq, dd, hq, hd)
     assert_p3(host(wl.out)[0], y_ref, S_norm(dq, dd, hq, hd), f"dense down T={T}")
