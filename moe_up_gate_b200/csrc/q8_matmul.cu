@@ -64,7 +64,9 @@ struct MatmulParams {
     Plan plan;
 };
 
-template <int NT>
+// Dense: an instantiation for dense calls (no grouping table, no ids), whose
+// activation staging takes the wide forms (stage_q8, stage_f32).
+template <int NT, bool Dense>
 __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     stream_matmul_kernel(const __grid_constant__ MatmulParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -74,8 +76,8 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
     const Geo g = geo_for_k(p.k, NT);
     const int tpm = (p.rows + g.nr - 1) / g.nr;
     griddep_launch_dependents();
-    const int32_t *tab = p.ws;
-    if (p.ids) {
+    const int32_t *tab = Dense ? nullptr : p.ws;
+    if (!Dense && p.ids) {
         griddep_wait();
         int32_t *stab = reinterpret_cast<int32_t *>(smem + p.plan.off_tab);
         GroupLayout L{};
@@ -173,9 +175,9 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                     return (!routed || p.a_per_slot) ? pr : pr / p.n_used;
                 };
                 if (p.af)
-                    stage_job_f32(R, J, xs, p.af, p.k, nx, arow, &g_err_matmul);
+                    stage_job_f32<Dense>(R, J, xs, p.af, p.k, nx, arow, &g_err_matmul);
                 else
-                    stage_q8(xs, p.aq, p.ad, p.k, nx, arow);
+                    stage_q8<Dense>(xs, p.aq, p.ad, p.k, nx, arow);
                 named_bar_sync(kBarConsumers, kCT);
                 Q8_TRACE(7);
                 staged_mi = mi;
@@ -254,11 +256,19 @@ q8_status launch_matmul(const MatmulParams &base, RowPlan rp, int64_t max_tiles,
                    tab_words, p.af != nullptr && aligned16(p.af)))
         Q8_FAIL(Q8_E_UNSUPPORTED, "matmul: k=%d does not fit the shared-memory plan", p.k);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * p.plan.ctas, max_tiles));
+    if (!p.ids && !p.ws) {
+        switch (nt) {
+            case 1: return launch_stream(stream_matmul_kernel<1, true>, grid, p.plan.bytes, s, p, "matmul");
+            case 2: return launch_stream(stream_matmul_kernel<2, true>, grid, p.plan.bytes, s, p, "matmul");
+            case 4: return launch_stream(stream_matmul_kernel<4, true>, grid, p.plan.bytes, s, p, "matmul");
+            default: return launch_stream(stream_matmul_kernel<8, true>, grid, p.plan.bytes, s, p, "matmul");
+        }
+    }
     switch (nt) {
-        case 1: return launch_stream(stream_matmul_kernel<1>, grid, p.plan.bytes, s, p, "matmul");
-        case 2: return launch_stream(stream_matmul_kernel<2>, grid, p.plan.bytes, s, p, "matmul");
-        case 4: return launch_stream(stream_matmul_kernel<4>, grid, p.plan.bytes, s, p, "matmul");
-        default: return launch_stream(stream_matmul_kernel<8>, grid, p.plan.bytes, s, p, "matmul");
+        case 1: return launch_stream(stream_matmul_kernel<1, false>, grid, p.plan.bytes, s, p, "matmul");
+        case 2: return launch_stream(stream_matmul_kernel<2, false>, grid, p.plan.bytes, s, p, "matmul");
+        case 4: return launch_stream(stream_matmul_kernel<4, false>, grid, p.plan.bytes, s, p, "matmul");
+        default: return launch_stream(stream_matmul_kernel<8, false>, grid, p.plan.bytes, s, p, "matmul");
     }
 }
 

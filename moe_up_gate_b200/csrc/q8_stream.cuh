@@ -487,13 +487,52 @@ struct XStage {
     float *dx;   // [xmax][nb]
 };
 
-// Copy Q8_0 rows arow(j) of aq/ad, j < n, into the stage.
-template <class RowFn>
+// Copy Q8_0 rows arow(j) of aq/ad, j < n, into the stage.  Wide: each
+// thread issues the loads of a whole round (up to 4 quant vectors and 4
+// scales) before its first store, one memory latency per round of 4 * kCT
+// vectors, where a loop of one load and one shared store per step pays one
+// per step (the store may alias the next load as far as the compiler
+// knows).  Wide is for dense kernels, for the register-pressure reason given
+// at stage_f32.
+template <bool Wide = false, class RowFn>
 __device__ __forceinline__ void stage_q8(const XStage &xs, const int8_t *__restrict__ aq,
                                          const uint16_t *__restrict__ ad, int k, int n,
                                          RowFn arow) {
     const int nb = k / QK;
     const int v_per_row = k / 16;
+    if constexpr (Wide) {
+        constexpr int kU = 4;
+        const int nv = n * v_per_row, nd = n * nb;
+        const int tid = (int)threadIdx.x;
+        for (int base = 0; base < nv || base < nd; base += kU * kCT) {
+            uint4 v[kU];
+            uint16_t d[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int i = base + u * kCT + tid;
+                if (i < nv) {
+                    const int j = i / v_per_row;
+                    const int c = i - j * v_per_row;
+                    v[u] = *reinterpret_cast<const uint4 *>(aq + (int64_t)arow(j) * k + c * 16);
+                }
+                if (i < nd) {
+                    const int j = i / nb;
+                    d[u] = ad[(int64_t)arow(j) * nb + (i - j * nb)];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int i = base + u * kCT + tid;
+                if (i < nv) {
+                    const int j = i / v_per_row;
+                    const int c = i - j * v_per_row;
+                    *reinterpret_cast<uint4 *>(xs.q + (size_t)j * k + c * 16) = v[u];
+                }
+                if (i < nd) xs.dx[i] = scale_value(d[u]);  // row j = i / nb, block i - j * nb
+            }
+        }
+        return;
+    }
 #pragma unroll 4
     for (int i = threadIdx.x; i < n * v_per_row; i += kCT) {
         const int j = i / v_per_row;
