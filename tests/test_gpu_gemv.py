@@ -72,6 +72,35 @@ def test_gemv_batched_matches_quantize_then_gemv():
         assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
 
 
+@pytest.mark.parametrize("n_tok", [1, 3])
+def test_gemv_batched_long_rows(n_tok):
+    """Rows too long for the raw slot (k > 4096): every CTA quantizes the
+    fp32 activations from global memory with eight threads per block; the
+    short problem of the same launch then stages that way too.  P3 against
+    the oracle and the same bits as quantize + q8_gemv."""
+    shapes = [(300, 14336), (70, 8192), (768, 768)]
+    probs, refs = [], []
+    for i, (rows, k) in enumerate(shapes):
+        w = synth.normal((rows, k), seed=700 + i, std=0.02)
+        x = synth.normal((n_tok, k), seed=800 + i)
+        W = q8.pack(w.to(DEV))
+        y = torch.full((n_tok, rows), float("nan"), device=DEV)
+        probs.append((W, x.to(DEV), y))
+        refs.append((W, x))
+    q8.gemv_batched(probs, n_tok=n_tok)
+    torch.cuda.synchronize()
+    for (W, x), (_, xdev, y) in zip(refs, probs):
+        rq, rd = oracle.quantize_rows(x.numpy())
+        wq = host(W.qs)
+        wd = canon_d(W.d, W.k)
+        ref = oracle.gemv(wq, wd, rq, rd)
+        assert_p3(host(y), ref, S_norm(wq, wd, rq, rd), f"gemv_batched k={W.k}")
+        xq, xd = q8.quantize_row(xdev)
+        assert np.array_equal(host(xq), rq) and np.array_equal(bits(xd), rd)
+        y2 = q8.gemv(W, xq, xd)
+        assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
+
+
 def test_gemv_on_row_view():
     """A row view (offset rows of one matrix) reads exactly those rows."""
     w, x, W, xq, xd = _case(96, 128, 1, seed=77)
