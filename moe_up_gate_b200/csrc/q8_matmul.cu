@@ -29,6 +29,42 @@ q8_status clear_wait_errors_matmul() {
     return e == cudaSuccess ? Q8_OK : Q8_E_CUDA;
 }
 
+// Consumer side of a dense Q8_0 activation set that the producer copied with
+// the CTA's first tile (q8_copy_job): the quants straight into the stage,
+// the fp16 scales into the upper half of the fp32 scale area, widened here
+// in place.  Chunks of 2 * kCT scales: every thread reads its two, a
+// barrier, then writes them; a write of scale i overwrites fp16 scales
+// 2i - nd and 2i - nd + 1, which are below the chunk's end and so already
+// read (all nd of them when the chunk is the last).
+__device__ __forceinline__ void stage_q8_landed(const XStage &xs, int k, int n, const Ring &R,
+                                                int *err) {
+    mbar_wait(R.xfull, 0, err);
+    const int nd = n * (k / QK);
+    const uint16_t *h16 = reinterpret_cast<const uint16_t *>(xs.dx) + nd;
+    const int tid = (int)threadIdx.x;
+    for (int base = 0; base < nd; base += 2 * kCT) {  // the same trip count in every thread
+        const int i0 = base + tid, i1 = base + kCT + tid;
+        const uint16_t a = i0 < nd ? h16[i0] : (uint16_t)0;
+        const uint16_t b = i1 < nd ? h16[i1] : (uint16_t)0;
+        named_bar_sync(kBarConsumers, kCT);
+        if (i0 < nd) xs.dx[i0] = scale_value(a);
+        if (i1 < nd) xs.dx[i1] = scale_value(b);
+    }
+}
+
+// Producer side: n dense Q8_0 rows (quants aq, scales ad, both contiguous
+// and 16-byte aligned, n * k / 16 and n * (k / 32) / 8 whole) in two bulk
+// copies on R.xfull.
+__device__ __forceinline__ void q8_copy_job(const Ring &R, const Plan &pl, const int8_t *aq,
+                                            const uint16_t *ad, int k, int n) {
+    const uint32_t qbytes = (uint32_t)n * (uint32_t)k;
+    const uint32_t dbytes = (uint32_t)n * (uint32_t)(k / QK) * 2u;
+    unsigned char *base = reinterpret_cast<unsigned char *>(R.xfull) - pl.off_xfull;
+    mbar_arrive_expect_tx(R.xfull, qbytes + dbytes);
+    bulk_g2s_keep(base + pl.off_xq, aq, qbytes, R.xfull);
+    bulk_g2s_keep(base + pl.off_xd + dbytes, ad, dbytes, R.xfull);
+}
+
 // ---------------------------------------------------------------------------
 // matmul over the activation rows of each matrix.
 //   dense  (ws == nullptr): matrix 0; activation rows 0..n_dense-1; output
@@ -61,6 +97,9 @@ struct MatmulParams {
     int n_tok;
     int n_mat;
     int32_t *err_out;
+    // dense Q8_0 activations that the producer copies into the stage with
+    // the first tile (all rows in one group, contiguous, 16-byte aligned)
+    int q8_copy;
     Plan plan;
 };
 
@@ -134,6 +173,21 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                     }
                 };
                 produce(R, tb, te, src, &g_err_matmul, jobs, !routed);
+            } else if constexpr (Dense) {
+                if (p.q8_copy) {
+                    // the rows may come from the preceding grid: the first
+                    // tile goes out before the wait, the rows right after
+                    // it, ahead of the rest of the stream
+                    bool copied = false;
+                    auto qjob = [&](int64_t, int when) {
+                        if (when != 0 || copied) return;
+                        q8_copy_job(R, p.plan, p.aq, p.ad, p.k, p.n_dense);
+                        copied = true;
+                    };
+                    produce(R, tb, te, src, &g_err_matmul, qjob, true);
+                } else {
+                    produce(R, tb, te, src, &g_err_matmul);
+                }
             } else {
                 produce(R, tb, te, src, &g_err_matmul);
             }
@@ -174,10 +228,16 @@ __global__ void __launch_bounds__(kThreadsStream, ctas_per_sm(NT))
                     const int pr = plist ? plist[x0 + j] : x0 + j;
                     return (!routed || p.a_per_slot) ? pr : pr / p.n_used;
                 };
-                if (p.af)
+                if (p.af) {
                     stage_job_f32<Dense>(R, J, xs, p.af, p.k, nx, arow, &g_err_matmul);
-                else
+                } else if constexpr (Dense) {
+                    if (p.q8_copy)
+                        stage_q8_landed(xs, p.k, nx, R, &g_err_matmul);
+                    else
+                        stage_q8<Dense>(xs, p.aq, p.ad, p.k, nx, arow);
+                } else {
                     stage_q8<Dense>(xs, p.aq, p.ad, p.k, nx, arow);
+                }
                 named_bar_sync(kBarConsumers, kCT);
                 Q8_TRACE(7);
                 staged_mi = mi;
@@ -256,6 +316,10 @@ q8_status launch_matmul(const MatmulParams &base, RowPlan rp, int64_t max_tiles,
                    tab_words, p.af != nullptr && aligned16(p.af)))
         Q8_FAIL(Q8_E_UNSUPPORTED, "matmul: k=%d does not fit the shared-memory plan", p.k);
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms() * p.plan.ctas, max_tiles));
+    const int64_t nd = (int64_t)p.n_dense * (p.k / QK);
+    p.q8_copy = !p.ids && !p.ws && p.aq && p.ad && aligned16(p.aq) && aligned16(p.ad) &&
+                p.n_dense >= 1 && p.n_dense <= p.plan.xmax && p.k <= p.plan.max_nb * QK &&
+                nd % 8 == 0;
     if (!p.ids && !p.ws) {
         switch (nt) {
             case 1: return launch_stream(stream_matmul_kernel<1, true>, grid, p.plan.bytes, s, p, "matmul");
