@@ -333,7 +333,9 @@ ORACLE_TOKENS = 16
 class MoeWorkload:
     """MoE (or dense) feed-forward layers through the public calls:
     quantize x -> group -> fused up/gate + SwiGLU (+ h quantization) -> down
-    mul_mat_id -> combine (dense: quantize -> up/gate -> down GEMV).
+    mul_mat_id -> combine (dense: quantize -> up/gate -> down GEMV; small
+    dense batches: fp32 up/gate -> down GEMV on fp32 h, or, for h rows
+    longer than the raw slot, h quantized once and the int8 down GEMV)
 
     layer_ids: the layers to build (default all; a parity test builds a few
     of them, with the same seeds and the same calls).  packed: the packed
